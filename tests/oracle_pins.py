@@ -1,0 +1,444 @@
+"""Pins for the fp64 oracle: checks against what the pages and the mathematics fix.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with a value
+printed on a page (golden fixtures under tests/golden/), a closed form, an invariant,
+or a brute-force evaluation written independently here in pure Python.  They are
+collected by ``test_oracle_pins.py`` and re-run against deliberately broken builds of
+the oracle by ``test_oracle_mutants.py`` (every planted mistake must trip at least one).
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+
+import oracle
+from seeded_inputs import normal_f32
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+EXACT = 1e-12
+
+
+def load_golden(name: str) -> dict:
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, val = line.split(":", 1)
+            out[key.strip()] = np.array([float(x) for x in val.split(",")], dtype=np.float64)
+    return out
+
+
+def _close(a, b, tol, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    err = np.max(np.abs(a - b)) if a.size else 0.0
+    assert err <= tol, f"{what}: max abs error {err:.3e} > {tol:.1e}"
+
+
+# ------------------------------------------------------------------------------------------
+# Independent brute force (pure Python, log-domain, different algebra from the oracle)
+# ------------------------------------------------------------------------------------------
+
+def _exp(x: float) -> float:
+    return math.exp(x) if x < 709.0 else math.inf
+
+
+def brute_attention(q, k, v, scale, causal, rope_base=0.0, q_pos0=0):
+    """Exact attention evaluated as weights w_j = 1 / sum_k exp(s_k - s_j) over the visible
+    keys, with LSE = s_j + ln(sum_k exp(s_k - s_j)) for any visible j.  Pure Python floats.
+    RoPE here rotates complex numbers z = x_{2i} + i x_{2i+1} by e^{i theta}."""
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    g = Hq // Hkv
+    o = np.zeros((B, Sq, Hq, D))
+    lse = np.zeros((B, Hq, Sq))
+
+    def rot(vec, pos):
+        if rope_base <= 0:
+            return [float(x) for x in vec]
+        out = []
+        for i in range(D // 2):
+            th = pos * rope_base ** (-(2.0 * i) / D)
+            z = complex(float(vec[2 * i]), float(vec[2 * i + 1])) * complex(math.cos(th), math.sin(th))
+            out += [z.real, z.imag]
+        return out
+
+    for b in range(B):
+        for h in range(Hq):
+            kh = h // g
+            keys = [rot(k[b, j, kh], j) for j in range(Skv)]
+            for i in range(Sq):
+                qi = rot(q[b, i, h], q_pos0 + i)
+                vis = [j for j in range(Skv) if not (causal and j > i + (Skv - Sq))]
+                if not vis:
+                    lse[b, h, i] = -math.inf
+                    continue
+                s = {j: scale * math.fsum(qi[d] * keys[j][d] for d in range(D)) for j in vis}
+                j0 = max(vis, key=lambda j: s[j])
+                lse[b, h, i] = s[j0] + math.log(math.fsum(_exp(s[kk] - s[j0]) for kk in vis))
+                for d in range(D):
+                    o[b, i, h, d] = math.fsum(
+                        float(v[b, j, kh, d]) / math.fsum(_exp(s[kk] - s[j]) for kk in vis)
+                        for j in vis)
+    return o, lse
+
+
+# ------------------------------------------------------------------------------------------
+# Golden fixtures from the pages
+# ------------------------------------------------------------------------------------------
+
+def pin_golden_sdpa_basic():
+    g = load_golden("p3_sdpa_basic.txt")
+    q = g["q"].reshape(1, 2, 1, 4)
+    k = g["k"].reshape(1, 2, 1, 4)
+    v = g["v"].reshape(1, 2, 1, 4)
+    o, lse = oracle.attn_fwd(q, k, v, float(g["scale"][0]), causal=False)
+    _close(o.reshape(-1), g["expected_o"], 1e-6, "P3 basic O (fixture, 7 decimals)")
+    _close(lse.reshape(-1), g["expected_lse"], 1e-6, "P3 basic LSE (fixture)")
+    # the same values from the closed form sigma(1/2)
+    s = 1.0 / (1.0 + math.exp(-0.5))
+    o0 = [s * a + (1 - s) * b for a, b in zip((1, 2, 3, 4), (5, 6, 7, 8))]
+    o1 = [(1 - s) * a + s * b for a, b in zip((1, 2, 3, 4), (5, 6, 7, 8))]
+    _close(o.reshape(2, 4), np.array([o0, o1]), EXACT, "P3 basic O (closed form)")
+    _close(lse.reshape(-1), [math.log1p(math.exp(0.5))] * 2, EXACT, "P3 basic LSE (closed form)")
+
+
+def pin_golden_causal_first_row():
+    g = load_golden("p3_flash_attention_causal_first_row.txt")
+    q = g["q"].reshape(1, 2, 1, 4)
+    k = g["k"].reshape(1, 2, 1, 4)
+    v = g["v"].reshape(1, 2, 1, 4)
+    o, lse = oracle.attn_fwd(q, k, v, float(g["scale"][0]), causal=True)
+    _close(o[0, 0, 0], g["expected_o_row0"], EXACT, "P3 causal row 0")
+    # row 0 has one visible key: LSE = its score = 0.5 * (q0 . k0) = 0.5
+    _close(lse[0, 0, 0], 0.5, EXACT, "P3 causal row 0 LSE")
+    # row 1 sees both keys with equal scores: mean of v0, v1; LSE = 0.5 + ln 2
+    _close(o[0, 1, 0], 0.5 * (g["v"][:4] + g["v"][4:]), EXACT, "P3 causal row 1")
+    _close(lse[0, 0, 1], 0.5 + math.log(2.0), EXACT, "P3 causal row 1 LSE")
+
+
+def _decode_case(g):
+    D = int(g["head_dim"][0])
+    L = int(g["seq_len"][0])
+    q = g["q"].reshape(1, 1, D)
+    k = g["k"].reshape(1, L, 1, D)
+    v = g["v"].reshape(1, L, 1, D)
+    return q, k, v, np.array([L], dtype=np.int32), float(g["scale"][0])
+
+
+def pin_golden_decode_single_token():
+    g = load_golden("p4_flash_decode_single_token.txt")
+    q, k, v, sl, scale = _decode_case(g)
+    for o, lse in (oracle.decode(q, k, v, sl, scale), oracle.decode_split(q, k, v, sl, scale, 4)):
+        _close(o.reshape(-1), g["expected_o"], EXACT, "P4 single token")
+        _close(lse.reshape(-1), [scale * 0.5], EXACT, "P4 single token LSE = its score")
+
+
+def pin_golden_decode_uniform_keys():
+    g = load_golden("p4_flash_decode_uniform_keys.txt")
+    q, k, v, sl, scale = _decode_case(g)
+    s = scale * 4 * float(np.float32(0.1)) ** 2      # every score equal
+    for nt in (1, 2, 3, 4, 7):
+        o, lse = oracle.decode_split(q, k, v, sl, scale, nt)
+        _close(o.reshape(-1), g["expected_o"], EXACT, f"P4 uniform keys, {nt} tiles")
+        _close(lse.reshape(-1), [s + math.log(4.0)], EXACT, "P4 uniform keys LSE = s + ln n")
+    o, lse = oracle.decode(q, k, v, sl, scale)
+    _close(o.reshape(-1), g["expected_o"], EXACT, "P4 uniform keys, unsplit")
+
+
+def pin_golden_rope_position_zero():
+    g = load_golden("p2_rope_position_zero.txt")
+    D, T, H = int(g["head_dim"][0]), int(g["seq_len"][0]), int(g["num_heads"][0])
+    x = np.ones((T, H, D), dtype=np.float32)
+    y = oracle.rope(x, np.arange(T), float(g["base"][0]))
+    _close(y[0, 0], g["expected_pos0"], 1e-10, "P2 RoPE position 0 is the identity")
+    assert np.max(np.abs(y[1, 0] - y[0, 0])) > 1e-10, "P2: position 1 must differ from position 0"
+
+
+# ------------------------------------------------------------------------------------------
+# Closed forms and invariants
+# ------------------------------------------------------------------------------------------
+
+def pin_softmax_rows_sum_to_one():
+    # V = identity basis (Skv == D): O row i is the probability row p_i itself.
+    D = 8
+    q = normal_f32(7, 0, (1, 5, 2, D))
+    k = normal_f32(7, 1, (1, D, 2, D))
+    v = np.tile(np.eye(D, dtype=np.float32)[None, :, None, :], (1, 1, 2, 1))
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, 0.3, causal)
+        p = o.transpose(0, 2, 1, 3)                      # [B,H,Sq,Skv]
+        _close(p.sum(-1), np.ones(p.shape[:-1]), EXACT, "rows of P sum to 1")
+        assert (p >= 0).all()
+        # ratios p_ij / p_ik = exp(s_ij - s_ik) computed here independently
+        for h in range(2):
+            for i in range(5):
+                vis = [j for j in range(D) if not (causal and j > i + D - 5)]
+                s = [0.3 * math.fsum(float(q[0, i, h, d]) * float(k[0, j, h, d]) for d in range(D))
+                     for j in range(D)]
+                for j in vis:
+                    _close(p[0, h, i, j] / p[0, h, i, vis[0]], math.exp(s[j] - s[vis[0]]), 1e-10,
+                           "p ratio")
+                for j in range(D):
+                    if j not in vis:
+                        assert p[0, h, i, j] == 0.0, "masked key must get zero weight"
+    # V all ones: O = 1 exactly (up to rounding)
+    o, _ = oracle.attn_fwd(q, k, np.ones_like(k), 1.7, True)
+    _close(o, np.ones_like(o), EXACT, "V = 1 gives O = 1")
+
+
+def pin_single_key():
+    q = normal_f32(11, 0, (2, 3, 4, 6))
+    k = normal_f32(11, 1, (2, 1, 2, 6))
+    v = normal_f32(11, 2, (2, 1, 2, 6))
+    o, lse = oracle.attn_fwd(q, k, v, 0.7, causal=False)
+    for b in range(2):
+        for i in range(3):
+            for h in range(4):
+                _close(o[b, i, h], v[b, 0, h // 2], EXACT, "single key returns V")
+                s = 0.7 * math.fsum(float(q[b, i, h, d]) * float(k[b, 0, h // 2, d]) for d in range(6))
+                _close(lse[b, h, i], s, EXACT, "single key LSE = its score")
+
+
+def pin_equal_scores_mean_of_v():
+    # identical keys: every score equal, O = mean of visible V rows, LSE = s + ln n
+    D, S = 5, 6
+    q = normal_f32(13, 0, (1, S, 1, D))
+    k = np.tile(normal_f32(13, 1, (1, 1, 1, D)), (1, S, 1, 1))
+    v = normal_f32(13, 2, (1, S, 1, D))
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, 0.4, causal)
+        for i in range(S):
+            n = i + 1 if causal else S
+            _close(o[0, i, 0], v[0, :n, 0].astype(np.float64).mean(0), EXACT, "mean of V")
+            s = 0.4 * math.fsum(float(q[0, i, 0, d]) * float(k[0, 0, 0, d]) for d in range(D))
+            _close(lse[0, 0, i], s + math.log(n), EXACT, "LSE = s + ln n")
+
+
+def pin_scale_two_keys():
+    # two keys whose dot products with q differ by exactly 2: p0 = sigmoid(2 * scale)
+    q = np.array([1, 0, 0, 0], dtype=np.float32).reshape(1, 1, 1, 4)
+    k = np.array([[2, 0, 0, 0], [0, 3, 0, 0]], dtype=np.float32).reshape(1, 2, 1, 4)
+    v = np.array([[1, 0, 0, 0], [0, 1, 0, 0]], dtype=np.float32).reshape(1, 2, 1, 4)
+    for scale in (0.125, 0.5, 1.0, 3.0):
+        o, lse = oracle.attn_fwd(q, k, v, scale, False)
+        p0 = 1.0 / (1.0 + math.exp(-2.0 * scale))
+        _close(o.reshape(-1), [p0, 1 - p0, 0, 0], EXACT, f"scale {scale}")
+        _close(lse.reshape(-1), [2 * scale + math.log1p(math.exp(-2 * scale))], EXACT, "LSE")
+
+
+def pin_large_scores_stable():
+    # scores of order 1e3: no overflow, rows still sum to 1 (whisper-apr softmax stability test)
+    q = (normal_f32(17, 0, (1, 4, 1, 8)) * 40).astype(np.float32)
+    k = (normal_f32(17, 1, (1, 9, 1, 8)) * 40).astype(np.float32)
+    v = np.ones((1, 9, 1, 8), dtype=np.float32)
+    o, lse = oracle.attn_fwd(q, k, v, 1.0, False)
+    assert np.isfinite(o).all() and np.isfinite(lse).all()
+    _close(o, np.ones_like(o), EXACT, "large scores: O = 1 for V = 1")
+    ob, lb = brute_attention(q, k, v, 1.0, False)
+    _close(lse, lb, 1e-9, "large-score LSE vs brute force")
+
+
+def pin_brute_force_tiny():
+    cases = [
+        # B, Sq, Skv, Hq, Hkv, D, causal, scale
+        (1, 3, 3, 1, 1, 4, False, 0.5),
+        (2, 4, 4, 2, 2, 3, True, 0.8),
+        (1, 2, 5, 4, 2, 6, True, 0.35),     # Sq < Skv: bottom-right causal
+        (1, 5, 3, 3, 1, 2, True, 1.1),      # Sq > Skv: first rows fully masked
+        (2, 3, 4, 4, 1, 5, False, 0.2),     # MQA
+        (1, 4, 4, 2, 1, 4, True, 0.9),
+    ]
+    for n, (B, Sq, Skv, Hq, Hkv, D, causal, scale) in enumerate(cases):
+        q = normal_f32(100 + n, 0, (B, Sq, Hq, D))
+        k = normal_f32(100 + n, 1, (B, Skv, Hkv, D))
+        v = normal_f32(100 + n, 2, (B, Skv, Hkv, D))
+        o, lse = oracle.attn_fwd(q, k, v, scale, causal)
+        ob, lb = brute_attention(q, k, v, scale, causal)
+        _close(o, ob, 1e-12, f"brute force O case {n}")
+        fin = np.isfinite(lb)
+        assert (np.isfinite(lse) == fin).all(), f"case {n}: masked rows"
+        _close(lse[fin], lb[fin], 1e-12, f"brute force LSE case {n}")
+
+
+def pin_brute_force_rope():
+    for n, (Sq, Skv, D, base, p0) in enumerate([(3, 3, 4, 10000.0, 0), (2, 4, 6, 500.0, 2),
+                                                (4, 4, 8, 10.0, 0)]):
+        q = normal_f32(200 + n, 0, (1, Sq, 2, D))
+        k = normal_f32(200 + n, 1, (1, Skv, 1, D))
+        v = normal_f32(200 + n, 2, (1, Skv, 1, D))
+        o, lse = oracle.attn_fwd(q, k, v, 0.6, True, rope_base=base, q_pos0=p0)
+        ob, lb = brute_attention(q, k, v, 0.6, True, rope_base=base, q_pos0=p0)
+        _close(o, ob, 1e-12, f"RoPE brute force O case {n}")
+        fin = np.isfinite(lb)
+        _close(lse[fin], lb[fin], 1e-12, f"RoPE brute force LSE case {n}")
+
+
+def pin_fully_masked_rows():
+    # Sq > Skv with causal bottom-right alignment: rows i < Sq - Skv see no key.
+    q = normal_f32(19, 0, (1, 6, 1, 4))
+    k = normal_f32(19, 1, (1, 2, 1, 4))
+    v = normal_f32(19, 2, (1, 2, 1, 4))
+    o, lse = oracle.attn_fwd(q, k, v, 0.5, True)
+    for i in range(4):
+        assert (o[0, i, 0] == 0.0).all(), "fully masked row -> O = 0"
+        assert lse[0, 0, i] == -math.inf, "fully masked row -> LSE = -inf"
+    _close(o[0, 4, 0], v[0, 0, 0], EXACT, "row Sq-Skv sees exactly key 0")
+    on, ln = oracle.attn_fwd(q, k, v, 0.5, False)
+    _close(o[0, 5, 0], on[0, 5, 0], EXACT, "last row sees every key")
+
+
+def pin_causal_alignment():
+    # Sq == Skv: causal row i equals non-causal attention over keys 0..i;
+    # Sq < Skv: the last query row sees every key (bottom-right).
+    q = normal_f32(23, 0, (1, 5, 1, 4))
+    k = normal_f32(23, 1, (1, 5, 1, 4))
+    v = normal_f32(23, 2, (1, 5, 1, 4))
+    o, lse = oracle.attn_fwd(q, k, v, 0.9, True)
+    for i in range(5):
+        oi, li = oracle.attn_fwd(q[:, i:i + 1], k[:, :i + 1], v[:, :i + 1], 0.9, False)
+        _close(o[0, i, 0], oi[0, 0, 0], EXACT, f"causal row {i} = prefix attention")
+        _close(lse[0, 0, i], li[0, 0, 0], EXACT, "causal LSE")
+    o2, _ = oracle.attn_fwd(q[:, 3:], k, v, 0.9, True)     # Sq=2, Skv=5
+    _close(o2[0, 0, 0], o[0, 3, 0], EXACT, "bottom-right: chunk row 0 = full row 3")
+    _close(o2[0, 1, 0], o[0, 4, 0], EXACT, "bottom-right: chunk row 1 = full row 4")
+
+
+def pin_gqa_equals_repeated_mha():
+    B, S, Hq, Hkv, D = 2, 7, 6, 2, 5
+    q = normal_f32(29, 0, (B, S, Hq, D))
+    k = normal_f32(29, 1, (B, S, Hkv, D))
+    v = normal_f32(29, 2, (B, S, Hkv, D))
+    g = Hq // Hkv
+    kr = np.repeat(k, g, axis=2)
+    vr = np.repeat(v, g, axis=2)
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, 0.45, causal)
+        om, lm = oracle.attn_fwd(q, kr, vr, 0.45, causal)
+        _close(o, om, EXACT, "GQA == MHA with repeated KV heads")
+        _close(lse, lm, EXACT, "GQA LSE")
+    # MQA: Hkv = 1, each q head equals a single-head problem
+    o, lse = oracle.attn_fwd(q, k[:, :, :1], v[:, :, :1], 0.45, True)
+    for h in range(Hq):
+        oh, lh = oracle.attn_fwd(q[:, :, h:h + 1], k[:, :, :1], v[:, :, :1], 0.45, True)
+        _close(o[:, :, h], oh[:, :, 0], EXACT, "MQA head")
+
+
+def pin_tiled_equals_three_pass():
+    # the online-softmax recurrence (any block sizes) reaches the three-pass definition
+    B, Sq, Skv, Hq, Hkv, D = 1, 37, 45, 4, 2, 8
+    q = normal_f32(31, 0, (B, Sq, Hq, D), 2.5)
+    k = normal_f32(31, 1, (B, Skv, Hkv, D), 2.5)
+    v = normal_f32(31, 2, (B, Skv, Hkv, D))
+    for causal in (False, True):
+        o, lse = oracle.attn_fwd(q, k, v, 0.7, causal)
+        for bq, bkv in ((1, 1), (4, 8), (16, 16), (64, 5), (37, 45)):
+            ot, lt = oracle.attn_fwd_tiled(q, k, v, 0.7, causal, bq, bkv)
+            _close(ot, o, EXACT, f"tiled O ({bq},{bkv}) causal={causal}")
+            _close(lt, lse, EXACT, f"tiled LSE ({bq},{bkv})")
+    # with fully masked rows (Sq > Skv)
+    o, lse = oracle.attn_fwd(q, k[:, :20], v[:, :20], 0.7, True)
+    ot, lt = oracle.attn_fwd_tiled(q, k[:, :20], v[:, :20], 0.7, True, 8, 8)
+    _close(ot, o, EXACT, "tiled O, masked rows")
+    assert (np.isneginf(lt) == np.isneginf(lse)).all()
+
+
+def pin_decode_split_equals_unsplit():
+    B, Hq, Hkv, Smax, D = 3, 4, 2, 40, 6
+    q = normal_f32(37, 0, (B, Hq, D), 2.0)
+    kc = normal_f32(37, 1, (B, Smax, Hkv, D), 2.0)
+    vc = normal_f32(37, 2, (B, Smax, Hkv, D))
+    sl = np.array([1, 17, 40], dtype=np.int32)
+    o, lse = oracle.decode(q, kc, vc, sl, 0.5)
+    for nt in (1, 2, 3, 5, 16, 40, 64):
+        os_, ls = oracle.decode_split(q, kc, vc, sl, 0.5, nt)
+        _close(os_, o, EXACT, f"split decode, {nt} tiles")
+        _close(ls, lse, EXACT, f"split decode LSE, {nt} tiles")
+    # decode == the last row of a causal prefill over the cache (cached decode == full forward)
+    for b in range(B):
+        L = int(sl[b])
+        qf = np.zeros((1, L, Hq, D), dtype=np.float32)
+        qf[0, L - 1] = q[b]
+        of, lf = oracle.attn_fwd(qf, kc[b:b + 1, :L], vc[b:b + 1, :L], 0.5, True)
+        _close(of[0, L - 1], o[b], EXACT, "decode == last causal row")
+        _close(lf[0, :, L - 1], lse[b], EXACT, "decode LSE == last causal row")
+
+
+def pin_rope_rotation():
+    # D = 2: the single pair rotates by exactly pos radians, counter-clockwise
+    for pos in (1, 2, 5, -3):
+        y = oracle.rope(np.array([[[1.0, 0.0]], [[0.0, 1.0]]], dtype=np.float32), [pos, pos], 123.0)
+        _close(y[0, 0], [math.cos(pos), math.sin(pos)], EXACT, "e0 -> (cos, sin)")
+        _close(y[1, 0], [-math.sin(pos), math.cos(pos)], EXACT, "e1 -> (-sin, cos)")
+    # D = 4, base 10^4: pair 1 has frequency 10^4^(-2/4) = 1/100; at pos 100 the angle is 1
+    y = oracle.rope(np.array([[[0, 0, 1, 0]]], dtype=np.float32), [100], 10000.0)
+    _close(y[0, 0], [0, 0, math.cos(1.0), math.sin(1.0)], EXACT, "pair frequency base^(-2i/D)")
+    y = oracle.rope(np.array([[[1, 0, 0, 0]]], dtype=np.float32), [100], 10000.0)
+    _close(y[0, 0], [math.cos(100.0), math.sin(100.0), 0, 0], EXACT, "pair 0 frequency 1")
+
+
+def pin_rope_invariants():
+    T, H, D = 9, 3, 16
+    x = normal_f32(41, 0, (T, H, D))
+    pos = np.array([0, 1, 2, 7, 100, 511, 4095, 30000, -5], dtype=np.int32)
+    y = oracle.rope(x, pos, 10000.0)
+    _close(np.linalg.norm(y, axis=-1), np.linalg.norm(x.astype(np.float64), axis=-1), 1e-12,
+           "norm preserved")
+    # inverse: rotating the rotated vector by -pos returns x (RoPE inverse = negated angle)
+    back = oracle.rope(y.astype(np.float32), -pos, 10000.0)
+    _close(back, x, 2e-6, "R(-p) R(p) = I (up to the float32 re-rounding of y)")
+    # relative position: <R(m) a, R(n) b> depends only on n - m
+    a = normal_f32(43, 0, (1, 1, D))
+    b = normal_f32(43, 1, (1, 1, D))
+    dots = []
+    for m in (0, 3, 50, 1000):
+        ra = oracle.rope(a, [m], 10000.0)[0, 0]
+        rb = oracle.rope(b, [m + 17], 10000.0)[0, 0]
+        dots.append(float(np.dot(ra, rb)))
+    _close(dots, [dots[0]] * len(dots), 1e-10, "q.k after RoPE depends only on the offset")
+    # different offsets give different results (scirs2-neural test_rope_position_offset)
+    x1 = np.full((4, 1, 4), 0.5, dtype=np.float32)
+    assert np.max(np.abs(oracle.rope(x1, np.arange(4), 1e4) - oracle.rope(x1, np.arange(2, 6), 1e4))) > 1e-10
+
+
+def pin_error_paths():
+    q = np.zeros((1, 2, 3, 4), dtype=np.float32)
+    k = np.zeros((1, 2, 2, 4), dtype=np.float32)
+    try:
+        oracle.attn_fwd(q, k, k, 1.0, False)       # Hq = 3 not a multiple of Hkv = 2
+        raise AssertionError("Hq % Hkv != 0 must be rejected")
+    except oracle.OracleError:
+        pass
+    try:
+        oracle.rope(np.zeros((1, 1, 7), dtype=np.float32), [0], 1e4)   # odd head dim
+        raise AssertionError("odd RoPE head dim must be rejected")
+    except oracle.OracleError:
+        pass
+    try:
+        oracle.attn_fwd(q[:, :, :2], np.zeros((1, 0, 2, 4), np.float32),
+                        np.zeros((1, 0, 2, 4), np.float32), 1.0, False)
+        raise AssertionError("empty KV must be rejected")
+    except oracle.OracleError:
+        pass
+
+
+def pin_sampled_rows_match_full():
+    B, Sq, Hq, Hkv, D = 2, 9, 4, 2, 6
+    q = normal_f32(47, 0, (B, Sq, Hq, D))
+    k = normal_f32(47, 1, (B, Sq, Hkv, D))
+    v = normal_f32(47, 2, (B, Sq, Hkv, D))
+    o, lse = oracle.attn_fwd(q, k, v, 0.3, True, rope_base=100.0, q_pos0=0)
+    rows = np.array([0, 5, 17, 40, 71, 3, 8], dtype=np.int64)   # (b*Hq + h)*Sq + i
+    os_, ls = oracle.attn_fwd(q, k, v, 0.3, True, rope_base=100.0, q_pos0=0, rows=rows)
+    for r, row in enumerate(rows):
+        b, h, i = row // (Hq * Sq), (row // Sq) % Hq, row % Sq
+        _close(os_[r], o[b, i, h], 0.0, "sampled row")
+        _close(ls[r], lse[b, h, i], 0.0, "sampled LSE")
+
+
+ALL_PINS = [obj for name, obj in sorted(globals().items()) if name.startswith("pin_")]

@@ -1,0 +1,62 @@
+"""Every plausible mistake planted in a copy of the oracle's C source must fail at least
+one pin (CPU only).  The copy is compiled into a temporary library; the real oracle
+source is never modified."""
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")
+
+# (name, original text, planted text) -- each original must occur in the source.
+# Dropping the tiled recurrence's "running max is -inf" guard is not listed: with prefix
+# (causal) visibility a row meets an all-masked key block before a visible one only when it
+# has no visible key at all, and then the final "l > 0" test already yields O = 0, LSE = -inf,
+# so that mutant computes the same function.
+MUTANTS = [
+    ("rope_sign", "x[2 * i] = x0 * c - x1 * s;", "x[2 * i] = x0 * c + x1 * s;"),
+    ("rope_frequency", "pow(base, 2.0 * (double)i / (double)D)", "pow(base, (double)i / (double)D)"),
+    ("rope_q_offset", "(double)q_pos0 + (double)i", "(double)i"),
+    ("rope_on_values", "gather_head(v, b, kvh, Skv, Hkv, D, 0.0, Vd);",
+     "gather_head(v, b, kvh, Skv, Hkv, D, rope_base, Vd);"),
+    ("drop_scale", "s[j] = scale * dot;", "s[j] = dot;"),
+    ("causal_off_by_one", "(long)(Skv - Sq) + 1;", "(long)(Skv - Sq);"),
+    ("causal_top_left", "long n = (long)i + (long)(Skv - Sq) + 1;", "long n = (long)i + 1;"),
+    ("lse_without_max", "*lse = m + log(l);", "*lse = log(l);"),
+    ("no_normalisation", "double p = exp(s[j] - m) / l;", "double p = exp(s[j] - m);"),
+    ("values_from_keys", "o[d] += p * V[(long)j * D + d];", "o[d] += p * K[(long)j * D + d];"),
+    ("gqa_head_zero", "gather_head(k, b, kvh, Skv, Hkv, D, rope_base, Kd);",
+     "gather_head(k, b, 0, Skv, Hkv, D, rope_base, Kd);"),
+    ("masked_row_lse_zero", "        *lse = -INFINITY;\n        return;\n    }\n    for (int j = 0; j < Skv",
+     "        *lse = 0.0;\n        return;\n    }\n    for (int j = 0; j < Skv"),
+    ("combine_weight_max", "double w = exp(lses[t] - L);", "double w = exp(lses[t] - gmax);"),
+    ("split_drops_remainder", "int len = base + (t < rem ? 1 : 0);", "int len = base;"),
+    ("tiled_no_correction", "for (int d = 0; d < D; ++d) acc[(long)i * D + d] *= c;", ""),
+    ("decode_drops_last_key", "attn_row(qq, Kd, Vd, L, D, L, scale", "attn_row(qq, Kd, Vd, L, D, L - 1, scale"),
+]
+
+
+@pytest.mark.parametrize("name,orig,planted", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_pins_reject_planted_mistake(name, orig, planted, tmp_path):
+    src = open(SRC).read()
+    assert src.count(orig) >= 1, f"mutation site for {name} not found"
+    mutated = src.replace(orig, planted, 1)
+    c_path = tmp_path / f"oracle_{name}.c"
+    so_path = tmp_path / f"liboracle_{name}.so"
+    c_path.write_text(mutated)
+    subprocess.check_call(["gcc", "-O1", "-std=c11", "-fopenmp", "-fPIC", "-shared", str(c_path),
+                           "-o", str(so_path), "-lm"])
+    failed = []
+    oracle.swap_library(str(so_path))
+    try:
+        for pin in ALL_PINS:
+            try:
+                pin()
+            except (AssertionError, oracle.OracleError, FloatingPointError, ValueError):
+                failed.append(pin.__name__)
+    finally:
+        oracle.swap_library(None)
+    assert failed, f"planted mistake {name!r} passed every pin"
