@@ -1,0 +1,177 @@
+"""B200-native exact attention: Python binding of libattn_b200.so (the C ABI in include/attn_b200.h).
+
+This module only marshals arguments: torch tensors supply device memory and the CUDA stream,
+every computation runs in the library's sm_100a kernels.  There is no fallback: if the library
+is missing or no CUDA device is present, calls raise.
+
+Entry points (same names as the C ABI):
+    attn_fwd(q, k, v, scale, causal, o=None, lse=None)                 -> (o, lse)
+    attn_fwd_ex(q, k, v, scale, causal, rope_base, q_pos0, ...)        -> (o, lse)
+    attn_decode(q, kcache, vcache, seqlens, scale, num_splits, ...)    -> (o, lse)
+    rope_apply(x, pos, base)                                           -> x (in place)
+Layouts: q/o [B, Sq, Hq, D]; k/v [B, Skv, Hkv, D]; lse [B, Hq, Sq] float32;
+decode q/o [B, Hq, D], caches [B, Smax, Hkv, D], seqlens int32 [B], lse [B, Hq];
+rope x [T, H, D], pos int32 [T].
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+
+ATTN_BF16, ATTN_FP32 = 0, 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV",
+          4: "unsupported configuration", 5: "workspace missing or too small", 6: "CUDA error",
+          7: "device wait timed out"}
+
+# symbols the library exports (kept in step with include/attn_b200.h)
+EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
+           "attn_decode_workspace_size", "rope_apply", "attn_status_string",
+           "attn_read_device_status")
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} (status {status})")
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load (once) and type the C ABI.  Raises if the library was not built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} not found: build it with `python -m exact_attention_160_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, P]
+    lib.attn_fwd_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
+    lib.attn_fwd_ex_workspace_size.argtypes = [I, I, I, I, I, I, F, I]
+    lib.attn_fwd_ex_workspace_size.restype = Z
+    lib.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, Z, I, P]
+    lib.attn_decode_workspace_size.argtypes = [I, I, I, I]
+    lib.attn_decode_workspace_size.restype = Z
+    lib.rope_apply.argtypes = [P, P, I, I, I, F, I, P]
+    lib.attn_status_string.argtypes = [I]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    lib.attn_read_device_status.argtypes = [P]
+    for f in (lib.attn_fwd, lib.attn_fwd_ex, lib.attn_decode, lib.rope_apply, lib.attn_read_device_status):
+        f.restype = I
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float32:
+        return ATTN_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise AttnError(st, what)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+def attn_fwd(q, k, v, scale: float, causal: bool, o=None, lse=None, want_lse: bool = True, stream=None):
+    """Exact attention forward.  Returns (o, lse); lse is None when want_lse is False."""
+    return attn_fwd_ex(q, k, v, scale, causal, 0.0, 0, o=o, lse=lse, want_lse=want_lse, stream=stream)
+
+
+def fwd_workspace_bytes(q, k, rope_base: float, q_pos0: int) -> int:
+    lib = load_library()
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    return int(lib.attn_fwd_ex_workspace_size(B, Hkv, Sq, Skv, D, _dtype_code(q), float(rope_base), int(q_pos0)))
+
+
+def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: int = 0, o=None, lse=None,
+                want_lse: bool = True, workspace=None, stream=None):
+    """Exact attention forward with RoPE on Q (positions q_pos0 + i) and K (positions j)."""
+    lib = load_library()
+    _need_cuda(q, k, v, o, lse, workspace)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    ws_bytes = 0
+    if rope_base > 0:
+        need = fwd_workspace_bytes(q, k, rope_base, q_pos0)
+        if workspace is None:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+        ws_bytes = workspace.numel() * workspace.element_size()
+    if rope_base > 0:
+        st = lib.attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                             float(scale), int(bool(causal)), _dtype_code(q), float(rope_base), int(q_pos0),
+                             _ptr(workspace), ws_bytes, _stream(stream))
+        _check(st, "attn_fwd_ex")
+    else:
+        st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
+                          float(scale), int(bool(causal)), _dtype_code(q), _stream(stream))
+        _check(st, "attn_fwd")
+    return o, lse
+
+
+def decode_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
+    return int(load_library().attn_decode_workspace_size(B, Hq, D, num_splits))
+
+
+def attn_decode(q, kcache, vcache, seqlens, scale: float, num_splits: int, o=None, lse=None,
+                want_lse: bool = True, workspace=None, stream=None):
+    """Split-KV decode of one token per (sequence, q head).  Returns (o, lse)."""
+    lib = load_library()
+    _need_cuda(q, kcache, vcache, seqlens, o, lse, workspace)
+    B, Hq, D = q.shape
+    Smax, Hkv = kcache.shape[1], kcache.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    st = lib.attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv,
+                         Smax, D, float(scale), int(num_splits), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream))
+    _check(st, "attn_decode")
+    return o, lse
+
+
+def rope_apply(x, pos, base: float, stream=None):
+    """Rotate x [T, H, D] in place at positions pos [T] (int32)."""
+    lib = load_library()
+    _need_cuda(x, pos)
+    T, H, D = x.shape
+    st = lib.rope_apply(_ptr(x), _ptr(pos), T, H, D, float(base), _dtype_code(x), _stream(stream))
+    _check(st, "rope_apply")
+    return x
+
+
+def read_device_status(stream=None) -> int:
+    """Read and clear the library's device status word (synchronises the stream)."""
+    return int(load_library().attn_read_device_status(_stream(stream)))

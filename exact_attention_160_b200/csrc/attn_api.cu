@@ -1,0 +1,324 @@
+// attn_api.cu -- the C ABI declared in include/attn_b200.h: host-side validation, TMA descriptor
+// encoding and kernel launches.  No function here allocates device memory.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "../../include/attn_b200.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "prefill_f32.cuh"
+#include "prefill_tc.cuh"
+#include "rope.cuh"
+
+using namespace attn;
+
+namespace {
+
+// ------------------------------------------------------------------------------------------
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda)
+// ------------------------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Tensor [B][S][H][D] bf16 viewed as 4-D (D, H, S, B); box = 64 elements x 1 head x 128 rows,
+// 128-byte swizzle (the UMMA SW128 K-major / MN-major operand layout).  Rows past S read as 0.
+bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+attn_status launch_status() {
+    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || D <= 0) return ATTN_ERR_INVALID_ARG;
+    if (Skv == 0) return ATTN_ERR_EMPTY_KV;
+    if (Skv < 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_ERR_DIM_MISMATCH;
+    if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+// Layout of the attn_fwd_ex workspace: rope table, then (bf16) rotated K as hi and lo halves.
+struct ExWorkspace {
+    size_t tab_off, khi_off, klo_off, total;
+    int positions;
+};
+
+ExWorkspace ex_workspace(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, int q_pos0) {
+    ExWorkspace w{};
+    long pq = static_cast<long>(q_pos0) + Sq;
+    w.positions = static_cast<int>(pq > Skv ? pq : Skv);
+    w.tab_off = 0;
+    size_t tab = static_cast<size_t>(w.positions) * (D / 2) * sizeof(float2);
+    w.khi_off = round_up(tab, 256);
+    size_t kbytes = dtype == ATTN_BF16 ? static_cast<size_t>(B) * Skv * Hkv * D * 2 : 0;
+    w.klo_off = round_up(w.khi_off + kbytes, 256);
+    w.total = round_up(w.klo_off + kbytes, 256);
+    return w;
+}
+
+template <int D, bool ROPE>
+attn_status launch_tc(const void* q, const void* k, const void* klo, const void* v, void* o, float* lse, int B,
+                      int Hq, int Hkv, int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0,
+                      cudaStream_t st) {
+    CUtensorMap tq, tk, tkl, tv;
+    if (!make_tmap_bshd(&tq, q, B, Sq, Hq, D) || !make_tmap_bshd(&tk, k, B, Skv, Hkv, D) ||
+        !make_tmap_bshd(&tv, v, B, Skv, Hkv, D) || !make_tmap_bshd(&tkl, ROPE ? klo : k, B, Skv, Hkv, D))
+        return ATTN_ERR_CUDA;
+    using C = TcCfg<D, ROPE>;
+    TcParams p{};
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.rope_tab = tab;
+    p.B = B, p.Hq = Hq, p.Hkv = Hkv, p.Sq = Sq, p.Skv = Skv;
+    p.causal = causal;
+    const int G = Hq / Hkv;
+    p.pair_heads = (G % 2 == 0) ? 1 : 0;
+    p.n_row_tiles = p.pair_heads ? (Sq + 127) / 128 : (Sq + 255) / 256;
+    p.heads_per_item = p.pair_heads ? Hq / 2 : Hq;
+    p.q_pos0 = q_pos0;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    const long grid = static_cast<long>(p.n_row_tiles) * B * p.heads_per_item;
+    if (grid > 2147483647L) return ATTN_ERR_UNSUPPORTED;
+    auto kern = prefill_tc_kernel<D, ROPE>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        attr_set = true;
+    }
+    kern<<<static_cast<unsigned>(grid), kTcThreads, C::SMEM_BYTES, st>>>(tq, tk, tkl, tv, p);
+    return launch_status();
+}
+
+template <int D>
+attn_status launch_f32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0, cudaStream_t st) {
+    const size_t smem = 2 * 64 * D * sizeof(float);
+    auto kern = prefill_f32_kernel<D>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+            return ATTN_ERR_CUDA;
+        attr_set = true;
+    }
+    dim3 grid((Sq + 63) / 64, Hq, B);
+    if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
+    kern<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
+                                  static_cast<const float*>(v), static_cast<float*>(o), lse, Hq, Hkv, Sq, Skv, scale,
+                                  causal, tab, q_pos0);
+    return launch_status();
+}
+
+attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                     int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
+                     void* workspace, size_t workspace_bytes, cudaStream_t st) {
+    attn_status s = check_common(B, Hq, Hkv, Sq, Skv, D, scale, causal);
+    if (s != ATTN_OK) return s;
+    if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;
+    const bool rope = rope_base > 0.f;
+    if (rope && !isfinite(rope_base)) return ATTN_ERR_INVALID_ARG;
+    if (rope && q_pos0 < 0) return ATTN_ERR_INVALID_ARG;
+    if (rope && (D % 2) != 0) return ATTN_ERR_DIM_MISMATCH;
+
+    const float2* tab = nullptr;
+    ExWorkspace w{};
+    if (rope) {
+        w = ex_workspace(B, Hkv, Sq, Skv, D, dtype, q_pos0);
+        if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+        uint8_t* ws = static_cast<uint8_t*>(workspace);
+        float2* t = reinterpret_cast<float2*>(ws + w.tab_off);
+        const long n = static_cast<long>(w.positions) * (D / 2);
+        rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, st>>>(
+            t, w.positions, D, static_cast<double>(rope_base));
+        if ((s = launch_status()) != ATTN_OK) return s;
+        tab = t;
+    }
+
+    if (dtype == ATTN_FP32) {
+        return D == 64 ? launch_f32<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st)
+                       : launch_f32<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st);
+    }
+    if (!rope) {
+        return D == 64 ? launch_tc<64, false>(q, k, nullptr, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, nullptr, 0, st)
+                       : launch_tc<128, false>(q, k, nullptr, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, nullptr, 0, st);
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    uint32_t* khi = reinterpret_cast<uint32_t*>(ws + w.khi_off);
+    uint32_t* klo = reinterpret_cast<uint32_t*>(ws + w.klo_off);
+    const long npairs = static_cast<long>(B) * Skv * Hkv * (D / 2);
+    rope_split_kv_kernel<<<static_cast<unsigned>((npairs + 255) / 256 < 148 * 64 ? (npairs + 255) / 256 : 148 * 64), 256,
+                           0, st>>>(static_cast<const uint32_t*>(k), khi, klo, tab, npairs, Skv, Hkv, D);
+    if ((s = launch_status()) != ATTN_OK) return s;
+    return D == 64 ? launch_tc<64, true>(q, khi, klo, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st)
+                   : launch_tc<128, true>(q, khi, klo, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st);
+}
+
+template <int D, int GC>
+attn_status launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o, float* lse,
+                          int B, int Hq, int Hkv, int Smax, float scale, int num_splits, float* o_part,
+                          float* lse_part, cudaStream_t st) {
+    constexpr int LPK = D / 8, SLOTS = 32 / LPK, NPART = kDecodeWarps * SLOTS;
+    const size_t smem = (2 * NPART * GC + NPART * GC * D) * sizeof(float);
+    const int G = Hq / Hkv;
+    dim3 grid(num_splits, Hkv * (G / GC), B);
+    if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
+    decode_split_kernel<D, GC><<<grid, kDecodeWarps * 32, smem, st>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kc),
+        static_cast<const __nv_bfloat16*>(vc), seqlens, o_part, lse_part, Hkv, G, Smax, num_splits,
+        scale * 1.4426950408889634f);
+    attn_status s = launch_status();
+    if (s != ATTN_OK) return s;
+    const int warps = B * Hq;
+    decode_combine_kernel<D><<<(warps + 3) / 4, 128, 0, st>>>(o_part, lse_part, seqlens,
+                                                               static_cast<__nv_bfloat16*>(o), lse, B, Hq, Smax,
+                                                               num_splits);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
+                     int Skv, int D, float scale, int causal, attn_dtype dtype, attn_stream_t stream) {
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, 0.f, 0, nullptr, 0,
+                    static_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
+                        void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base, q_pos0, workspace,
+                    workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+size_t attn_fwd_ex_workspace_size(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
+                                  int q_pos0) {
+    if (!(rope_base > 0.f) || B <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0 || q_pos0 < 0) return 0;
+    return ex_workspace(B, Hkv, Sq, Skv, D, dtype, q_pos0).total;
+}
+
+size_t attn_decode_workspace_size(int B, int Hq, int D, int num_splits) {
+    if (B <= 0 || Hq <= 0 || D <= 0 || num_splits <= 0) return 0;
+    const size_t slots = static_cast<size_t>(B) * Hq * num_splits;
+    return round_up(slots * D * sizeof(float), 256) + round_up(slots * sizeof(float), 256);
+}
+
+attn_status attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens, void* o,
+                        float* lse, int B, int Hq, int Hkv, int Smax, int D, float scale, int num_splits,
+                        void* workspace, size_t workspace_bytes, attn_dtype dtype, attn_stream_t stream) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_splits <= 0) return ATTN_ERR_INVALID_ARG;
+    if (Smax == 0) return ATTN_ERR_EMPTY_KV;
+    if (Smax < 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_ERR_DIM_MISMATCH;
+    if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !kcache || !vcache || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
+    const size_t need = attn_decode_workspace_size(B, Hq, D, num_splits);
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+    const size_t slots = static_cast<size_t>(B) * Hq * num_splits;
+    float* o_part = static_cast<float*>(workspace);
+    float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(slots * D * sizeof(float), 256));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int G = Hq / Hkv;
+    const int GC = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
+#define ATTN_DECODE_CASE(DD, GG)                                                                              \
+    if (D == DD && GC == GG)                                                                                  \
+        return launch_decode<DD, GG>(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Smax, scale, num_splits, \
+                                     o_part, lse_part, st);
+    ATTN_DECODE_CASE(64, 1)
+    ATTN_DECODE_CASE(64, 2)
+    ATTN_DECODE_CASE(64, 4)
+    ATTN_DECODE_CASE(128, 1)
+    ATTN_DECODE_CASE(128, 2)
+    ATTN_DECODE_CASE(128, 4)
+#undef ATTN_DECODE_CASE
+    return ATTN_ERR_UNSUPPORTED;
+}
+
+attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float base, attn_dtype dtype,
+                       attn_stream_t stream) {
+    if (T <= 0 || H <= 0 || D <= 0) return ATTN_ERR_INVALID_ARG;
+    if (D % 2 != 0) return ATTN_ERR_DIM_MISMATCH;
+    if (!(base > 0.f) || !isfinite(base)) return ATTN_ERR_INVALID_ARG;
+    if (!x || !pos) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(x) & (dtype == ATTN_BF16 ? 3u : 7u)) != 0) return ATTN_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned grid = T < 65535 * 4 ? static_cast<unsigned>(T) : 65535u * 4;
+    const size_t smem = (D / 2) * sizeof(float2);
+    if (dtype == ATTN_BF16)
+        rope_apply_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>(static_cast<__nv_bfloat16*>(x), pos, T, H, D,
+                                                                  static_cast<double>(base));
+    else
+        rope_apply_kernel<float><<<grid, 128, smem, st>>>(static_cast<float*>(x), pos, T, H, D,
+                                                          static_cast<double>(base));
+    return launch_status();
+}
+
+const char* attn_status_string(attn_status s) {
+    switch (s) {
+        case ATTN_OK: return "ok";
+        case ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case ATTN_ERR_DIM_MISMATCH: return "dimension mismatch";
+        case ATTN_ERR_EMPTY_KV: return "empty KV";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case ATTN_ERR_CUDA: return "CUDA error";
+        case ATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+int attn_read_device_status(attn_stream_t stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return -1;
+    int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return -1;
+    if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+    return v;
+}
+
+}  // extern "C"

@@ -1,0 +1,468 @@
+// prefill_tc.cuh -- exact attention forward on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// The method (scirs2-neural 0.4.3, src/layers/flash_attention.rs): for a block of query rows,
+// walk the key/value blocks; per block form S = Q K^T * scale, mask, and fold it into a running
+// row max m and row sum l with the online-softmax recurrence (online_softmax_update):
+//   m' = max(m, rowmax S);  l' = l e^(m-m') + sum e^(S-m');  O' = O e^(m-m') + e^(S-m') V
+// skipping key blocks that lie wholly above the causal diagonal (flash_attention_forward), and
+// finish with O / l and the logsumexp m + ln l.  Grouped-query head sharing follows
+// scirs2-neural 0.4.4 grouped_query_attention.rs (q head h reads kv head h / (Hq/Hkv)).
+//
+// B200 design (not the pages' CPU loop structure):
+//   * One CTA holds two 128-row query tiles that read the same K/V: two q heads of one GQA group
+//     at the same rows when the group size is even, else two consecutive row tiles of one head.
+//     Each K/V tile is therefore loaded once for 256 query rows.
+//   * Warp roles (10 warps): warp 0 issues TMA loads (Q once, then a ring of K/V stages);
+//     warp 1 owns tensor memory and issues every tcgen05.mma from one thread; warps 2-5 and
+//     6-9 are the softmax warpgroups of query tile 0 and 1, one thread per query row.  A warp
+//     may only touch TMEM lanes 32*(warp%4) .. +31, so the row of a softmax thread is
+//     32*(warp%4) + lane: each group of four consecutive warps covers all 128 lanes.
+//   * S = Q K^T is a bf16 MMA (A and B from shared memory, M=128, N=128) into TMEM; the softmax
+//     threads read their row of S with tcgen05.ld, compute P = exp2(S*scale*log2e - m) in fp32,
+//     round P to bf16 and write it back to TMEM; O += P V is an MMA with A = P from TMEM and
+//     B = V from shared memory (N = D), accumulating in TMEM.
+//   * Lazy rescale: the running max used for the exponent only moves when the block max exceeds
+//     it by more than kRescaleThreshold (log2 units, i.e. a factor 256), which keeps P <= 256
+//     while skipping the O correction on almost every block.  The "running max is -inf" guard
+//     makes rows with no visible key yet contribute nothing.
+//   * With RoPE, Q is rotated in shared memory right after its TMA load and K arrives
+//     pre-rotated; both carry hi + lo bf16 halves and S = Qh Kh^T + Qh Kl^T + Ql Kh^T.
+//
+// TMEM columns (512 allocated): S0 [0,128) S1 [128,256) O0, O1 (D each) after them; with D=64
+// P0 and P1 get their own 64 columns, with D=128 P_i overwrites the first 64 columns of S_i
+// (S_i is fully in registers by then; the next S_i MMA is issued only after PV_i completed).
+#pragma once
+
+#include "common.cuh"
+
+namespace attn {
+
+constexpr int kTcThreads = 320;
+constexpr float kRescaleThreshold = 8.0f;
+constexpr float kLn2 = 0.69314718055994531f;
+
+template <int D, bool ROPE>
+struct TcCfg {
+    static constexpr int BM = 128;                    // query rows per tile
+    static constexpr int BN = 128;                    // keys per KV tile
+    static constexpr int NBOX = D / 64;               // 128-byte-wide TMA boxes per row
+    static constexpr int TILE_BYTES = BN * D * 2;     // one 128 x D bf16 tile
+    static constexpr int KSTEPS = D / 16;             // MMA K steps of S = Q K^T
+    // D=128 with RoPE holds four Q tiles (hi, lo for both query tiles): one K/V stage fits.
+    static constexpr int STAGES = (D == 64) ? (ROPE ? 3 : 4) : (ROPE ? 1 : 2);
+    static constexpr int K_TILES = ROPE ? 2 : 1;      // Kh, Kl
+    static constexpr int Q_TILES = ROPE ? 2 : 1;      // Qh, Ql
+    static constexpr int STAGE_BYTES = (K_TILES + 1) * TILE_BYTES;
+    static constexpr int Q_BYTES = 2 * Q_TILES * TILE_BYTES;
+    static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = SMEM_DATA + 1024 /* alignment slack */ + 256 /* barriers */;
+    static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
+    static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
+    static constexpr uint32_t COL_P0 = (D == 64) ? 384 : 0;
+    static constexpr uint32_t COL_P1 = (D == 64) ? 448 : 128;
+    static constexpr bool P_ALIASES_S = (D != 64);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct TcParams {
+    __nv_bfloat16* o;
+    float* lse;
+    const float2* rope_tab;   // [positions][D/2] (cos, sin), ROPE only
+    int B, Hq, Hkv, Sq, Skv;
+    int causal;
+    int pair_heads;           // 1: tile pair = two heads of a group; 0: two row tiles of one head
+    int q_pos0;
+    int n_row_tiles;          // row tiles per head in the work decomposition
+    int heads_per_item;       // Hq / 2 when pairing heads, Hq otherwise
+    float scale_log2;         // scale * log2(e)
+};
+
+struct TcTile {
+    int h;        // q head
+    int r0;       // first query row
+    int nkv;      // key tiles to process (0: nothing visible or inactive)
+    bool active;
+};
+
+__device__ __forceinline__ int tc_kv_tiles(const TcParams& p, int r0) {
+    const int nkv_all = (p.Skv + 127) / 128;
+    if (!p.causal) return nkv_all;
+    const long last = static_cast<long>(r0) + 127 + (static_cast<long>(p.Skv) - p.Sq);
+    if (last < 0) return 0;
+    const long n = last / 128 + 1;
+    return n < nkv_all ? static_cast<int>(n) : nkv_all;
+}
+
+template <int D, bool ROPE>
+__global__ void __maxnreg__(200) prefill_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
+    const TcParams p) {
+    using C = TcCfg<D, ROPE>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;                                   // [2][Q_TILES][TILE_BYTES]
+    uint8_t* sKV = smem + C::Q_BYTES;                     // [STAGES][(K_TILES+1)][TILE_BYTES]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_DATA);
+    uint64_t* bar_q_full = bars + 0;
+    uint64_t* bar_q_ready = bars + 1;
+    uint64_t* bar_s_full = bars + 2;       // [2]
+    uint64_t* bar_p_ready = bars + 4;      // [2]
+    uint64_t* bar_pv_done = bars + 6;      // [2]
+    uint64_t* bar_k_full = bars + 8;       // [STAGES]
+    uint64_t* bar_v_full = bar_k_full + C::STAGES;
+    uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
+    uint64_t* bar_mma_final = bar_kv_empty + C::STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma_final + 1);
+
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+
+    // ---- work item -> (batch, two query tiles) -------------------------------------------
+    const int items_per_rowtile = p.B * p.heads_per_item;
+    const int rt = (p.n_row_tiles - 1) - static_cast<int>(blockIdx.x) / items_per_rowtile;   // heavy first
+    const int rem = static_cast<int>(blockIdx.x) % items_per_rowtile;
+    const int b = rem / p.heads_per_item;
+    const int hi = rem % p.heads_per_item;
+    TcTile tile[2];
+    if (p.pair_heads) {
+        tile[0].h = 2 * hi;
+        tile[1].h = 2 * hi + 1;
+        tile[0].r0 = tile[1].r0 = rt * 128;
+    } else {
+        tile[0].h = tile[1].h = hi;
+        tile[0].r0 = rt * 256;
+        tile[1].r0 = rt * 256 + 128;
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        tile[i].active = tile[i].r0 < p.Sq;
+        tile[i].nkv = tile[i].active ? tc_kv_tiles(p, tile[i].r0) : 0;
+    }
+    const int kvh = tile[0].h / (p.Hq / p.Hkv);
+    const int nkv = max(tile[0].nkv, tile[1].nkv);
+
+    // ---- set-up --------------------------------------------------------------------------
+    if (tid == 0) {
+        mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_ready, 256);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(bar_s_full + i, 1);
+            mbar_init(bar_p_ready + i, 128);
+            mbar_init(bar_pv_done + i, 1);
+        }
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(bar_k_full + s, 1);
+            mbar_init(bar_v_full + s, 1);
+            mbar_init(bar_kv_empty + s, 1);
+        }
+        mbar_init(bar_mma_final, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        if (ROPE) tma_prefetch_desc(&tm_klo);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // =============================== TMA producer ===================================
+        if (lane == 0) {
+            const uint64_t pol_q = l2_policy_evict_first();
+            const uint64_t pol_kv = l2_policy_evict_last();
+            uint32_t qbytes = 0;
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+                if (tile[i].active) qbytes += C::TILE_BYTES;
+            mbar_arrive_expect_tx(bar_q_full, qbytes);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                if (!tile[i].active) continue;
+                uint8_t* dst = sQ + i * C::Q_TILES * C::TILE_BYTES;
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    tma_load_4d(&tm_q, bar_q_full, dst + bx * (C::TILE_BYTES / C::NBOX), bx * 64, tile[i].h,
+                                tile[i].r0, b, pol_q);
+            }
+            int issued = 0;
+            for (int j = 0; j < nkv; ++j) {
+                const int s = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                if (!mbar_wait(bar_kv_empty + s, ph ^ 1)) break;
+                issued = j + 1;
+                uint8_t* st = sKV + s * C::STAGE_BYTES;
+                mbar_arrive_expect_tx(bar_k_full + s, C::K_TILES * C::TILE_BYTES);
+                for (int bx = 0; bx < C::NBOX; ++bx) {
+                    tma_load_4d(&tm_k, bar_k_full + s, st + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
+                                j * 128, b, pol_kv);
+                    if (ROPE)
+                        tma_load_4d(&tm_klo, bar_k_full + s, st + C::TILE_BYTES + bx * (C::TILE_BYTES / C::NBOX),
+                                    bx * 64, kvh, j * 128, b, pol_kv);
+                }
+                uint8_t* sv = st + C::K_TILES * C::TILE_BYTES;
+                mbar_arrive_expect_tx(bar_v_full + s, C::TILE_BYTES);
+                for (int bx = 0; bx < C::NBOX; ++bx)
+                    tma_load_4d(&tm_v, bar_v_full + s, sv + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
+                                j * 128, b, pol_kv);
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            mbar_wait(bar_q_full, 0);
+            for (int j = issued - C::STAGES > 0 ? issued - C::STAGES : 0; j < issued; ++j) {
+                mbar_wait(bar_k_full + j % C::STAGES, (j / C::STAGES) & 1);
+                mbar_wait(bar_v_full + j % C::STAGES, (j / C::STAGES) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // =============================== MMA issuer ======================================
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            bool ok = mbar_wait(ROPE ? bar_q_ready : bar_q_full, 0);
+            tc_fence_after();
+            for (int j = 0; ok && j < nkv; ++j) {
+                const int s = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                const uint32_t sK = smem_u32(sKV + s * C::STAGE_BYTES);
+                const uint32_t sV = sK + C::K_TILES * C::TILE_BYTES;
+                if (!mbar_wait(bar_k_full + s, ph)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (j >= tile[i].nkv) continue;
+                    if (C::P_ALIASES_S && j > 0) {
+                        // PV_i(j-1) still reads P_i from the columns S_i(j) will overwrite
+                        if (!mbar_wait(bar_pv_done + i, (j - 1) & 1)) { ok = false; break; }
+                        tc_fence_after();
+                    }
+                    const uint32_t sQi = smem_u32(sQ + i * C::Q_TILES * C::TILE_BYTES);
+                    const uint32_t dS = tmem + (i ? C::COL_S1 : C::COL_S0);
+                    // chains: (Qh,Kh) [+ (Qh,Kl) + (Ql,Kh) with RoPE]
+                    constexpr int NCHAIN = ROPE ? 3 : 1;
+#pragma unroll
+                    for (int ch = 0; ch < NCHAIN; ++ch) {
+                        const uint32_t qa = sQi + (ch == 2 ? C::TILE_BYTES : 0);
+                        const uint32_t kb = sK + (ch == 1 ? C::TILE_BYTES : 0);
+#pragma unroll
+                        for (int kk = 0; kk < C::KSTEPS; ++kk) {
+                            // K step kk: box kk/4, 32-byte column offset (kk%4) inside the 128-byte row
+                            const uint32_t off = (kk >> 2) * (C::TILE_BYTES / C::NBOX) + (kk & 3) * 32;
+                            const uint64_t da = smem_desc_sw128(qa + off, 16, 1024);
+                            const uint64_t db = smem_desc_sw128(kb + off, 16, 1024);
+                            mma_ss(dS, da, db, idesc_qk, (ch > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    mma_commit(bar_s_full + i);
+                }
+                if (!ok) break;
+                if (!mbar_wait(bar_v_full + s, ph)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (j >= tile[i].nkv) continue;
+                    if (!mbar_wait(bar_p_ready + i, j & 1)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        // keys [16kk, 16kk+16): 16 rows of 128 B in every 64-wide D box
+                        const uint64_t db = smem_desc_sw128(sV + kk * 2048, C::TILE_BYTES / C::NBOX, 1024);
+                        mma_ts(tmem + (i ? C::COL_O1 : C::COL_O0), tmem + (i ? C::COL_P1 : C::COL_P0) + kk * 8, db,
+                               idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(bar_pv_done + i);
+                }
+                if (!ok) break;
+                mma_commit(bar_kv_empty + s);
+            }
+            // every MMA issued above must be complete before tensor memory is released
+            mma_commit(bar_mma_final);
+            mbar_wait(bar_mma_final, 0);
+        }
+    } else {
+        // =============================== softmax warpgroups =============================
+        const int wg = (warp - 2) >> 2;             // query tile index
+        const int row = (warp & 3) * 32 + lane;     // 0..127 == TMEM lane
+        TcTile T;
+        T.h = wg ? tile[1].h : tile[0].h;
+        T.r0 = wg ? tile[1].r0 : tile[0].r0;
+        T.nkv = wg ? tile[1].nkv : tile[0].nkv;
+        T.active = wg ? tile[1].active : tile[0].active;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_base + (wg ? C::COL_S1 : C::COL_S0);
+        const uint32_t tO = tmem + lane_base + (wg ? C::COL_O1 : C::COL_O0);
+        const uint32_t tP = tmem + lane_base + (wg ? C::COL_P1 : C::COL_P0);
+        const int qrow = T.r0 + row;                // absolute query row
+        const long off_c = static_cast<long>(p.Skv) - p.Sq;
+        bool ok = true;
+
+        if (ROPE) {
+            // rotate this row of the query tile in place: hi half -> Qh, remainder -> Ql
+            ok = mbar_wait(bar_q_full, 0);
+            if (ok && T.active && qrow < p.Sq) {
+                uint8_t* qh = sQ + wg * C::Q_TILES * C::TILE_BYTES;
+                uint8_t* ql = qh + C::TILE_BYTES;
+                const float2* tab = p.rope_tab + static_cast<long>(p.q_pos0 + qrow) * (D / 2);
+#pragma unroll
+                for (int bx = 0; bx < C::NBOX; ++bx) {
+#pragma unroll
+                    for (int ck = 0; ck < 8; ++ck) {
+                        const uint32_t o = bx * (C::TILE_BYTES / C::NBOX) + sw128_offset(row, ck);
+                        uint4 w = *reinterpret_cast<uint4*>(qh + o);
+                        uint32_t ww[4] = {w.x, w.y, w.z, w.w}, hh[4], ll[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 cs = tab[bx * 32 + ck * 4 + e];
+                            const float x0 = bf16lo_to_f32(ww[e]), x1 = bf16hi_to_f32(ww[e]);
+                            const float y0 = x0 * cs.x - x1 * cs.y;
+                            const float y1 = x0 * cs.y + x1 * cs.x;
+                            hh[e] = pack_bf16x2(y0, y1);
+                            ll[e] = pack_bf16x2(y0 - bf16lo_to_f32(hh[e]), y1 - bf16hi_to_f32(hh[e]));
+                        }
+                        *reinterpret_cast<uint4*>(qh + o) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+                        *reinterpret_cast<uint4*>(ql + o) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
+                    }
+                }
+            } else if (ok && T.active) {
+                // rows past Sq were zero-filled by TMA; give Ql zeros too
+                uint8_t* ql = sQ + wg * C::Q_TILES * C::TILE_BYTES + C::TILE_BYTES;
+#pragma unroll
+                for (int bx = 0; bx < C::NBOX; ++bx)
+#pragma unroll
+                    for (int ck = 0; ck < 8; ++ck)
+                        *reinterpret_cast<uint4*>(ql + bx * (C::TILE_BYTES / C::NBOX) + sw128_offset(row, ck)) =
+                            make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(bar_q_ready);
+        }
+
+        float m_run = -INFINITY;   // running max used in the exponent (log2 units)
+        float l_run = 0.f;
+        const float sl2 = p.scale_log2;
+        for (int j = 0; ok && j < T.nkv; ++j) {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) tmem_ld32(tS + cb * 32, sr[cb]);
+            tmem_wait_ld();
+            // mask: keys past Skv, and (causal) keys beyond this row's diagonal
+            const int k0 = j * 128;
+            const long lim_causal = p.causal ? static_cast<long>(qrow) + off_c : static_cast<long>(p.Skv) - 1;
+            const long lim = lim_causal < p.Skv - 1 ? lim_causal : static_cast<long>(p.Skv) - 1;
+            float mx = -INFINITY;
+            if (static_cast<long>(k0) + 127 > lim) {
+                const long nvis = lim - k0 + 1;     // keys [k0, k0+nvis) visible
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (cb * 32 + e >= nvis) sr[cb][e] = __float_as_uint(-INFINITY);
+            }
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[cb][e]));
+            const float tmax = mx * sl2;
+            // lazy rescale: move the exponent's max only when the block max exceeds it by > threshold
+            const bool need = tmax > m_run + kRescaleThreshold;
+            float corr = 1.f;
+            if (need) {
+                corr = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - tmax);
+                m_run = tmax;
+            }
+            // O correction: only warps with a rescaling row, only once O holds earlier blocks
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int cb = 0; cb < D / 32; ++cb) {
+                    uint32_t orr[32];
+                    tmem_ld32(tO + cb * 32, orr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
+                    tmem_st32(tO + cb * 32, orr);
+                }
+                tmem_wait_st();
+            }
+            l_run *= corr;
+            const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+            if (!C::P_ALIASES_S && j > 0) {
+                // P_i(j-1) must have been consumed by PV_i(j-1) before it is overwritten
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) { ok = false; break; }
+                tc_fence_after();
+            }
+            float lsum = 0.f;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = fast_exp2(fmaf(__uint_as_float(sr[cb][2 * e]), sl2, -mu));
+                    const float p1 = fast_exp2(fmaf(__uint_as_float(sr[cb][2 * e + 1]), sl2, -mu));
+                    lsum += p0 + p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                }
+                tmem_st16(tP + cb * 16, pk);
+            }
+            l_run += lsum;
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(bar_p_ready + wg);
+        }
+
+        // epilogue: O / l -> bf16, lse.  The TMEM reads are warp-collective, so every lane of
+        // the warp takes part; only rows inside [0, Sq) are stored.
+        if (T.active) {
+            bool have = ok && T.nkv > 0;
+            if (have) {
+                have = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (T.nkv - 1) & 1));
+                tc_fence_after();
+            }
+            const bool store = qrow < p.Sq;
+            const float inv = (have && l_run > 0.f) ? 1.f / l_run : 0.f;
+            __nv_bfloat16* orow = p.o + ((static_cast<long>(b) * p.Sq + qrow) * p.Hq + T.h) * D;
+#pragma unroll
+            for (int cb = 0; cb < D / 32; ++cb) {
+                uint32_t orr[32];
+                if (have) {
+                    tmem_ld32(tO + cb * 32, orr);
+                    tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) orr[e] = 0u;
+                }
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
+                if (store) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+            if (store && p.lse != nullptr)
+                p.lse[(static_cast<long>(b) * p.Hq + T.h) * p.Sq + qrow] =
+                    (have && l_run > 0.f) ? (m_run + fast_log2(l_run)) * kLn2 : -INFINITY;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace attn

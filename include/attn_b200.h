@@ -1,0 +1,144 @@
+/*
+ * attn_b200.h -- C ABI of the B200 (sm_100a) exact-attention library, libattn_b200.so.
+ *
+ * Operations (sources are docs.rs source pages, cited as crate version, file, Rust item):
+ *   attn_fwd     exact scaled-dot-product attention O = softmax(Q K^T * scale + mask) V with
+ *                the per-row logsumexp, grouped-query head sharing and an optional causal mask.
+ *                scirs2-neural 0.4.3 src/layers/flash_attention.rs (flash_attention_forward,
+ *                online_softmax_update); scirs2-neural 0.4.4 src/layers/grouped_query_attention.rs
+ *                (GroupedQueryAttention::forward_with_cache: head groups, causal mask with a
+ *                cache offset).
+ *   attn_fwd_ex  attn_fwd with rotary position embedding applied to Q and K first.
+ *                scirs2-neural 0.4.4 grouped_query_attention.rs (RotaryPositionEmbedding::apply).
+ *   attn_decode  one query token per (sequence, q head) against a KV cache, split along the keys
+ *                and merged by logsumexp.  oxibonsai-model 0.1.4 src/layers/flash_decode.rs
+ *                (flash_decode_tile, combine_tile_outputs, flash_decode_single_head);
+ *                whisper-apr 0.3.1 src/model/lfm2/gqa.rs (attention_cached).
+ *   rope_apply   the rotation alone, in place.  RotaryPositionEmbedding::apply as above.
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers (CUDA global memory), row-major and contiguous in
+ *     the layouts stated below, 16-byte aligned.  The caller owns every buffer; the library
+ *     allocates no memory on these paths.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     No call synchronises the device.  Arguments are validated on the host before any launch;
+ *     an invalid call returns an error status and launches nothing.
+ *   - ATTN_ERR_CUDA means a launch or driver call failed; the CUDA error is left for the caller's
+ *     next cudaGetLastError() / synchronisation to report as well.
+ *   - Kernels never trap.  Device-side anomalies (a bounded wait that gave up, a decode length
+ *     outside [1, Smax]) set bits in a device status word read by attn_read_device_status().
+ *   - Softmax semantics: s_ij = scale * <q_i, k_j>; with `causal`, key j is masked for query
+ *     row i when j > i + (Skv - Sq) (bottom-right alignment: the last query row sees every key).
+ *     lse_i = ln sum_j exp(s_ij) over unmasked keys (natural log, scaled scores).  A row with no
+ *     unmasked key gets o_i = 0 and lse_i = -inf.
+ *   - GQA: q head h reads kv head h / (Hq / Hkv); Hq must be a multiple of Hkv (Hkv == Hq is
+ *     multi-head, Hkv == 1 is multi-query attention).
+ *   - Supported head dims: D in {64, 128}.  Other values return ATTN_ERR_UNSUPPORTED.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = 1,    /* a size <= 0, a NULL required pointer, a bad flag          */
+    ATTN_ERR_DIM_MISMATCH = 2,   /* Hq not a multiple of Hkv; odd D with RoPE                 */
+    ATTN_ERR_EMPTY_KV = 3,       /* Skv == 0 / Smax == 0: no key to attend to                 */
+    ATTN_ERR_UNSUPPORTED = 4,    /* valid request outside what the kernels implement          */
+    ATTN_ERR_WORKSPACE = 5,      /* workspace NULL or smaller than the *_workspace_size query */
+    ATTN_ERR_CUDA = 6,           /* a CUDA launch or driver call failed                       */
+    ATTN_ERR_DEVICE_TIMEOUT = 7  /* reserved for status-word decoding by callers              */
+} attn_status;
+
+typedef enum {
+    ATTN_BF16 = 0, /* q, k, v, o, x stored as bfloat16; fp32 accumulation                    */
+    ATTN_FP32 = 1  /* q, k, v, o, x stored as float32; fp32 arithmetic (no TF32)              */
+} attn_dtype;
+
+typedef void* attn_stream_t; /* a cudaStream_t */
+
+/*
+ * attn_fwd -- exact attention forward (prefill).
+ *   q    [B, Sq, Hq, D]   dtype          read
+ *   k, v [B, Skv, Hkv, D] dtype          read
+ *   o    [B, Sq, Hq, D]   dtype          written
+ *   lse  [B, Hq, Sq]      float32        written; may be NULL (not produced)
+ *   scale                  the score multiplier (commonly 1/sqrt(D)); must be finite and > 0
+ *   causal                 0 or 1
+ * Returns ATTN_OK, or INVALID_ARG / DIM_MISMATCH / EMPTY_KV / UNSUPPORTED / CUDA.
+ * bf16 path: QK^T and PV on tcgen05 tensor cores, P rounded to bf16, fp32 accumulators.
+ */
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                     int Hkv, int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype,
+                     attn_stream_t stream);
+
+/*
+ * attn_fwd_ex -- attn_fwd with RoPE on Q and K (rope_base > 0; rope_base <= 0 is attn_fwd).
+ *   Query row i is rotated at position q_pos0 + i, key j at position j:
+ *   theta_p = pos * rope_base^(-2p/D) for pair p; (x_2p, x_2p+1) -> (x_2p cos - x_2p+1 sin,
+ *   x_2p sin + x_2p+1 cos).  Angles are formed in double precision.  q_pos0 >= 0; D even.
+ *   workspace / workspace_bytes: device scratch of at least attn_fwd_ex_workspace_size(...)
+ *   bytes, owned by the caller; its contents are overwritten.  With rope_base <= 0 the
+ *   workspace may be NULL.
+ * bf16 path: rotated Q and K are carried as a pair of bf16 values (hi + lo) each, so the
+ * rotated operands keep about 16 mantissa bits; QK^T runs as three bf16 MMA chains.
+ */
+attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal,
+                        attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
+                        size_t workspace_bytes, attn_stream_t stream);
+
+/* Bytes of workspace attn_fwd_ex needs for these sizes (0 when rope_base <= 0).            */
+size_t attn_fwd_ex_workspace_size(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtype,
+                                  float rope_base, int q_pos0);
+
+/*
+ * attn_decode -- one query token per (sequence b, q head) against a KV cache, split-KV.
+ *   q       [B, Hq, D]          bf16    read
+ *   kcache  [B, Smax, Hkv, D]   bf16    read (rows >= seqlens[b] are never read)
+ *   vcache  [B, Smax, Hkv, D]   bf16    read
+ *   seqlens [B]                 int32   read on the device; values outside [1, Smax] are
+ *                                       clamped and flagged in the device status word
+ *   o       [B, Hq, D]          bf16    written
+ *   lse     [B, Hq]             float32 written; may be NULL
+ *   num_splits  upper bound on KV splits per sequence (>= 1); sequence b uses
+ *               clamp(seqlens[b] / 512, 1, num_splits) contiguous near-equal splits
+ *   workspace   device scratch of >= attn_decode_workspace_size(B, Hq, D, num_splits) bytes
+ * No causal mask: the single new token sees the whole cache.  Only dtype ATTN_BF16.
+ */
+attn_status attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                        void* o, float* lse, int B, int Hq, int Hkv, int Smax, int D, float scale,
+                        int num_splits, void* workspace, size_t workspace_bytes, attn_dtype dtype,
+                        attn_stream_t stream);
+
+/* Bytes of workspace attn_decode needs (partial outputs and logsumexps of every split).    */
+size_t attn_decode_workspace_size(int B, int Hq, int D, int num_splits);
+
+/*
+ * rope_apply -- rotate x in place: x [T, H, D] (dtype), token t at position pos[t]
+ * (int32 device array [T]); rotation as in attn_fwd_ex.  D must be even (DIM_MISMATCH).
+ */
+attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float base, attn_dtype dtype,
+                       attn_stream_t stream);
+
+/* Static description of a status code.                                                     */
+const char* attn_status_string(attn_status s);
+
+/*
+ * Read and clear the device status word (bit 1: a bounded wait gave up; bit 2: a decode
+ * sequence length was clamped; bit 4: tensor memory allocation failed).  Synchronises
+ * `stream` first.  Returns the bits, or -1 if the read itself failed.
+ */
+int attn_read_device_status(attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

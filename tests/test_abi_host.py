@@ -1,0 +1,96 @@
+"""The C-ABI library loads, exports every symbol the header declares, and rejects invalid calls on
+the host before any launch (CPU only: these paths make no CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_160_b200 as ea
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_attention_160_b200 import build
+    build.build()
+    return ea.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    assert set(names) == set(ea.EXPORTS), names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} not exported"
+
+
+FAKE = ctypes.c_void_p(1 << 20)   # aligned, never dereferenced: validation rejects first
+
+
+def fwd(lib, B=1, Hq=2, Hkv=2, Sq=8, Skv=8, D=64, scale=0.125, causal=0, dtype=0, ptr=FAKE):
+    return lib.attn_fwd(ptr, ptr, ptr, ptr, None, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, None)
+
+
+def test_fwd_validation(lib):
+    assert fwd(lib, B=0) == 1
+    assert fwd(lib, Sq=-1) == 1
+    assert fwd(lib, Skv=0) == 3                   # empty KV (flash_decode.rs EmptyKv)
+    assert fwd(lib, Hq=3, Hkv=2) == 2             # Hq not a multiple of Hkv
+    assert fwd(lib, D=96) == 4                    # head dims other than 64/128
+    assert fwd(lib, scale=0.0) == 1
+    assert fwd(lib, scale=float("nan")) == 1
+    assert fwd(lib, causal=2) == 1
+    assert fwd(lib, dtype=7) == 1
+    assert fwd(lib, ptr=None) == 1
+    assert fwd(lib, ptr=ctypes.c_void_p((1 << 20) + 2)) == 1   # misaligned
+
+
+def test_fwd_ex_validation(lib):
+    P = FAKE
+    need = lib.attn_fwd_ex_workspace_size(1, 2, 8, 8, 64, 0, 10000.0, 0)
+    assert need > 0
+    assert lib.attn_fwd_ex_workspace_size(1, 2, 8, 8, 64, 0, 0.0, 0) == 0
+    # workspace missing / too small
+    assert lib.attn_fwd_ex(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0.1, 1, 0, 10000.0, 0, None, 0, None) == 5
+    assert lib.attn_fwd_ex(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0.1, 1, 0, 10000.0, 0, P, need - 1, None) == 5
+    assert lib.attn_fwd_ex(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0.1, 1, 0, 10000.0, -1, P, need, None) == 1
+
+
+def test_decode_validation(lib):
+    P = FAKE
+    need = lib.attn_decode_workspace_size(2, 8, 64, 4)
+    assert need >= 2 * 8 * 4 * 64 * 4 + 2 * 8 * 4 * 4
+    call = lambda **kw: lib.attn_decode(P, P, P, P, P, None, kw.get("B", 2), kw.get("Hq", 8), kw.get("Hkv", 2),
+                                        kw.get("Smax", 100), kw.get("D", 64), kw.get("scale", 0.125),
+                                        kw.get("ns", 4), kw.get("ws", P), kw.get("wsb", need),
+                                        kw.get("dtype", 0), None)
+    assert call(Smax=0) == 3
+    assert call(Hq=6, Hkv=4) == 2
+    assert call(ns=0) == 1
+    assert call(wsb=need - 1) == 5
+    assert call(ws=None) == 5
+    assert call(dtype=1) == 4
+    assert call(D=80) == 4
+
+
+def test_rope_validation(lib):
+    P = FAKE
+    assert lib.rope_apply(P, P, 4, 2, 7, 10000.0, 0, None) == 2      # odd head dim
+    assert lib.rope_apply(P, P, 0, 2, 8, 10000.0, 0, None) == 1
+    assert lib.rope_apply(P, P, 4, 2, 8, -1.0, 0, None) == 1
+
+
+def test_status_strings(lib):
+    for s in range(8):
+        assert lib.attn_status_string(s).decode() == ea.STATUS[s]
