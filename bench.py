@@ -1,0 +1,417 @@
+"""Benchmark of the exact-attention hot path on B200.
+
+Default workload (one GPU): MHA causal prefill, bf16 inputs / fp32 accumulation, B=4, Hq=Hkv=8,
+S=2048, D=64, scale 1/8 (synthetic N(0,1) inputs).  A step is one attn_fwd call over that batch.
+The same JSON line carries a secondary measurement of the split-KV decode path (B=16, Hq=32,
+Hkv=8, D=64, KV cache Smax=32768 with lengths uniform in [1024, 32768]) in KV-read GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
+
+--impl reference times the fp64 CPU oracle (the deliberately slow reference definition) on a
+bounded sample of the same workload, on this machine's host cores.
+
+Multi-GPU (launched by torch.distributed.run): the path has no exchange step, so each rank runs an
+independent replica of the workload on its own GPU ("replicas only"); value = work of all ranks
+divided by the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import seeded_inputs as si  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s & decode KV-read GB/s, % of B200 roofline"
+L2_FLUSH_BYTES = 256 << 20          # > 126 MB of L2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ------------------------------------------------------------------------------------------
+# ranks
+# ------------------------------------------------------------------------------------------
+
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Maximum of a per-rank scalar over all ranks (identity on one rank)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        import torch
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _query(self):
+        out = subprocess.run(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
+                              "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
+        return [x.strip() for x in out.stdout.strip().split(",")]
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._query())
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+        if not self.samples:
+            try:
+                self.samples.append(self._query())
+            except Exception:
+                pass
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        reasons = set()
+        for s in self.samples:
+            for name, val in zip(self.NAMES, s[2:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------
+# peaks and profile evidence
+# ------------------------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profile_traffic(name: str):
+    """Per-launch DRAM bytes recorded in profiles/<name>.md ('traffic_bytes_per_launch: N'), if the
+    summary is current; None otherwise."""
+    p = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        if line.strip().startswith("traffic_bytes_per_launch:"):
+            v = line.split(":", 1)[1].strip()
+            return None if v in ("null", "") else float(v)
+    return None
+
+
+# ------------------------------------------------------------------------------------------
+# GPU measurement
+# ------------------------------------------------------------------------------------------
+
+def dev_bf16(bits, torch):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def time_steps(fn, steps, warmup, flush, torch, dist, device):
+    """W untimed warm-up steps, then K steps each bracketed by CUDA events on the launching
+    stream, L2 flushed before each (outside the events).  Returns per-step ms (this rank)."""
+    for _ in range(warmup):
+        flush()
+        fn()
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def bench_prefill_gpu(w: si.Prefill, args, torch, ea, dist, device):
+    x = si.prefill_inputs(w)
+    q, k, v = (dev_bf16(x[n + "_bits"], torch) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
+    ws = None
+    if w.rope_base > 0:
+        ws = torch.empty(ea.fwd_workspace_bytes(q, k, w.rope_base, w.q_pos0), dtype=torch.uint8, device=device)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def step():
+        ea.attn_fwd_ex(q, k, v, w.scale, w.causal, w.rope_base, w.q_pos0, o=o, lse=lse, workspace=ws)
+
+    def flush():
+        flush_buf.zero_()
+
+    launches_per_step = 1 if w.rope_base <= 0 else 3
+    with ClockSampler(device.index) as clk:
+        ms = time_steps(step, args.steps, args.warmup, flush, torch, dist, device)
+    status = ea.read_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    mean_ms = statistics.mean(ms)
+
+    # end to end through the public API: pinned host inputs -> device -> attn -> host output
+    hq, hk, hv = (torch.from_numpy(np.ascontiguousarray(x[n + "_bits"]).view(np.int16)).view(torch.bfloat16)
+                  .pin_memory() for n in ("q", "k", "v"))
+    ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def step_e2e():
+        dq, dk, dv = (t.to(device, non_blocking=True) for t in (hq, hk, hv))
+        oo, ll = ea.attn_fwd_ex(dq, dk, dv, w.scale, w.causal, w.rope_base, w.q_pos0, workspace=ws)
+        ho.copy_(oo, non_blocking=True)
+        hl.copy_(ll, non_blocking=True)
+
+    ms_e2e = time_steps(step_e2e, max(3, args.steps // 4), args.warmup, flush, torch, dist, device)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+    return {"ms": mean_ms, "ms_list": ms, "clocks": clk.summary(), "ms_e2e": statistics.mean(ms_e2e),
+            "h2d": h2d, "d2h": d2h, "launches_per_step": launches_per_step}
+
+
+def bench_decode_gpu(w: si.Decode, args, torch, ea, dist, device, steps=None):
+    d = si.decode_inputs(w, fill_tail_nan=False)
+    q, kc, vc = (dev_bf16(d[n], torch) for n in ("q_bits", "k_bits", "v_bits"))
+    sl = torch.from_numpy(d["seqlens"]).to(device)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
+    ws = torch.empty(ea.decode_workspace_bytes(w.B, w.Hq, w.D, w.num_splits), dtype=torch.uint8, device=device)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def step():
+        ea.attn_decode(q, kc, vc, sl, w.scale, w.num_splits, o=o, lse=lse, workspace=ws)
+
+    ms = time_steps(step, steps or args.steps, args.warmup, lambda: flush_buf.zero_(), torch, dist, device)
+    if ea.read_device_status() != 0:
+        raise RuntimeError("device status set after decode timing")
+    kv_bytes = si.decode_kv_bytes(d["seqlens"], w.Hkv, w.D)
+    return {"ms": statistics.mean(ms), "kv_bytes": kv_bytes,
+            "qo_bytes": 2 * w.B * w.Hq * w.D * 2 + 4 * w.B * w.Hq}
+
+
+def cpu_baseline_prefill(w: si.Prefill, max_seconds: float = 30.0):
+    """The fp64 oracle on a bounded sample of the workload's rows (all (b, h), every r-th row)."""
+    import oracle
+    x = si.prefill_inputs(w)
+    stride = 1
+    # size the sample so that the oracle runs roughly 5-30 s: start with 1/16 of the rows
+    for stride in (16, 4, 1):
+        rows = np.arange(0, w.B * w.Hq * w.Sq, stride, dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.rope_base, w.q_pos0, rows=rows)
+        dt = time.perf_counter() - t0
+        if dt * 4 > max_seconds or stride == 1:
+            break
+    i = rows % w.Sq
+    off = w.Skv - w.Sq
+    vis = np.clip(i + off + 1, 0, w.Skv) if w.causal else np.full_like(i, w.Skv)
+    flops = float(np.sum(4.0 * w.D * vis))
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"{len(rows)} of {w.B * w.Hq * w.Sq} query rows (every {stride}th row of every "
+                      f"(batch, head)), {flops / 1e9:.2f} GFLOP fp64 in {dt:.2f} s"}
+
+
+def roofline_prefill(w: si.Prefill, ms: float, peaks, how: str, traffic):
+    achieved = w.flops / (ms * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "peak_source": f"{how} bf16_tflops (burst, cuBLAS bf16 GEMM)",
+            "kernel": "prefill_tc_kernel", "algorithmic_flop_per_launch": w.flops}
+
+
+def roofline_decode(dec, peaks, how: str):
+    achieved = dec["kv_bytes"] / (dec["ms"] * 1e-3) / 1e9
+    peak = float(peaks["hbm_gbs"])
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"{how} hbm_gbs (copy)",
+            "algorithmic_bytes_per_call": dec["kv_bytes"]}
+
+
+# ------------------------------------------------------------------------------------------
+# arms
+# ------------------------------------------------------------------------------------------
+
+def run_gpu(args):
+    import torch
+    rank, world, local = dist_env()
+    assert torch.cuda.is_available(), "bench.py needs CUDA devices (use --impl reference for the CPU oracle)"
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    from exact_attention_160_b200 import build as b
+    if rank == 0:
+        b.build()
+    barrier(dist, device)
+    import exact_attention_160_b200 as ea
+    ea.load_library()
+
+    w = si.WORKLOADS[args.workload]
+    peaks, how = load_peaks()
+    if isinstance(w, si.Prefill):
+        r = bench_prefill_gpu(w, args, torch, ea, dist, device)
+        ms = max_over_ranks(r["ms"], dist, device)
+        ms_e2e = max_over_ranks(r["ms_e2e"], dist, device)
+        value = world * w.flops / (ms * 1e-3) / 1e12
+        value_e2e = world * w.flops / (ms_e2e * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        dec_w = si.C4
+        dec = bench_decode_gpu(dec_w, args, torch, ea, dist, device, steps=max(5, args.steps // 2))
+        dec_ms = max_over_ranks(dec["ms"], dist, device)
+        dec["ms"] = dec_ms
+        roof = roofline_prefill(w, r["ms"], peaks, how, profile_traffic("prefill_tc_" + w.name.split("_")[0]))
+        extra = {"decode": {"workload": dec_w.name, "value": round(world * dec["kv_bytes"] / (dec_ms * 1e-3) / 1e9, 1),
+                            "unit": "GB/s", "ms_per_call": round(dec_ms, 4),
+                            "roofline": roofline_decode(dec, peaks, how)}}
+        clocks = r["clocks"]
+        e2e = {"value": round(value_e2e, 3), "unit": unit, "h2d_bytes_per_step": r["h2d"],
+               "d2h_bytes_per_step": r["d2h"], "ms_per_step": round(ms_e2e, 4)}
+        launches = r["launches_per_step"] * args.steps
+        config = {"workload": w.name, "global_batch": w.B * world, "seq_len": w.Sq, "heads_q": w.Hq,
+                  "heads_kv": w.Hkv, "head_dim": w.D, "causal": w.causal, "rope_base": w.rope_base,
+                  "parallelism": f"replicas{world}", "l2": "flushed before every timed step",
+                  "inputs": "seeded synthetic N(0,1) rounded to bf16 (seeded_inputs)"}
+    else:
+        with ClockSampler(device.index) as clk:
+            dec = bench_decode_gpu(w, args, torch, ea, dist, device)
+        ms = max_over_ranks(dec["ms"], dist, device)
+        dec["ms"] = ms
+        value = world * dec["kv_bytes"] / (ms * 1e-3) / 1e9
+        unit = "GB/s"
+        roof = roofline_decode(dec, peaks, how)
+        roof["traffic"] = profile_traffic("decode_split_" + w.name.split("_")[0])
+        extra = {}
+        clocks = clk.summary()
+        e2e = None
+        launches = 2 * args.steps
+        config = {"workload": w.name, "global_batch": w.B * world, "heads_q": w.Hq, "heads_kv": w.Hkv,
+                  "head_dim": w.D, "smax": w.Smax, "num_splits": w.num_splits,
+                  "parallelism": f"replicas{world}", "l2": "flushed before every timed step (cache > L2)"}
+
+    out = {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config, "roofline": roof,
+           "clocks": clocks, "gpu_launches": launches}
+    if e2e is not None:
+        out["e2e"] = e2e
+    out.update(extra)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and isinstance(w, si.Prefill):
+        out["cpu_baseline"] = cpu_baseline_prefill(w)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        barrier(dist, device)
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = si.WORKLOADS[args.workload]
+    if not isinstance(w, si.Prefill):
+        raise SystemExit("the reference arm times prefill workloads")
+    x = si.prefill_inputs(w)
+    # each step: every 64th query row of every (batch, head) -- a bounded slice of the workload
+    rows = np.arange(0, w.B * w.Hq * w.Sq, 64, dtype=np.int64)
+    i = rows % w.Sq
+    vis = np.clip(i + (w.Skv - w.Sq) + 1, 0, w.Skv) if w.causal else np.full_like(i, w.Skv)
+    flops = float(np.sum(4.0 * w.D * vis))
+    for _ in range(args.warmup):
+        oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.rope_base, w.q_pos0, rows=rows)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.rope_base, w.q_pos0, rows=rows)
+    dt = (time.perf_counter() - t0) / args.steps
+    value = flops / dt / 1e12
+    threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    sample = f"{len(rows)} query rows per step (every 64th row of every (batch, head)), {flops / 1e9:.3f} GFLOP fp64"
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.Sq, "parallelism": "cpu"},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default=si.C2.name, choices=sorted(si.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

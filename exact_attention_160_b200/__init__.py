@@ -30,7 +30,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 
 # symbols the library exports (kept in step with include/attn_b200.h)
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
-           "attn_decode_workspace_size", "rope_apply", "attn_status_string",
+           "attn_decode_workspace_size", "rope_apply", "attn_status_string", "attn_last_error",
            "attn_read_device_status")
 
 _lib = None
@@ -39,7 +39,10 @@ _lib = None
 class AttnError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {STATUS.get(status, status)} (status {status})")
+        detail = ""
+        if status == 6 and _lib is not None:
+            detail = " -- " + _lib.attn_last_error().decode(errors="replace")
+        super().__init__(f"{what}: {STATUS.get(status, status)} (status {status}){detail}")
 
 
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
@@ -62,6 +65,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_status_string.argtypes = [I]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_read_device_status.argtypes = [P]
+    lib.attn_last_error.argtypes = []
+    lib.attn_last_error.restype = ctypes.c_char_p
     for f in (lib.attn_fwd, lib.attn_fwd_ex, lib.attn_decode, lib.rope_apply, lib.attn_read_device_status):
         f.restype = I
     _lib = lib

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
+#include <stdio.h>
 #include <string.h>
 
 #include <mutex>
@@ -18,6 +19,14 @@
 using namespace attn;
 
 namespace {
+
+// Description of the most recent ATTN_ERR_CUDA of the calling thread.
+thread_local char g_last_error[256] = "";
+
+attn_status cuda_failure(const char* what, const char* detail) {
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", what, detail);
+    return ATTN_ERR_CUDA;
+}
 
 // ------------------------------------------------------------------------------------------
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda)
@@ -43,7 +52,10 @@ EncodeTiledFn encode_fn() {
 // 128-byte swizzle (the UMMA SW128 K-major / MN-major operand layout).  Rows past S read as 0.
 bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D) {
     EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
+    if (!enc) {
+        cuda_failure("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", "entry point unavailable");
+        return false;
+    }
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
     cuuint32_t box[4] = {64, 1, 128, 1};
@@ -51,15 +63,23 @@ bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D)
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char buf[96];
+        snprintf(buf, sizeof(buf), "CUresult %d (dims %d,%d,%d,%d)", static_cast<int>(r), D, H, S, B);
+        cuda_failure("cuTensorMapEncodeTiled", buf);
+    }
     return r == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-attn_status launch_status() {
-    return cudaPeekAtLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+// Status of the launch just made (clears the runtime's launch error so it is not reported twice).
+attn_status launch_status(const char* what) {
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? ATTN_OK : cuda_failure(what, cudaGetErrorString(e));
 }
 
 attn_status check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal) {
@@ -99,7 +119,7 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     CUtensorMap tq, tk, tkl, tv;
     if (!make_tmap_bshd(&tq, q, B, Sq, Hq, D) || !make_tmap_bshd(&tk, k, B, Skv, Hkv, D) ||
         !make_tmap_bshd(&tv, v, B, Skv, Hkv, D) || !make_tmap_bshd(&tkl, ROPE ? klo : k, B, Skv, Hkv, D))
-        return ATTN_ERR_CUDA;
+        return ATTN_ERR_CUDA;   // g_last_error set by make_tmap_bshd
     using C = TcCfg<D, ROPE>;
     TcParams p{};
     p.o = static_cast<__nv_bfloat16*>(o);
@@ -118,12 +138,24 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     auto kern = prefill_tc_kernel<D, ROPE>;
     static bool attr_set = false;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-            return ATTN_ERR_CUDA;
+        // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds
+        // fewer than the split asks for would stall in setmaxnreg.inc, so refuse it.
+        cudaFuncAttributes fa;
+        cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+        if (e != cudaSuccess) return cuda_failure("cudaFuncGetAttributes(prefill_tc_kernel)", cudaGetErrorString(e));
+        if (fa.numRegs < kTcLaunchRegsMin) {
+            char buf[96];
+            snprintf(buf, sizeof(buf), "compiled with %d registers per thread, the warpgroup split needs %d",
+                     fa.numRegs, kTcLaunchRegsMin);
+            cuda_failure("prefill_tc_kernel register budget", buf);
+            return ATTN_ERR_UNSUPPORTED;
+        }
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(prefill_tc_kernel)", cudaGetErrorString(e));
         attr_set = true;
     }
     kern<<<static_cast<unsigned>(grid), kTcThreads, C::SMEM_BYTES, st>>>(tq, tk, tkl, tv, p);
-    return launch_status();
+    return launch_status("prefill_tc_kernel");
 }
 
 template <int D>
@@ -133,9 +165,8 @@ attn_status launch_f32(const void* q, const void* k, const void* v, void* o, flo
     auto kern = prefill_f32_kernel<D>;
     static bool attr_set = false;
     if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-            cudaSuccess)
-            return ATTN_ERR_CUDA;
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(prefill_f32_kernel)", cudaGetErrorString(e));
         attr_set = true;
     }
     dim3 grid((Sq + 63) / 64, Hq, B);
@@ -143,7 +174,7 @@ attn_status launch_f32(const void* q, const void* k, const void* v, void* o, flo
     kern<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
                                   static_cast<const float*>(v), static_cast<float*>(o), lse, Hq, Hkv, Sq, Skv, scale,
                                   causal, tab, q_pos0);
-    return launch_status();
+    return launch_status("prefill_f32_kernel");
 }
 
 attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
@@ -169,7 +200,7 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
         const long n = static_cast<long>(w.positions) * (D / 2);
         rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, st>>>(
             t, w.positions, D, static_cast<double>(rope_base));
-        if ((s = launch_status()) != ATTN_OK) return s;
+        if ((s = launch_status("rope_table_kernel")) != ATTN_OK) return s;
         tab = t;
     }
 
@@ -187,7 +218,7 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
     const long npairs = static_cast<long>(B) * Skv * Hkv * (D / 2);
     rope_split_kv_kernel<<<static_cast<unsigned>((npairs + 255) / 256 < 148 * 64 ? (npairs + 255) / 256 : 148 * 64), 256,
                            0, st>>>(static_cast<const uint32_t*>(k), khi, klo, tab, npairs, Skv, Hkv, D);
-    if ((s = launch_status()) != ATTN_OK) return s;
+    if ((s = launch_status("rope_split_kv_kernel")) != ATTN_OK) return s;
     return D == 64 ? launch_tc<64, true>(q, khi, klo, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st)
                    : launch_tc<128, true>(q, khi, klo, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st);
 }
@@ -205,13 +236,13 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kc),
         static_cast<const __nv_bfloat16*>(vc), seqlens, o_part, lse_part, Hkv, G, Smax, num_splits,
         scale * 1.4426950408889634f);
-    attn_status s = launch_status();
+    attn_status s = launch_status("decode_split_kernel");
     if (s != ATTN_OK) return s;
     const int warps = B * Hq;
     decode_combine_kernel<D><<<(warps + 3) / 4, 128, 0, st>>>(o_part, lse_part, seqlens,
                                                                static_cast<__nv_bfloat16*>(o), lse, B, Hq, Smax,
                                                                num_splits);
-    return launch_status();
+    return launch_status("decode_combine_kernel");
 }
 
 }  // namespace
@@ -295,8 +326,10 @@ attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float b
     else
         rope_apply_kernel<float><<<grid, 128, smem, st>>>(static_cast<float*>(x), pos, T, H, D,
                                                           static_cast<double>(base));
-    return launch_status();
+    return launch_status("rope_apply_kernel");
 }
+
+const char* attn_last_error(void) { return g_last_error; }
 
 const char* attn_status_string(attn_status s) {
     switch (s) {

@@ -12,11 +12,11 @@
 //   * One CTA holds two 128-row query tiles that read the same K/V: two q heads of one GQA group
 //     at the same rows when the group size is even, else two consecutive row tiles of one head.
 //     Each K/V tile is therefore loaded once for 256 query rows.
-//   * Warp roles (10 warps): warp 0 issues TMA loads (Q once, then a ring of K/V stages);
-//     warp 1 owns tensor memory and issues every tcgen05.mma from one thread; warps 2-5 and
-//     6-9 are the softmax warpgroups of query tile 0 and 1, one thread per query row.  A warp
+//   * Warp roles (3 warpgroups): warp 0 issues TMA loads (Q once, then a ring of K/V stages);
+//     warp 1 owns tensor memory and issues every tcgen05.mma from one thread; warps 4-7 and
+//     8-11 are the softmax warpgroups of query tile 0 and 1, one thread per query row (a warp
 //     may only touch TMEM lanes 32*(warp%4) .. +31, so the row of a softmax thread is
-//     32*(warp%4) + lane: each group of four consecutive warps covers all 128 lanes.
+//     32*(warp%4) + lane).
 //   * S = Q K^T is a bf16 MMA (A and B from shared memory, M=128, N=128) into TMEM; the softmax
 //     threads read their row of S with tcgen05.ld, compute P = exp2(S*scale*log2e - m) in fp32,
 //     round P to bf16 and write it back to TMEM; O += P V is an MMA with A = P from TMEM and
@@ -37,7 +37,15 @@
 
 namespace attn {
 
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 384;
+// Register split between the warpgroups (setmaxnreg): the TMA/MMA warpgroup gives registers up,
+// the two softmax warpgroups take them.  The launch must provide kTcThreads * kTcLaunchRegsMin
+// registers, which covers 128 * kRegsControl + 256 * kRegsSoftmax; the host checks the compiled
+// register count before every launch.  Per sub-partition (warps w, w+4, w+8 share one):
+// (64 + 2 * 208) * 32 = 15360 <= 16384 registers.
+constexpr int kRegsControl = 64;
+constexpr int kRegsSoftmax = 208;
+constexpr int kTcLaunchRegsMin = (128 * kRegsControl + 256 * kRegsSoftmax + kTcThreads - 1) / kTcThreads;
 constexpr float kRescaleThreshold = 8.0f;
 constexpr float kLn2 = 0.69314718055994531f;
 
@@ -94,7 +102,7 @@ __device__ __forceinline__ int tc_kv_tiles(const TcParams& p, int r0) {
 }
 
 template <int D, bool ROPE>
-__global__ void __maxnreg__(200) prefill_tc_kernel(
+__global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
     const TcParams p) {
@@ -145,7 +153,7 @@ __global__ void __maxnreg__(200) prefill_tc_kernel(
     // ---- set-up --------------------------------------------------------------------------
     if (tid == 0) {
         mbar_init(bar_q_full, 1);
-        mbar_init(bar_q_ready, 256);
+        mbar_init(bar_q_ready, 256);   // both softmax warpgroups
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_s_full + i, 1);
             mbar_init(bar_p_ready + i, 128);
@@ -174,7 +182,9 @@ __global__ void __maxnreg__(200) prefill_tc_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      setmaxnreg_dec<kRegsControl>();
+      if (warp == 0) {
         // =============================== TMA producer ===================================
         if (lane == 0) {
             const uint64_t pol_q = l2_policy_evict_first();
@@ -220,7 +230,7 @@ __global__ void __maxnreg__(200) prefill_tc_kernel(
                 mbar_wait(bar_v_full + j % C::STAGES, (j / C::STAGES) & 1);
             }
         }
-    } else if (warp == 1) {
+      } else if (warp == 1) {
         // =============================== MMA issuer ======================================
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
@@ -285,9 +295,11 @@ __global__ void __maxnreg__(200) prefill_tc_kernel(
             mma_commit(bar_mma_final);
             mbar_wait(bar_mma_final, 0);
         }
+      }
     } else {
+        setmaxnreg_inc<kRegsSoftmax>();
         // =============================== softmax warpgroups =============================
-        const int wg = (warp - 2) >> 2;             // query tile index
+        const int wg = (warp - 4) >> 2;             // query tile index
         const int row = (warp & 3) * 32 + lane;     // 0..127 == TMEM lane
         TcTile T;
         T.h = wg ? tile[1].h : tile[0].h;

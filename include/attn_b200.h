@@ -130,6 +130,10 @@ attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float b
 /* Static description of a status code.                                                     */
 const char* attn_status_string(attn_status s);
 
+/* Which call failed, and the CUDA error text, for the calling thread's most recent
+ * ATTN_ERR_CUDA ("" if none).  The string stays valid until that thread's next failure.     */
+const char* attn_last_error(void);
+
 /*
  * Read and clear the device status word (bit 1: a bounded wait gave up; bit 2: a decode
  * sequence length was clamped; bit 4: tensor memory allocation failed).  Synchronises

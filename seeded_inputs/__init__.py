@@ -173,20 +173,20 @@ def prefill_inputs(w: Prefill):
     return out
 
 
-def decode_inputs(w: Decode, fill_tail_nan: bool = True):
+def decode_inputs(w: Decode, fill_tail_nan: bool = True, seqlens=None):
     """q [B,Hq,D]; kcache/vcache [B,Smax,Hkv,D] bf16; seqlens int32 [B].
 
     Cache rows at positions >= seqlens[b] are never part of the attention; they
     hold bf16 NaN (``fill_tail_nan``) so that any read past a sequence's end
-    poisons the output.
+    poisons the output.  ``seqlens`` overrides the workload's drawn lengths.
     """
-    seqlens = w.seqlens()
+    seqlens = w.seqlens() if seqlens is None else np.asarray(seqlens, dtype=np.int32)
     q_bits, q = bf16_normal(w.seed, STREAM_Q, (w.B, w.Hq, w.D))
     fill = BF16_NAN_BITS if fill_tail_nan else 0
     kb = np.full((w.B, w.Smax, w.Hkv, w.D), fill, dtype=np.uint16)
     vb = np.full((w.B, w.Smax, w.Hkv, w.D), fill, dtype=np.uint16)
     for b in range(w.B):
-        L = int(seqlens[b])
+        L = int(min(max(seqlens[b], 0), w.Smax))
         kb[b, :L] = bf16_normal(w.seed, STREAM_KCACHE_BASE + b, (L, w.Hkv, w.D))[0]
         vb[b, :L] = bf16_normal(w.seed, STREAM_VCACHE_BASE + b, (L, w.Hkv, w.D))[0]
     return {"q_bits": q_bits, "q": q, "k_bits": kb, "v_bits": vb, "seqlens": seqlens}

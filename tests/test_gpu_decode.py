@@ -13,9 +13,7 @@ pytestmark = pytest.mark.gpu
 
 
 def run_decode(w: si.Decode, num_splits=None, seqlens=None):
-    d = si.decode_inputs(w)
-    if seqlens is not None:
-        d["seqlens"] = np.asarray(seqlens, dtype=np.int32)
+    d = si.decode_inputs(w, seqlens=seqlens)
     q = bits_to_dev(d["q_bits"])
     kc = bits_to_dev(d["k_bits"])
     vc = bits_to_dev(d["v_bits"])
