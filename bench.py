@@ -188,7 +188,8 @@ def time_steps(fn, steps, warmup, flush, torch, dist, device):
 def bench_prefill_gpu(w: si.Prefill, args, torch, ea, dist, device):
     x = si.prefill_inputs(w)
     q, k, v = (dev_bf16(x[n + "_bits"], torch) for n in ("q", "k", "v"))
-    o = torch.empty_like(q)
+    # bf16 inputs, fp32 accumulation, O taken in fp32: the configuration the parity tests check
+    o = torch.empty(q.shape, dtype=torch.float32, device=device)
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
     ws = None
     if w.rope_base > 0:
@@ -217,7 +218,8 @@ def bench_prefill_gpu(w: si.Prefill, args, torch, ea, dist, device):
 
     def step_e2e():
         dq, dk, dv = (t.to(device, non_blocking=True) for t in (hq, hk, hv))
-        oo, ll = ea.attn_fwd_ex(dq, dk, dv, w.scale, w.causal, w.rope_base, w.q_pos0, workspace=ws)
+        oo, ll = ea.attn_fwd_ex(dq, dk, dv, w.scale, w.causal, w.rope_base, w.q_pos0, workspace=ws,
+                                out_dtype=torch.float32)
         ho.copy_(oo, non_blocking=True)
         hl.copy_(ll, non_blocking=True)
 
@@ -232,7 +234,7 @@ def bench_decode_gpu(w: si.Decode, args, torch, ea, dist, device, steps=None):
     d = si.decode_inputs(w, fill_tail_nan=False)
     q, kc, vc = (dev_bf16(d[n], torch) for n in ("q_bits", "k_bits", "v_bits"))
     sl = torch.from_numpy(d["seqlens"]).to(device)
-    o = torch.empty_like(q)
+    o = torch.empty(q.shape, dtype=torch.float32, device=device)
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
     ws = torch.empty(ea.decode_workspace_bytes(w.B, w.Hq, w.D, w.num_splits), dtype=torch.uint8, device=device)
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)

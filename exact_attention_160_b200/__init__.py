@@ -23,7 +23,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
 
-ATTN_BF16, ATTN_FP32 = 0, 1
+ATTN_BF16, ATTN_FP32, ATTN_BF16_OUT_F32 = 0, 1, 2
 STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV",
           4: "unsupported configuration", 5: "workspace missing or too small", 6: "CUDA error",
           7: "device wait timed out"}
@@ -82,10 +82,17 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _dtype_code(t: torch.Tensor) -> int:
+def _dtype_code(t: torch.Tensor, o: torch.Tensor = None) -> int:
+    """dtype code of the C ABI: inputs' storage type, and for bf16 inputs the output's."""
     if t.dtype == torch.bfloat16:
+        if o is not None and o.dtype == torch.float32:
+            return ATTN_BF16_OUT_F32
+        if o is not None and o.dtype != torch.bfloat16:
+            raise TypeError(f"unsupported output dtype {o.dtype}")
         return ATTN_BF16
     if t.dtype == torch.float32:
+        if o is not None and o.dtype != torch.float32:
+            raise TypeError("fp32 inputs take an fp32 output")
         return ATTN_FP32
     raise TypeError(f"unsupported dtype {t.dtype}")
 
@@ -101,9 +108,12 @@ def _need_cuda(*ts):
             raise ValueError("tensors must be contiguous CUDA tensors")
 
 
-def attn_fwd(q, k, v, scale: float, causal: bool, o=None, lse=None, want_lse: bool = True, stream=None):
-    """Exact attention forward.  Returns (o, lse); lse is None when want_lse is False."""
-    return attn_fwd_ex(q, k, v, scale, causal, 0.0, 0, o=o, lse=lse, want_lse=want_lse, stream=stream)
+def attn_fwd(q, k, v, scale: float, causal: bool, o=None, lse=None, want_lse: bool = True, out_dtype=None,
+             stream=None):
+    """Exact attention forward.  Returns (o, lse); lse is None when want_lse is False.
+    out_dtype: torch.float32 to take a bf16 problem's output in fp32 (default: q's dtype)."""
+    return attn_fwd_ex(q, k, v, scale, causal, 0.0, 0, o=o, lse=lse, want_lse=want_lse, out_dtype=out_dtype,
+                       stream=stream)
 
 
 def fwd_workspace_bytes(q, k, rope_base: float, q_pos0: int) -> int:
@@ -114,14 +124,14 @@ def fwd_workspace_bytes(q, k, rope_base: float, q_pos0: int) -> int:
 
 
 def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: int = 0, o=None, lse=None,
-                want_lse: bool = True, workspace=None, stream=None):
+                want_lse: bool = True, workspace=None, out_dtype=None, stream=None):
     """Exact attention forward with RoPE on Q (positions q_pos0 + i) and K (positions j)."""
     lib = load_library()
     _need_cuda(q, k, v, o, lse, workspace)
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     ws_bytes = 0
@@ -132,12 +142,12 @@ def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: i
         ws_bytes = workspace.numel() * workspace.element_size()
     if rope_base > 0:
         st = lib.attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
-                             float(scale), int(bool(causal)), _dtype_code(q), float(rope_base), int(q_pos0),
+                             float(scale), int(bool(causal)), _dtype_code(q, o), float(rope_base), int(q_pos0),
                              _ptr(workspace), ws_bytes, _stream(stream))
         _check(st, "attn_fwd_ex")
     else:
         st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
-                          float(scale), int(bool(causal)), _dtype_code(q), _stream(stream))
+                          float(scale), int(bool(causal)), _dtype_code(q, o), _stream(stream))
         _check(st, "attn_fwd")
     return o, lse
 
@@ -147,14 +157,14 @@ def decode_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
 
 
 def attn_decode(q, kcache, vcache, seqlens, scale: float, num_splits: int, o=None, lse=None,
-                want_lse: bool = True, workspace=None, stream=None):
+                want_lse: bool = True, workspace=None, out_dtype=None, stream=None):
     """Split-KV decode of one token per (sequence, q head).  Returns (o, lse)."""
     lib = load_library()
     _need_cuda(q, kcache, vcache, seqlens, o, lse, workspace)
     B, Hq, D = q.shape
     Smax, Hkv = kcache.shape[1], kcache.shape[2]
     if o is None:
-        o = torch.empty_like(q)
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     need = decode_workspace_bytes(B, Hq, D, num_splits)
@@ -162,7 +172,7 @@ def attn_decode(q, kcache, vcache, seqlens, scale: float, num_splits: int, o=Non
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     st = lib.attn_decode(_ptr(q), _ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(o), _ptr(lse), B, Hq, Hkv,
                          Smax, D, float(scale), int(num_splits), _ptr(workspace),
-                         workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream))
+                         workspace.numel() * workspace.element_size(), _dtype_code(q, o), _stream(stream))
     _check(st, "attn_decode")
     return o, lse
 

@@ -106,15 +106,15 @@ ExWorkspace ex_workspace(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtyp
     w.tab_off = 0;
     size_t tab = static_cast<size_t>(w.positions) * (D / 2) * sizeof(float2);
     w.khi_off = round_up(tab, 256);
-    size_t kbytes = dtype == ATTN_BF16 ? static_cast<size_t>(B) * Skv * Hkv * D * 2 : 0;
+    size_t kbytes = dtype != ATTN_FP32 ? static_cast<size_t>(B) * Skv * Hkv * D * 2 : 0;
     w.klo_off = round_up(w.khi_off + kbytes, 256);
     w.total = round_up(w.klo_off + kbytes, 256);
     return w;
 }
 
 template <int D, bool ROPE>
-attn_status launch_tc(const void* q, const void* k, const void* klo, const void* v, void* o, float* lse, int B,
-                      int Hq, int Hkv, int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0,
+attn_status launch_tc(const void* q, const void* k, const void* klo, const void* v, void* o, bool o_f32, float* lse,
+                      int B, int Hq, int Hkv, int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0,
                       cudaStream_t st) {
     CUtensorMap tq, tk, tkl, tv;
     if (!make_tmap_bshd(&tq, q, B, Sq, Hq, D) || !make_tmap_bshd(&tk, k, B, Skv, Hkv, D) ||
@@ -122,7 +122,8 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
         return ATTN_ERR_CUDA;   // g_last_error set by make_tmap_bshd
     using C = TcCfg<D, ROPE>;
     TcParams p{};
-    p.o = static_cast<__nv_bfloat16*>(o);
+    p.o = o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o);
+    p.o_f32 = o_f32 ? static_cast<float*>(o) : nullptr;
     p.lse = lse;
     p.rope_tab = tab;
     p.B = B, p.Hq = Hq, p.Hkv = Hkv, p.Sq = Sq, p.Skv = Skv;
@@ -184,7 +185,8 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
     if (s != ATTN_OK) return s;
     if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
-    if (dtype != ATTN_BF16 && dtype != ATTN_FP32) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP32 && dtype != ATTN_BF16_OUT_F32) return ATTN_ERR_INVALID_ARG;
+    const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
     const bool rope = rope_base > 0.f;
     if (rope && !isfinite(rope_base)) return ATTN_ERR_INVALID_ARG;
     if (rope && q_pos0 < 0) return ATTN_ERR_INVALID_ARG;
@@ -209,8 +211,10 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
                        : launch_f32<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st);
     }
     if (!rope) {
-        return D == 64 ? launch_tc<64, false>(q, k, nullptr, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, nullptr, 0, st)
-                       : launch_tc<128, false>(q, k, nullptr, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, nullptr, 0, st);
+        return D == 64 ? launch_tc<64, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
+                                              nullptr, 0, st)
+                       : launch_tc<128, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
+                                               nullptr, 0, st);
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* khi = reinterpret_cast<uint32_t*>(ws + w.khi_off);
@@ -219,12 +223,15 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
     rope_split_kv_kernel<<<static_cast<unsigned>((npairs + 255) / 256 < 148 * 64 ? (npairs + 255) / 256 : 148 * 64), 256,
                            0, st>>>(static_cast<const uint32_t*>(k), khi, klo, tab, npairs, Skv, Hkv, D);
     if ((s = launch_status("rope_split_kv_kernel")) != ATTN_OK) return s;
-    return D == 64 ? launch_tc<64, true>(q, khi, klo, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st)
-                   : launch_tc<128, true>(q, khi, klo, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st);
+    return D == 64 ? launch_tc<64, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
+                                         q_pos0, st)
+                   : launch_tc<128, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
+                                          q_pos0, st);
 }
 
 template <int D, int GC>
-attn_status launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o, float* lse,
+attn_status launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o, bool o_f32,
+                          float* lse,
                           int B, int Hq, int Hkv, int Smax, float scale, int num_splits, float* o_part,
                           float* lse_part, cudaStream_t st) {
     constexpr int LPK = D / 8, SLOTS = 32 / LPK, NPART = kDecodeWarps * SLOTS;
@@ -239,9 +246,9 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
     attn_status s = launch_status("decode_split_kernel");
     if (s != ATTN_OK) return s;
     const int warps = B * Hq;
-    decode_combine_kernel<D><<<(warps + 3) / 4, 128, 0, st>>>(o_part, lse_part, seqlens,
-                                                               static_cast<__nv_bfloat16*>(o), lse, B, Hq, Smax,
-                                                               num_splits);
+    decode_combine_kernel<D><<<(warps + 3) / 4, 128, 0, st>>>(
+        o_part, lse_part, seqlens, o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
+        o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Hq, Smax, num_splits);
     return launch_status("decode_combine_kernel");
 }
 
@@ -284,7 +291,9 @@ attn_status attn_decode(const void* q, const void* kcache, const void* vcache, c
     if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
     if (!q || !kcache || !vcache || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
-    if (dtype != ATTN_BF16) return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_BF16_OUT_F32)
+        return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
     const size_t need = attn_decode_workspace_size(B, Hq, D, num_splits);
@@ -297,7 +306,7 @@ attn_status attn_decode(const void* q, const void* kcache, const void* vcache, c
     const int GC = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
 #define ATTN_DECODE_CASE(DD, GG)                                                                              \
     if (D == DD && GC == GG)                                                                                  \
-        return launch_decode<DD, GG>(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Smax, scale, num_splits, \
+        return launch_decode<DD, GG>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, \
                                      o_part, lse_part, st);
     ATTN_DECODE_CASE(64, 1)
     ATTN_DECODE_CASE(64, 2)

@@ -256,8 +256,8 @@ __global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part,
-    const int32_t* __restrict__ seqlens, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-    int B, int Hq, int Smax, int max_splits) {
+    const int32_t* __restrict__ seqlens, __nv_bfloat16* __restrict__ o, float* __restrict__ o_f32,
+    float* __restrict__ lse, int B, int Hq, int Smax, int max_splits) {
     constexpr int DPL = D / 32;   // dims per lane
     const int warp_global = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
@@ -289,10 +289,15 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
         }
     }
     const float inv = total > 0.f ? 1.f / total : 0.f;
-    __nv_bfloat16* orow = o + static_cast<long>(warp_global) * D + lane * DPL;
+    if (o_f32 != nullptr) {
+        float* orow = o_f32 + static_cast<long>(warp_global) * D + lane * DPL;
 #pragma unroll
-    for (int e = 0; e < DPL; e += 2) {
-        *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+        for (int e = 0; e < DPL; ++e) orow[e] = acc[e] * inv;
+    } else {
+        __nv_bfloat16* orow = o + static_cast<long>(warp_global) * D + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; e += 2)
+            *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
     }
     if (lse != nullptr && lane == 0) lse[warp_global] = total > 0.f ? M + logf(total) : -INFINITY;
 }

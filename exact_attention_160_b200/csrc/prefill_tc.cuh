@@ -73,7 +73,8 @@ struct TcCfg {
 };
 
 struct TcParams {
-    __nv_bfloat16* o;
+    __nv_bfloat16* o;         // bf16 output, or
+    float* o_f32;             // fp32 output (when non-null)
     float* lse;
     const float2* rope_tab;   // [positions][D/2] (cos, sin), ROPE only
     int B, Hq, Hkv, Sq, Skv;
@@ -356,7 +357,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         }
 
         float m_run = -INFINITY;   // running max used in the exponent (log2 units)
-        float l_run = 0.f;
+        float l_run = 0.f;         // row sum of the fp32 weights (logsumexp)
+        float l_mma = 0.f;         // row sum of the bf16-rounded weights (normalises O)
         const float sl2 = p.scale_log2;
         for (int j = 0; ok && j < T.nkv; ++j) {
             if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) { ok = false; break; }
@@ -381,7 +383,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
-                for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[cb][e]));
+                for (int e = 0; e < 32; e += 2)
+                    mx = max3(mx, __uint_as_float(sr[cb][e]), __uint_as_float(sr[cb][e + 1]));
             const float tmax = mx * sl2;
             // lazy rescale: move the exponent's max only when the block max exceeds it by > threshold
             const bool need = tmax > m_run + kRescaleThreshold;
@@ -406,33 +409,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 tmem_wait_st();
             }
             l_run *= corr;
+            l_mma *= corr;
             const float mu = (m_run == -INFINITY) ? 0.f : m_run;
             if (!C::P_ALIASES_S && j > 0) {
                 // P_i(j-1) must have been consumed by PV_i(j-1) before it is overwritten
                 if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) { ok = false; break; }
                 tc_fence_after();
             }
-            float lsum = 0.f;
+            // p = exp2(s*scale*log2e - mu) in fp32, rounded to bf16 for the PV MMA.  Two row sums:
+            // the exact one (for the logsumexp) and the sum of the rounded values the MMA uses
+            // (O is normalised by it, so the rounding of a dominant weight cancels).
+            uint64_t lt2 = 0, lr2 = 0;   // packed (even, odd) partial sums
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
+            const uint64_t nmux2 = f2_pack(-mu, -mu);
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(fmaf(__uint_as_float(sr[cb][2 * e]), sl2, -mu));
-                    const float p1 = fast_exp2(fmaf(__uint_as_float(sr[cb][2 * e + 1]), sl2, -mu));
-                    lsum += p0 + p1;
+                    float t0, t1;
+                    f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[cb][2 * e]), __uint_as_float(sr[cb][2 * e + 1])),
+                                     sl2x2, nmux2),
+                              t0, t1);
+                    const float p0 = fast_exp2(t0);
+                    const float p1 = fast_exp2(t1);
+                    lt2 = f2_add(lt2, f2_pack(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
+                    lr2 = f2_add(lr2, f2_pack(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                 }
                 tmem_st16(tP + cb * 16, pk);
             }
-            l_run += lsum;
+            {
+                float a, c;
+                f2_unpack(lt2, a, c);
+                l_run += a + c;
+                f2_unpack(lr2, a, c);
+                l_mma += a + c;
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p_ready + wg);
         }
 
-        // epilogue: O / l -> bf16, lse.  The TMEM reads are warp-collective, so every lane of
-        // the warp takes part; only rows inside [0, Sq) are stored.
+        // epilogue: O / l -> bf16 or fp32, lse.  The TMEM reads are warp-collective, so every
+        // lane of the warp takes part; only rows inside [0, Sq) are stored.
         if (T.active) {
             bool have = ok && T.nkv > 0;
             if (have) {
@@ -440,8 +460,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 tc_fence_after();
             }
             const bool store = qrow < p.Sq;
-            const float inv = (have && l_run > 0.f) ? 1.f / l_run : 0.f;
-            __nv_bfloat16* orow = p.o + ((static_cast<long>(b) * p.Sq + qrow) * p.Hq + T.h) * D;
+            const float inv = (have && l_mma > 0.f) ? 1.f / l_mma : 0.f;
+            const long orow_off = ((static_cast<long>(b) * p.Sq + qrow) * p.Hq + T.h) * D;
 #pragma unroll
             for (int cb = 0; cb < D / 32; ++cb) {
                 uint32_t orr[32];
@@ -452,12 +472,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
 #pragma unroll
                     for (int e = 0; e < 32; ++e) orr[e] = 0u;
                 }
-                uint32_t pk[16];
+                if (!store) continue;
+                if (p.o_f32) {
+                    float4* dst = reinterpret_cast<float4*>(p.o_f32 + orow_off + cb * 32);
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
-                if (store) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + cb * 32);
+                    for (int e = 0; e < 8; ++e)
+                        dst[e] = make_float4(__uint_as_float(orr[4 * e]) * inv, __uint_as_float(orr[4 * e + 1]) * inv,
+                                             __uint_as_float(orr[4 * e + 2]) * inv, __uint_as_float(orr[4 * e + 3]) * inv);
+                } else {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
+                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow_off + cb * 32);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);

@@ -57,8 +57,11 @@ typedef enum {
 } attn_status;
 
 typedef enum {
-    ATTN_BF16 = 0, /* q, k, v, o, x stored as bfloat16; fp32 accumulation                    */
-    ATTN_FP32 = 1  /* q, k, v, o, x stored as float32; fp32 arithmetic (no TF32)              */
+    ATTN_BF16 = 0,        /* q, k, v, o, x stored as bfloat16; fp32 accumulation              */
+    ATTN_FP32 = 1,        /* q, k, v, o, x stored as float32; fp32 arithmetic (no TF32)       */
+    ATTN_BF16_OUT_F32 = 2 /* q, k, v bfloat16; o written as float32 (attn_fwd*, attn_decode).
+                             bf16 storage of o has a spacing of 2^-6 at |o| >= 2, so callers
+                             that need o to better than that take it in float32.              */
 } attn_dtype;
 
 typedef void* attn_stream_t; /* a cudaStream_t */
@@ -67,12 +70,14 @@ typedef void* attn_stream_t; /* a cudaStream_t */
  * attn_fwd -- exact attention forward (prefill).
  *   q    [B, Sq, Hq, D]   dtype          read
  *   k, v [B, Skv, Hkv, D] dtype          read
- *   o    [B, Sq, Hq, D]   dtype          written
+ *   o    [B, Sq, Hq, D]   dtype (float32 with ATTN_BF16_OUT_F32)   written
  *   lse  [B, Hq, Sq]      float32        written; may be NULL (not produced)
  *   scale                  the score multiplier (commonly 1/sqrt(D)); must be finite and > 0
  *   causal                 0 or 1
  * Returns ATTN_OK, or INVALID_ARG / DIM_MISMATCH / EMPTY_KV / UNSUPPORTED / CUDA.
- * bf16 path: QK^T and PV on tcgen05 tensor cores, P rounded to bf16, fp32 accumulators.
+ * bf16 path: QK^T and PV on tcgen05 tensor cores, P rounded to bf16, fp32 accumulators; O is
+ * normalised by the sum of the rounded P values (the weights the PV product used) and lse by
+ * the fp32 sum.
  */
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                      int Hkv, int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype,
@@ -105,12 +110,13 @@ size_t attn_fwd_ex_workspace_size(int B, int Hkv, int Sq, int Skv, int D, attn_d
  *   vcache  [B, Smax, Hkv, D]   bf16    read
  *   seqlens [B]                 int32   read on the device; values outside [1, Smax] are
  *                                       clamped and flagged in the device status word
- *   o       [B, Hq, D]          bf16    written
+ *   o       [B, Hq, D]          bf16    written (float32 with ATTN_BF16_OUT_F32)
  *   lse     [B, Hq]             float32 written; may be NULL
  *   num_splits  upper bound on KV splits per sequence (>= 1); sequence b uses
  *               clamp(seqlens[b] / 512, 1, num_splits) contiguous near-equal splits
  *   workspace   device scratch of >= attn_decode_workspace_size(B, Hq, D, num_splits) bytes
- * No causal mask: the single new token sees the whole cache.  Only dtype ATTN_BF16.
+ * No causal mask: the single new token sees the whole cache.  dtype ATTN_BF16 or
+ * ATTN_BF16_OUT_F32 (ATTN_FP32 returns ATTN_ERR_UNSUPPORTED).
  */
 attn_status attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                         void* o, float* lse, int B, int Hq, int Hkv, int Smax, int D, float scale,

@@ -52,6 +52,7 @@ def test_fwd_validation(lib):
     assert fwd(lib, scale=float("nan")) == 1
     assert fwd(lib, causal=2) == 1
     assert fwd(lib, dtype=7) == 1
+    assert fwd(lib, dtype=2, D=96) == 4
     assert fwd(lib, ptr=None) == 1
     assert fwd(lib, ptr=ctypes.c_void_p((1 << 20) + 2)) == 1   # misaligned
 

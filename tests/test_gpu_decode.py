@@ -12,13 +12,13 @@ from attn_cases import TOL_BF16_LSE, TOL_BF16_O, bits_to_dev, compare, to_host_f
 pytestmark = pytest.mark.gpu
 
 
-def run_decode(w: si.Decode, num_splits=None, seqlens=None):
+def run_decode(w: si.Decode, num_splits=None, seqlens=None, out_dtype=torch.float32):
     d = si.decode_inputs(w, seqlens=seqlens)
     q = bits_to_dev(d["q_bits"])
     kc = bits_to_dev(d["k_bits"])
     vc = bits_to_dev(d["v_bits"])
     sl = torch.from_numpy(d["seqlens"]).cuda()
-    o, lse = ea.attn_decode(q, kc, vc, sl, w.scale, num_splits or w.num_splits)
+    o, lse = ea.attn_decode(q, kc, vc, sl, w.scale, num_splits or w.num_splits, out_dtype=out_dtype)
     torch.cuda.synchronize()
     status = ea.read_device_status()
     og, lg = to_host_f64(o), to_host_f64(lse)
@@ -52,6 +52,11 @@ CASES = [
 @pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
 def test_decode_matches_oracle(w):
     assert run_decode(w) == 0
+
+
+def test_decode_bf16_output():
+    w = D("bf16_out", 3, 8, 2, 64, 2000, 1, 2000, 8, seed=21)
+    assert run_decode(w, out_dtype=torch.bfloat16) == 0
 
 
 @pytest.mark.parametrize("ns", [1, 2, 3, 7, 64])
