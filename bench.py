@@ -64,6 +64,12 @@ def max_over_ranks(x: float, dist, device) -> float:
     return float(t.item())
 
 
+def whole_job_rate(work_per_rank: float, ms_max: float, world: int) -> float:
+    """Units per second of the whole job: every rank (replica) did work_per_rank units, the
+    slowest rank took ms_max milliseconds."""
+    return world * work_per_rank / (ms_max * 1e-3)
+
+
 def barrier(dist, device):
     if dist is not None:
         import torch
@@ -314,15 +320,15 @@ def run_gpu(args):
         r = bench_prefill_gpu(w, args, torch, ea, dist, device)
         ms = max_over_ranks(r["ms"], dist, device)
         ms_e2e = max_over_ranks(r["ms_e2e"], dist, device)
-        value = world * w.flops / (ms * 1e-3) / 1e12
-        value_e2e = world * w.flops / (ms_e2e * 1e-3) / 1e12
+        value = whole_job_rate(w.flops, ms, world) / 1e12
+        value_e2e = whole_job_rate(w.flops, ms_e2e, world) / 1e12
         unit = "TFLOP/s"
         dec_w = si.C4
         dec = bench_decode_gpu(dec_w, args, torch, ea, dist, device, steps=max(5, args.steps // 2))
         dec_ms = max_over_ranks(dec["ms"], dist, device)
         dec["ms"] = dec_ms
         roof = roofline_prefill(w, r["ms"], peaks, how, profile_traffic("prefill_tc_" + w.name.split("_")[0]))
-        extra = {"decode": {"workload": dec_w.name, "value": round(world * dec["kv_bytes"] / (dec_ms * 1e-3) / 1e9, 1),
+        extra = {"decode": {"workload": dec_w.name, "value": round(whole_job_rate(dec["kv_bytes"], dec_ms, world) / 1e9, 1),
                             "unit": "GB/s", "ms_per_call": round(dec_ms, 4),
                             "roofline": roofline_decode(dec, peaks, how)}}
         clocks = r["clocks"]
@@ -338,7 +344,7 @@ def run_gpu(args):
             dec = bench_decode_gpu(w, args, torch, ea, dist, device)
         ms = max_over_ranks(dec["ms"], dist, device)
         dec["ms"] = ms
-        value = world * dec["kv_bytes"] / (ms * 1e-3) / 1e9
+        value = whole_job_rate(dec["kv_bytes"], ms, world) / 1e9
         unit = "GB/s"
         roof = roofline_decode(dec, peaks, how)
         roof["traffic"] = profile_traffic("decode_split_" + w.name.split("_")[0])
