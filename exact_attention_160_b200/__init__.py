@@ -30,8 +30,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 
 # symbols the library exports (kept in step with include/attn_b200.h)
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
-           "attn_decode_workspace_size", "rope_apply", "attn_status_string", "attn_last_error",
-           "attn_read_device_status")
+           "attn_decode_workspace_size", "attn_decode_noalloc", "rope_apply", "attn_status_string",
+           "attn_last_error", "attn_read_device_status")
 
 _lib = None
 
@@ -61,6 +61,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, Z, I, P]
     lib.attn_decode_workspace_size.argtypes = [I, I, I, I]
     lib.attn_decode_workspace_size.restype = Z
+    lib.attn_decode_noalloc.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, I, P]
+    lib.attn_decode_noalloc.restype = I
     lib.rope_apply.argtypes = [P, P, I, I, I, F, I, P]
     lib.attn_status_string.argtypes = [I]
     lib.attn_status_string.restype = ctypes.c_char_p

@@ -254,6 +254,47 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
 
 }  // namespace
 
+// ------------------------------------------------------------------------------------------
+// Built-in decode scratch for callers that cannot allocate device memory.
+//
+// attn_decode needs somewhere to put the per-split partial outputs; normally the caller passes a
+// workspace.  Some callers cannot provide one: code that runs inside a host framework owning
+// every device allocation (a plugin handed only its input and output buffers), or a serving
+// path that must not call cudaMalloc because it can synchronise the device and take an
+// unbounded time.  For them attn_decode_noalloc keeps the partials in this fixed array, which
+// exists once per GPU that loads the library and stays allocated until the process exits.
+// ------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};   // device address of g_noalloc_scratch, per device
+
+// Device address of the scratch array on the current device, looked up once per device.  A
+// host-side reference to g_noalloc_scratch is only a stand-in for the symbol, never a device
+// address, so the address must come from cudaGetSymbolAddress with that device current.
+attn_status noalloc_scratch(void** out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_failure("cudaGetDevice", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices) return cuda_failure("attn_decode_noalloc", "device ordinal out of range");
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+        void* ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || ptr == nullptr)
+            return cuda_failure("cudaGetSymbolAddress(g_noalloc_scratch)",
+                                e != cudaSuccess ? cudaGetErrorString(e) : "null address");
+        g_noalloc_addr[dev] = ptr;
+    }
+    *out = g_noalloc_addr[dev];
+    return ATTN_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
@@ -315,6 +356,55 @@ attn_status attn_decode(const void* q, const void* kcache, const void* vcache, c
     ATTN_DECODE_CASE(128, 2)
     ATTN_DECODE_CASE(128, 4)
 #undef ATTN_DECODE_CASE
+    return ATTN_ERR_UNSUPPORTED;
+}
+
+attn_status attn_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
+                                void* o, float* lse, int B, int Hq, int Hkv, int Smax, int D, float scale,
+                                int num_splits, attn_dtype dtype, attn_stream_t stream) {
+    // Same checks as attn_decode, then the size check against the built-in scratch.
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_splits <= 0) return ATTN_ERR_INVALID_ARG;
+    if (Smax == 0) return ATTN_ERR_EMPTY_KV;
+    if (Smax < 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_ERR_DIM_MISMATCH;
+    if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !kcache || !vcache || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_BF16_OUT_F32)
+        return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
+    const size_t need = attn_decode_workspace_size(B, Hq, D, num_splits);
+    if (need > ATTN_NOALLOC_SCRATCH_BYTES) {
+        char buf[160];
+        snprintf(buf, sizeof(buf), "split partials need %zu bytes, the built-in scratch holds %zu (lower num_splits or B*Hq)",
+                 need, static_cast<size_t>(ATTN_NOALLOC_SCRATCH_BYTES));
+        snprintf(g_last_error, sizeof(g_last_error), "attn_decode_noalloc: %s", buf);
+        return ATTN_ERR_WORKSPACE;
+    }
+    void* scratch = nullptr;
+    attn_status s = noalloc_scratch(&scratch);
+    if (s != ATTN_OK) return s;
+    // Nothing in the scratch has to start at zero: every partial the combine reads is written
+    // earlier in the same call by the split kernel.
+    const size_t slots = static_cast<size_t>(B) * Hq * num_splits;
+    float* o_part = static_cast<float*>(scratch);
+    float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + round_up(slots * D * sizeof(float), 256));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
+    const int G = Hq / Hkv;
+    const int GC = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
+#define ATTN_DECODE_NOALLOC_CASE(DD, GG)                                                                      \
+    if (D == DD && GC == GG)                                                                                  \
+        return launch_decode<DD, GG>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale,       \
+                                     num_splits, o_part, lse_part, st);
+    ATTN_DECODE_NOALLOC_CASE(64, 1)
+    ATTN_DECODE_NOALLOC_CASE(64, 2)
+    ATTN_DECODE_NOALLOC_CASE(64, 4)
+    ATTN_DECODE_NOALLOC_CASE(128, 1)
+    ATTN_DECODE_NOALLOC_CASE(128, 2)
+    ATTN_DECODE_NOALLOC_CASE(128, 4)
+#undef ATTN_DECODE_NOALLOC_CASE
     return ATTN_ERR_UNSUPPORTED;
 }
 

@@ -127,6 +127,33 @@ attn_status attn_decode(const void* q, const void* kcache, const void* vcache, c
 size_t attn_decode_workspace_size(int B, int Hq, int D, int num_splits);
 
 /*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device memory.
+ *   (Not an operation of the method: the pages have no counterpart.  It is attn_decode with
+ *   the split partials kept in scratch memory that the library owns.)
+ *   Some callers cannot hand attn_decode a workspace: code inside a host framework that owns
+ *   every device allocation and gives it only input and output buffers, or a latency-bound
+ *   serving path that must not call cudaMalloc, which can synchronise the device and take an
+ *   unbounded time.  This entry point takes the same arguments as attn_decode minus the
+ *   workspace and allocates nothing: the partials go to a fixed array of
+ *   ATTN_NOALLOC_SCRATCH_BYTES bytes that exists once on every GPU that loads the library and
+ *   stays allocated until the process exits.
+ *   - Sizes: attn_decode_workspace_size(B, Hq, D, num_splits) must not exceed
+ *     ATTN_NOALLOC_SCRATCH_BYTES, else ATTN_ERR_WORKSPACE (attn_last_error() says by how much).
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, which may load the library's GPU code onto that device); make that
+ *     first call before any stream capture.  Failure returns ATTN_ERR_CUDA.
+ *   - Sharing: every call on a device uses the same array, and it keeps the last call's
+ *     contents.  Calls that overlap on the GPU (different streams, no ordering between them)
+ *     race on it and may return wrong results; order them on one stream or with events.
+ *     Nothing in the array needs to start at zero.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (16u << 20)
+attn_status attn_decode_noalloc(const void* q, const void* kcache, const void* vcache,
+                                const int32_t* seqlens, void* o, float* lse, int B, int Hq, int Hkv,
+                                int Smax, int D, float scale, int num_splits, attn_dtype dtype,
+                                attn_stream_t stream);
+
+/*
  * rope_apply -- rotate x in place: x [T, H, D] (dtype), token t at position pos[t]
  * (int32 device array [T]); rotation as in attn_fwd_ex.  D must be even (DIM_MISMATCH).
  */
