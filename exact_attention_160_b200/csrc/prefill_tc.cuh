@@ -21,6 +21,9 @@
 //     threads read their row of S with tcgen05.ld, compute P = exp2(S*scale*log2e - m) in fp32,
 //     round P to bf16 and write it back to TMEM; O += P V is an MMA with A = P from TMEM and
 //     B = V from shared memory (N = D), accumulating in TMEM.
+//   * At D=128 the two softmax warpgroups take turns for their exponentiation phase (ping-pong
+//     through two mbarriers): the MUFU unit of each sub-partition is shared by one warp of each
+//     group, so while one group exponentiates the other loads S, takes its row max, corrects O.
 //   * Lazy rescale: the running max used for the exponent only moves when the block max exceeds
 //     it by more than kRescaleThreshold (log2 units, i.e. a factor 256), which keeps P <= 256
 //     while skipping the O correction on almost every block.  The "running max is -inf" guard
@@ -64,11 +67,16 @@ struct TcCfg {
     static constexpr int Q_BYTES = 2 * Q_TILES * TILE_BYTES;
     static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = SMEM_DATA + 1024 /* alignment slack */ + 256 /* barriers */;
+    static_assert(8 * (14 + 3 * STAGES) + 4 <= 256, "barrier area");
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
     static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
     static constexpr uint32_t COL_P0 = (D == 64) ? 384 : 0;
     static constexpr uint32_t COL_P1 = (D == 64) ? 448 : 128;
     static constexpr bool P_ALIASES_S = (D != 64);
+    // Exponentiation turns between the two softmax warpgroups: at D=128 the softmax otherwise
+    // idles while P_i -> PV_i -> S_i(j+1) runs, so alternating keeps MUFU busy; at D=64 one warp
+    // alone cannot keep MUFU busy and the groups do better exponentiating concurrently.
+    static constexpr bool PINGPONG = (D != 64);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -118,11 +126,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     uint64_t* bar_s_full = bars + 2;       // [2]
     uint64_t* bar_p_ready = bars + 4;      // [2]
     uint64_t* bar_pv_done = bars + 6;      // [2]
-    uint64_t* bar_k_full = bars + 8;       // [STAGES]
+    uint64_t* bar_s_free = bars + 8;       // [2] softmax has read S_i into registers
+    uint64_t* bar_turn = bars + 10;        // [2] exponentiation turn of softmax warpgroup i
+    uint64_t* bar_k_full = bars + 12;      // [STAGES]
     uint64_t* bar_v_full = bar_k_full + C::STAGES;
     uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
-    uint64_t* bar_mma_final = bar_kv_empty + C::STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma_final + 1);
+    uint64_t* bar_mma_final = bar_kv_empty + C::STAGES;   // [2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma_final + 2);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -159,13 +169,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             mbar_init(bar_s_full + i, 1);
             mbar_init(bar_p_ready + i, 128);
             mbar_init(bar_pv_done + i, 1);
+            mbar_init(bar_s_free + i, 128);
+            mbar_init(bar_turn + i, 128);      // the other warpgroup's 128 threads hand over
         }
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(bar_k_full + s, 1);
             mbar_init(bar_v_full + s, 1);
-            mbar_init(bar_kv_empty + s, 1);
+            mbar_init(bar_kv_empty + s, 2);   // one commit from each MMA warp
         }
         mbar_init(bar_mma_final, 1);
+        mbar_init(bar_mma_final + 1, 1);
         mbar_fence_init();
     }
     if (warp == 0 && lane == 0) {
@@ -231,70 +244,98 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 mbar_wait(bar_v_full + j % C::STAGES, (j / C::STAGES) & 1);
             }
         }
-      } else if (warp == 1) {
-        // =============================== MMA issuer ======================================
+      } else if (warp == 1 || warp == 2) {
+        // =============================== MMA issuers =====================================
+        // Warp 1 issues every MMA of query tile 0, warp 2 those of tile 1 (one thread each), so
+        // the two tiles' pipelines do not wait on each other.  Per KV tile j:
+        //   S_i(j) = Q_i K_j^T  -> s_full_i ;  softmax_i reads S_i, writes P_i -> p_ready_i
+        //   O_i += P_i V_j      -> pv_done_i ;  both warps commit kv_empty once per stage
+        // D=64 (P_i has its own TMEM columns): S_i(j+1) is issued as soon as softmax_i has read
+        // S_i(j) (s_free_i), so the next scores are computed while the current ones are
+        // exponentiated.  D=128 (P_i overwrites S_i): S_i(j+1) waits until PV_i(j) consumed P_i(j).
+        const int i = warp - 1;
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            const uint32_t dS = tmem + (i ? C::COL_S1 : C::COL_S0);
+            const uint32_t dO = tmem + (i ? C::COL_O1 : C::COL_O0);
+            const uint32_t aP = tmem + (i ? C::COL_P1 : C::COL_P0);
+            const uint32_t sQi = smem_u32(sQ + i * C::Q_TILES * C::TILE_BYTES);
+            uint64_t* s_full = bar_s_full + i;
+            uint64_t* s_free = bar_s_free + i;
+            uint64_t* p_ready = bar_p_ready + i;
+            uint64_t* pv_done = bar_pv_done + i;
+            const int ni = i ? tile[1].nkv : tile[0].nkv;
             bool ok = mbar_wait(ROPE ? bar_q_ready : bar_q_full, 0);
             tc_fence_after();
-            for (int j = 0; ok && j < nkv; ++j) {
+            auto issue_s = [&](int j) {
+                const uint32_t sK = smem_u32(sKV + (j % C::STAGES) * C::STAGE_BYTES);
+                // chains: (Qh,Kh) [+ (Qh,Kl) + (Ql,Kh) with RoPE]
+                constexpr int NCHAIN = ROPE ? 3 : 1;
+#pragma unroll
+                for (int ch = 0; ch < NCHAIN; ++ch) {
+                    const uint32_t qa = sQi + (ch == 2 ? C::TILE_BYTES : 0);
+                    const uint32_t kb = sK + (ch == 1 ? C::TILE_BYTES : 0);
+#pragma unroll
+                    for (int kk = 0; kk < C::KSTEPS; ++kk) {
+                        // K step kk: box kk/4, 32-byte column offset (kk%4) inside the 128-byte row
+                        const uint32_t off = (kk >> 2) * (C::TILE_BYTES / C::NBOX) + (kk & 3) * 32;
+                        mma_ss(dS, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                               idesc_qk, (ch > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+                mma_commit(s_full);
+            };
+            auto issue_pv = [&](int j) {
+                const uint32_t sV = smem_u32(sKV + (j % C::STAGES) * C::STAGE_BYTES) + C::K_TILES * C::TILE_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // keys [16kk, 16kk+16): 16 rows of 128 B in every 64-wide D box
+                    const uint64_t db = smem_desc_sw128(sV + kk * 2048, C::TILE_BYTES / C::NBOX, 1024);
+                    mma_ts(dO, aP + kk * 8, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                mma_commit(pv_done);
+            };
+            auto wait_k = [&](int j) {
+                const bool r = mbar_wait(bar_k_full + j % C::STAGES, (j / C::STAGES) & 1);
+                tc_fence_after();
+                return r;
+            };
+            if (ok && ni > 0) {
+                ok = wait_k(0);
+                if (ok) issue_s(0);
+            }
+            for (int j = 0; j < nkv; ++j) {
                 const int s = j % C::STAGES;
-                const uint32_t ph = (j / C::STAGES) & 1;
-                const uint32_t sK = smem_u32(sKV + s * C::STAGE_BYTES);
-                const uint32_t sV = sK + C::K_TILES * C::TILE_BYTES;
-                if (!mbar_wait(bar_k_full + s, ph)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (j >= tile[i].nkv) continue;
-                    if (C::P_ALIASES_S && j > 0) {
-                        // PV_i(j-1) still reads P_i from the columns S_i(j) will overwrite
-                        if (!mbar_wait(bar_pv_done + i, (j - 1) & 1)) { ok = false; break; }
+                if (j < ni) {
+                    if (ok && !C::P_ALIASES_S && j + 1 < ni) {
+                        ok = wait_k(j + 1) && mbar_wait(s_free, j & 1);
                         tc_fence_after();
+                        if (ok) issue_s(j + 1);
                     }
-                    const uint32_t sQi = smem_u32(sQ + i * C::Q_TILES * C::TILE_BYTES);
-                    const uint32_t dS = tmem + (i ? C::COL_S1 : C::COL_S0);
-                    // chains: (Qh,Kh) [+ (Qh,Kl) + (Ql,Kh) with RoPE]
-                    constexpr int NCHAIN = ROPE ? 3 : 1;
-#pragma unroll
-                    for (int ch = 0; ch < NCHAIN; ++ch) {
-                        const uint32_t qa = sQi + (ch == 2 ? C::TILE_BYTES : 0);
-                        const uint32_t kb = sK + (ch == 1 ? C::TILE_BYTES : 0);
-#pragma unroll
-                        for (int kk = 0; kk < C::KSTEPS; ++kk) {
-                            // K step kk: box kk/4, 32-byte column offset (kk%4) inside the 128-byte row
-                            const uint32_t off = (kk >> 2) * (C::TILE_BYTES / C::NBOX) + (kk & 3) * 32;
-                            const uint64_t da = smem_desc_sw128(qa + off, 16, 1024);
-                            const uint64_t db = smem_desc_sw128(kb + off, 16, 1024);
-                            mma_ss(dS, da, db, idesc_qk, (ch > 0 || kk > 0) ? 1u : 0u);
-                        }
-                    }
-                    mma_commit(bar_s_full + i);
-                }
-                if (!ok) break;
-                if (!mbar_wait(bar_v_full + s, ph)) { ok = false; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (j >= tile[i].nkv) continue;
-                    if (!mbar_wait(bar_p_ready + i, j & 1)) { ok = false; break; }
+                    if (ok) ok = mbar_wait(bar_v_full + s, (j / C::STAGES) & 1) && mbar_wait(p_ready, j & 1);
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        // keys [16kk, 16kk+16): 16 rows of 128 B in every 64-wide D box
-                        const uint64_t db = smem_desc_sw128(sV + kk * 2048, C::TILE_BYTES / C::NBOX, 1024);
-                        mma_ts(tmem + (i ? C::COL_O1 : C::COL_O0), tmem + (i ? C::COL_P1 : C::COL_P0) + kk * 8, db,
-                               idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    mma_commit(bar_pv_done + i);
+                    if (ok) issue_pv(j);
+                } else {
+                    // No work for this tile, but the stage's release still needs this warp's
+                    // arrival.  Wait until the stage holds tile j first: an arrival made earlier
+                    // could complete a later phase of kv_empty on its own and free the stage
+                    // while the other warp's MMAs still read it.
+                    mbar_wait(bar_k_full + s, (j / C::STAGES) & 1);
+                    mbar_wait(bar_v_full + s, (j / C::STAGES) & 1);
                 }
-                if (!ok) break;
+                // this warp is done with stage s once its MMAs so far complete (S_i(j), PV_i(j))
                 mma_commit(bar_kv_empty + s);
+                if (ok && C::P_ALIASES_S && j + 1 < ni) {
+                    // S_i(j+1) overwrites P_i(j): PV_i(j) must have consumed it
+                    ok = wait_k(j + 1) && mbar_wait(pv_done, j & 1);
+                    tc_fence_after();
+                    if (ok) issue_s(j + 1);
+                }
             }
             // every MMA issued above must be complete before tensor memory is released
-            mma_commit(bar_mma_final);
-            mbar_wait(bar_mma_final, 0);
+            mma_commit(bar_mma_final + i);
+            mbar_wait(bar_mma_final + i, 0);
         }
       }
     } else {
@@ -360,13 +401,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         float l_run = 0.f;         // row sum of the fp32 weights (logsumexp)
         float l_mma = 0.f;         // row sum of the bf16-rounded weights (normalises O)
         const float sl2 = p.scale_log2;
-        for (int j = 0; ok && j < T.nkv; ++j) {
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) { ok = false; break; }
+        // Turn passing: round r of group 0 waits turn_0 (phase r), exponentiates, hands turn_1;
+        // group 1 the reverse.  Group 1 gives group 0 the first turn.  Both groups run all nkv
+        // rounds (idle rounds only pass the turn), so neither waits for a hand-over that never
+        // comes; after a failed wait a group stops waiting but keeps handing over.
+        if (C::PINGPONG && wg == 1 && nkv > 0) mbar_arrive(bar_turn + 0);
+        for (int j = 0; j < nkv; ++j) {
+          const bool work = j < T.nkv;
+          uint32_t sr[4][32];
+          float mu = 0.f;
+          if (ok && work) {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) ok = false;
             tc_fence_after();
-            uint32_t sr[4][32];
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tmem_ld32(tS + cb * 32, sr[cb]);
             tmem_wait_ld();
+            if (!C::P_ALIASES_S) {
+                // S_i is in registers: the next S_i MMA may overwrite it
+                tc_fence_before();
+                mbar_arrive(bar_s_free + wg);
+            }
             // mask: keys past Skv, and (causal) keys beyond this row's diagonal
             const int k0 = j * 128;
             const long lim_causal = p.causal ? static_cast<long>(qrow) + off_c : static_cast<long>(p.Skv) - 1;
@@ -380,11 +434,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     for (int e = 0; e < 32; ++e)
                         if (cb * 32 + e >= nvis) sr[cb][e] = __float_as_uint(-INFINITY);
             }
+            {
+                // eight independent three-input max chains, then a short tree
+                float mp[8];
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb)
+                for (int c = 0; c < 8; ++c) {
+                    const uint32_t* r = &sr[c >> 1][(c & 1) * 16];
+                    float a = fmaxf(__uint_as_float(r[0]), __uint_as_float(r[1]));
 #pragma unroll
-                for (int e = 0; e < 32; e += 2)
-                    mx = max3(mx, __uint_as_float(sr[cb][e]), __uint_as_float(sr[cb][e + 1]));
+                    for (int e = 2; e < 16; e += 2) a = max3(a, __uint_as_float(r[e]), __uint_as_float(r[e + 1]));
+                    mp[c] = a;
+                }
+                mx = max3(max3(mp[0], mp[1], mp[2]), max3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+            }
             const float tmax = mx * sl2;
             // lazy rescale: move the exponent's max only when the block max exceeds it by > threshold
             const bool need = tmax > m_run + kRescaleThreshold;
@@ -394,8 +456,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 m_run = tmax;
             }
             // O correction: only warps with a rescaling row, only once O holds earlier blocks
-            if (j > 0 && __any_sync(0xffffffffu, need)) {
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) { ok = false; break; }
+            if (ok && j > 0 && __any_sync(0xffffffffu, need)) {
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) ok = false;
                 tc_fence_after();
 #pragma unroll
                 for (int cb = 0; cb < D / 32; ++cb) {
@@ -410,16 +472,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             }
             l_run *= corr;
             l_mma *= corr;
-            const float mu = (m_run == -INFINITY) ? 0.f : m_run;
+            mu = (m_run == -INFINITY) ? 0.f : m_run;
             if (!C::P_ALIASES_S && j > 0) {
                 // P_i(j-1) must have been consumed by PV_i(j-1) before it is overwritten
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) { ok = false; }
                 tc_fence_after();
             }
+          }
+          // wait for this group's exponentiation turn (every round, also idle ones)
+          if (C::PINGPONG && ok && !__all_sync(0xffffffffu, mbar_wait(bar_turn + wg, j & 1))) ok = false;
+          if (ok && work) {
             // p = exp2(s*scale*log2e - mu) in fp32, rounded to bf16 for the PV MMA.  Two row sums:
             // the exact one (for the logsumexp) and the sum of the rounded values the MMA uses
             // (O is normalised by it, so the rounding of a dominant weight cancels).
-            uint64_t lt2 = 0, lr2 = 0;   // packed (even, odd) partial sums
+            uint64_t lt2[4] = {0, 0, 0, 0}, lr2[4] = {0, 0, 0, 0};   // packed partial sums, 4 chains each
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t nmux2 = f2_pack(-mu, -mu);
 #pragma unroll
@@ -433,22 +499,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                               t0, t1);
                     const float p0 = fast_exp2(t0);
                     const float p1 = fast_exp2(t1);
-                    lt2 = f2_add(lt2, f2_pack(p0, p1));
+                    lt2[e & 3] = f2_add(lt2[e & 3], f2_pack(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
-                    lr2 = f2_add(lr2, f2_pack(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
+                    lr2[e & 3] = f2_add(lr2[e & 3], f2_pack(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                 }
                 tmem_st16(tP + cb * 16, pk);
             }
             {
                 float a, c;
-                f2_unpack(lt2, a, c);
+                f2_unpack(f2_add(f2_add(lt2[0], lt2[1]), f2_add(lt2[2], lt2[3])), a, c);
                 l_run += a + c;
-                f2_unpack(lr2, a, c);
+                f2_unpack(f2_add(f2_add(lr2[0], lr2[1]), f2_add(lr2[2], lr2[3])), a, c);
                 l_mma += a + c;
             }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p_ready + wg);
+          }
+          // hand the exponentiation turn to the other group (group 1 skips its last hand-over,
+          // which nobody would wait for)
+          if (C::PINGPONG && !(wg == 1 && j == nkv - 1)) mbar_arrive(bar_turn + (wg ^ 1));
         }
 
         // epilogue: O / l -> bf16 or fp32, lse.  The TMEM reads are warp-collective, so every
