@@ -48,9 +48,10 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Tensor [B][S][H][D] bf16 viewed as 4-D (D, H, S, B); box = 64 elements x 1 head x 128 rows,
-// 128-byte swizzle (the UMMA SW128 K-major / MN-major operand layout).  Rows past S read as 0.
-bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D) {
+// Tensor [B][S][H][D] bf16 viewed as 4-D (D, H, S, B); box = 64 elements x 1 head x `rows` rows,
+// 128-byte swizzle (the UMMA SW128 K-major / MN-major operand layout, and a bank-conflict-free
+// ldmatrix layout).  Rows past S read as 0.
+bool make_tmap_bshd_rows(CUtensorMap* m, const void* ptr, int B, int S, int H, int D, int rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) {
         cuda_failure("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", "entry point unavailable");
@@ -58,7 +59,7 @@ bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D)
     }
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
-    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -69,6 +70,10 @@ bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D)
         cuda_failure("cuTensorMapEncodeTiled", buf);
     }
     return r == CUDA_SUCCESS;
+}
+
+bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D) {
+    return make_tmap_bshd_rows(m, ptr, B, S, H, D, 128);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -229,24 +234,33 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
                                           q_pos0, st);
 }
 
-template <int D, int GC>
+template <int D>
 attn_status launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* o, bool o_f32,
-                          float* lse,
-                          int B, int Hq, int Hkv, int Smax, float scale, int num_splits, float* o_part,
+                          float* lse, int B, int Hq, int Hkv, int Smax, float scale, int num_splits, float* o_part,
                           float* lse_part, cudaStream_t st) {
-    constexpr int LPK = D / 8, SLOTS = 32 / LPK, NPART = kDecodeWarps * SLOTS;
-    const size_t smem = (2 * NPART * GC + NPART * GC * D) * sizeof(float);
+    using C = DecCfg<D>;
+    CUtensorMap tk, tv;
+    if (!make_tmap_bshd_rows(&tk, kc, B, Smax, Hkv, D, C::TK) || !make_tmap_bshd_rows(&tv, vc, B, Smax, Hkv, D, C::TK))
+        return ATTN_ERR_CUDA;
     const int G = Hq / Hkv;
+    // heads per CTA: the largest power of two <= 16 dividing the group size
+    int GC = 16;
+    while (G % GC != 0) GC >>= 1;
     dim3 grid(num_splits, Hkv * (G / GC), B);
     if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
-    decode_split_kernel<D, GC><<<grid, kDecodeWarps * 32, smem, st>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(kc),
-        static_cast<const __nv_bfloat16*>(vc), seqlens, o_part, lse_part, Hkv, G, Smax, num_splits,
-        scale * 1.4426950408889634f);
+    auto kern = decode_split_kernel<D>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(decode_split_kernel)", cudaGetErrorString(e));
+        attr_set = true;
+    }
+    kern<<<grid, kDecodeThreads, C::SMEM_BYTES, st>>>(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, o_part,
+                                                      lse_part, Hkv, G, GC, Smax, num_splits,
+                                                      scale * 1.4426950408889634f);
     attn_status s = launch_status("decode_split_kernel");
     if (s != ATTN_OK) return s;
-    const int warps = B * Hq;
-    decode_combine_kernel<D><<<(warps + 3) / 4, 128, 0, st>>>(
+    decode_combine_kernel<D><<<B * Hq, kCombineWarps * 32, 0, st>>>(
         o_part, lse_part, seqlens, o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
         o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Hq, Smax, num_splits);
     return launch_status("decode_combine_kernel");
@@ -337,25 +351,19 @@ attn_status attn_decode(const void* q, const void* kcache, const void* vcache, c
     const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
     if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
     if (num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long>(B) * Hq > 2147483647L) return ATTN_ERR_UNSUPPORTED;
     const size_t need = attn_decode_workspace_size(B, Hq, D, num_splits);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
     const size_t slots = static_cast<size_t>(B) * Hq * num_splits;
     float* o_part = static_cast<float*>(workspace);
     float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(slots * D * sizeof(float), 256));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int G = Hq / Hkv;
-    const int GC = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
-#define ATTN_DECODE_CASE(DD, GG)                                                                              \
-    if (D == DD && GC == GG)                                                                                  \
-        return launch_decode<DD, GG>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, \
-                                     o_part, lse_part, st);
-    ATTN_DECODE_CASE(64, 1)
-    ATTN_DECODE_CASE(64, 2)
-    ATTN_DECODE_CASE(64, 4)
-    ATTN_DECODE_CASE(128, 1)
-    ATTN_DECODE_CASE(128, 2)
-    ATTN_DECODE_CASE(128, 4)
-#undef ATTN_DECODE_CASE
+    if (D == 64)
+        return launch_decode<64>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, o_part,
+                                 lse_part, st);
+    if (D == 128)
+        return launch_decode<128>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits,
+                                  o_part, lse_part, st);
     return ATTN_ERR_UNSUPPORTED;
 }
 
@@ -392,19 +400,12 @@ attn_status attn_decode_noalloc(const void* q, const void* kcache, const void* v
     float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + round_up(slots * D * sizeof(float), 256));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
-    const int G = Hq / Hkv;
-    const int GC = (G % 4 == 0) ? 4 : (G % 2 == 0) ? 2 : 1;
-#define ATTN_DECODE_NOALLOC_CASE(DD, GG)                                                                      \
-    if (D == DD && GC == GG)                                                                                  \
-        return launch_decode<DD, GG>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale,       \
-                                     num_splits, o_part, lse_part, st);
-    ATTN_DECODE_NOALLOC_CASE(64, 1)
-    ATTN_DECODE_NOALLOC_CASE(64, 2)
-    ATTN_DECODE_NOALLOC_CASE(64, 4)
-    ATTN_DECODE_NOALLOC_CASE(128, 1)
-    ATTN_DECODE_NOALLOC_CASE(128, 2)
-    ATTN_DECODE_NOALLOC_CASE(128, 4)
-#undef ATTN_DECODE_NOALLOC_CASE
+    if (D == 64)
+        return launch_decode<64>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, o_part,
+                                 lse_part, st);
+    if (D == 128)
+        return launch_decode<128>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits,
+                                  o_part, lse_part, st);
     return ATTN_ERR_UNSUPPORTED;
 }
 

@@ -8,23 +8,22 @@
 // src/model/lfm2/gqa.rs, attention_cached: the new token attends to the whole cache, no mask,
 // q head h reading kv head h / (Hq/Hkv).
 //
-// Split kernel: one CTA per (split, kv head x head block, sequence), 4 warps.  GC query heads of a
-// group (GC = the whole group when it has at most 4 heads) are handled together so every K/V row
-// is read from HBM once per GC heads; larger groups run G/GC CTAs that meet in L2.  A key row of one kv
-// head is D bf16 = D*2 contiguous bytes; LPK = D/8 lanes read it with one 16-byte load each
-// (coalesced: a warp load instruction covers 32/LPK whole rows).  Each lane keeps 8 dims of q for
-// every head of the group and computes partial dot products for the rows it loaded; partials are
-// reduce-scattered over the LPK lanes of a row with shuffles so that each lane ends with whole
-// scores, exponentiated once, then gathered back for the P.V update.
+// Split kernel: one CTA per (split, kv head x head block, sequence).  A producer warp streams the
+// split's K and V rows (one kv head: D bf16 = 2D contiguous bytes per key) into a two-stage
+// shared-memory ring with TMA; four consumer warps compute.  Up to 16 query heads of a group are
+// handled together as the rows of 16x8x16 bf16 tensor-core MMAs (fp32 accumulation), so every
+// K/V row is read from HBM once for the whole group and the dot products cost about one MMA per
+// key instead of dozens of FMA, shuffle and conversion instructions -- which is what lets the
+// kernel run at memory speed.  The S accumulators, exponentiated and rounded to bf16, are the A
+// operand of O += P V directly (no shuffles).
 //
-// Combine kernel: one warp per (sequence, q head) merges the splits by logsumexp.
+// Combine kernel: eight warps per (sequence, q head) merge the splits by logsumexp.
 #pragma once
 
 #include "common.cuh"
 
 namespace attn {
 
-constexpr int kDecodeWarps = 4;
 constexpr int kDecodeMinKeysPerSplit = 512;
 
 // Number of splits sequence length L uses, and the key range of split s (near-equal contiguous
@@ -44,230 +43,303 @@ __device__ __forceinline__ int clamp_seqlen(int L, int Smax) {
     return L;
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
-    uint4 r;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-                 : "l"(p));
-    return r;
+constexpr int kDecodeConsumerWarps = 4;
+constexpr int kDecodeThreads = (kDecodeConsumerWarps + 1) * 32;   // + one TMA producer warp
+constexpr int kDecodeStages = 2;
+constexpr int kDecodeMaxHeads = 16;                                 // q heads per CTA (MMA rows)
+
+// A tile is TK keys of one kv head: one 128-byte-swizzled TMA box per 64 dims, for K and for V
+// (16 KB each).  Each consumer warp owns KW = TK/4 keys of the tile.
+template <int D>
+struct DecCfg {
+    static constexpr int TK = (D == 64) ? 128 : 64;
+    static constexpr int KW = TK / kDecodeConsumerWarps;     // keys per warp per tile
+    static constexpr int NBOX = D / 64;
+    static constexpr int BOX_BYTES = TK * 128;
+    static constexpr int TILE_BYTES = NBOX * BOX_BYTES;
+    static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr int RING_BYTES = kDecodeStages * STAGE_BYTES;
+    static constexpr int SMEM_BYTES = RING_BYTES + 128 /* barriers */ + 1024 /* alignment */;
+};
+
+// Byte offset of the 16-byte chunk holding dims [8*ch, 8*ch+8) of row `row` in a tile made of
+// 128-byte-swizzled boxes of 64 dims (TMA SWIZZLE_128B layout, 1024-byte aligned boxes).
+template <int D>
+__device__ __forceinline__ uint32_t dec_chunk(int row, int ch) {
+    return static_cast<uint32_t>((ch >> 3) * DecCfg<D>::BOX_BYTES + row * 128 + (((ch & 7) ^ (row & 7)) << 4));
 }
 
-template <int D, int G>   // G: query heads handled by one CTA
-__global__ void __launch_bounds__(kDecodeWarps * 32) decode_split_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kc,
-    const __nv_bfloat16* __restrict__ vc, const int32_t* __restrict__ seqlens,
-    float* __restrict__ o_part, float* __restrict__ lse_part, int Hkv, int group, int Smax,
-    int max_splits, float scale_log2) {
-    constexpr int LPK = D / 8;            // lanes per key row
-    constexpr int SLOTS = 32 / LPK;       // rows per warp load instruction
-    constexpr int NLOAD = 8;              // load instructions per tensor per iteration
-    constexpr int KPW = NLOAD * SLOTS;    // keys per warp iteration
-    constexpr int DUP = LPK / NLOAD;      // lanes ending with the same key's scores (1 or 2)
-    static_assert(DUP >= 1, "head dim too small for this layout");
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// D(16x8 f32) += A(16x16 bf16, row) * B(16x8 bf16, col)
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
-    extern __shared__ float sm_dec[];
+// One CTA per (split, kv head x head block, sequence): warp 4 streams the split's K and V rows
+// into a two-stage shared-memory ring with TMA; warps 0-3 each take a quarter of every tile.
+// The group's query heads (up to 16) are the rows of 16x8x16 bf16 MMAs: S = Q K^T with the keys
+// as MMA columns, then the S accumulators, exponentiated and rounded to bf16, are directly the
+// A operand of O += P V.  Every K/V row is read from HBM once for all heads of the CTA.
+template <int D>
+__global__ void __launch_bounds__(kDecodeThreads, 3) decode_split_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ seqlens, float* __restrict__ o_part,
+    float* __restrict__ lse_part, int Hkv, int group, int heads_per_cta, int Smax, int max_splits,
+    float scale_log2) {
+    using C = DecCfg<D>;
+    constexpr int KW = C::KW;
+    constexpr int NT = KW / 8;        // key columns of S per warp (8 keys each)
+    constexpr int KS = D / 16;        // k steps of S = Q K^T
+    constexpr int NKS = KW / 16;      // k steps of O += P V
+    constexpr int ND = D / 8;         // dim columns of O
+    extern __shared__ uint8_t sm_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar_full = reinterpret_cast<uint64_t*>(ring + C::RING_BYTES);
+    uint64_t* bar_empty = bar_full + kDecodeStages;
+
     const int split = blockIdx.x, b = blockIdx.z;
-    const int kvh = blockIdx.y / (group / G);
-    const int h0 = kvh * group + (blockIdx.y % (group / G)) * G;   // first q head of this CTA
+    const int GC = heads_per_cta;
+    const int kvh = blockIdx.y / (group / GC);
+    const int h0 = kvh * group + (blockIdx.y % (group / GC)) * GC;   // first q head of this CTA
     const int L = clamp_seqlen(seqlens[b], Smax);
     const int nsplit = decode_num_splits(L, max_splits);
     if (split >= nsplit) return;
     const int base = L / nsplit, rem = L % nsplit;
     const int kbeg = split * base + (split < rem ? split : rem);
     const int kend = kbeg + base + (split < rem ? 1 : 0);
+    const int ntiles = (kend - kbeg + C::TK - 1) / C::TK;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int c = lane % LPK, r = lane / LPK;
-    const int Hq = Hkv * group;
-
-    // q of the group, dims [8c, 8c+8), pre-scaled so that q.k is already in log2 units
-    float qf[G][8];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const uint4 w = *reinterpret_cast<const uint4*>(q + (static_cast<long>(b) * Hq + h0 + g) * D + c * 8);
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            qf[g][2 * e] = bf16lo_to_f32(ww[e]) * scale_log2;
-            qf[g][2 * e + 1] = bf16hi_to_f32(ww[e]) * scale_log2;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kDecodeStages; ++s) {
+            mbar_init(bar_full + s, 1);
+            mbar_init(bar_empty + s, kDecodeConsumerWarps);
         }
+        mbar_fence_init();
     }
-
-    float m[G], lsum[G], acc[G][8];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        m[g] = -INFINITY;
-        lsum[g] = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
-    }
-
-    const long row_stride = static_cast<long>(Hkv) * D;   // elements between consecutive keys
-    const __nv_bfloat16* kbase = kc + (static_cast<long>(b) * Smax * Hkv + kvh) * D + c * 8;
-    const __nv_bfloat16* vbase = vc + (static_cast<long>(b) * Smax * Hkv + kvh) * D + c * 8;
-
-    for (int chunk = kbeg + warp * KPW; chunk < kend; chunk += kDecodeWarps * KPW) {
-        uint4 kr[NLOAD], vr[NLOAD];
-#pragma unroll
-        for (int n = 0; n < NLOAD; ++n) {
-            const int key = chunk + n * SLOTS + r;
-            if (key < kend) {
-                kr[n] = ldg_stream(kbase + key * row_stride);
-                vr[n] = ldg_stream(vbase + key * row_stride);
-            } else {
-                kr[n] = make_uint4(0, 0, 0, 0);
-                vr[n] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        // partial dot products over this lane's 8 dims
-        float part[NLOAD][G];
-#pragma unroll
-        for (int n = 0; n < NLOAD; ++n) {
-            const uint32_t ww[4] = {kr[n].x, kr[n].y, kr[n].z, kr[n].w};
-            float kf[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                kf[2 * e] = bf16lo_to_f32(ww[e]);
-                kf[2 * e + 1] = bf16hi_to_f32(ww[e]);
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float s = 0.f;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) s = fmaf(qf[g][e], kf[e], s);
-                part[n][g] = s;
-            }
-        }
-        // reduce-scatter over the LPK lanes of a row: round k halves the set of keys a lane keeps
-#pragma unroll
-        for (int h = NLOAD / 2, off = LPK / 2; h >= 1; h /= 2, off /= 2) {
-            const bool upper = (lane & off) != 0;
-#pragma unroll
-            for (int n = 0; n < h; ++n) {
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float send = upper ? part[n][g] : part[n + h][g];
-                    const float keep = upper ? part[n + h][g] : part[n][g];
-                    part[n][g] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-                }
-            }
-        }
-#pragma unroll
-        for (int off = DUP / 2; off >= 1; off /= 2)
-#pragma unroll
-            for (int g = 0; g < G; ++g) part[0][g] += __shfl_xor_sync(0xffffffffu, part[0][g], off);
-
-        // this lane's whole scores: key n_own of the iteration, every head of the group
-        const int n_own = c / DUP;
-        const bool valid = chunk + n_own * SLOTS + r < kend;
-        float t[G], mx[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            t[g] = valid ? part[0][g] : -INFINITY;
-            mx[g] = t[g];
-        }
-#pragma unroll
-        for (int off = LPK / 2; off >= 1; off /= 2)
-#pragma unroll
-            for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], off));
-
-        float p[G], corr[G];
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            const float mn = fmaxf(m[g], mx[g]);
-            corr[g] = (m[g] == -INFINITY) ? 0.f : fast_exp2(m[g] - mn);
-            m[g] = mn;
-            const float mu = (mn == -INFINITY) ? 0.f : mn;
-            p[g] = fast_exp2(t[g] - mu);
-            lsum[g] = lsum[g] * corr[g] + ((c % DUP) == 0 ? p[g] : 0.f);
-        }
-        // gather every key's weights and update the output dims this lane owns
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[g][e] *= corr[g];
-#pragma unroll
-        for (int n = 0; n < NLOAD; ++n) {
-            const int src = r * LPK + n * DUP;
-            const uint32_t ww[4] = {vr[n].x, vr[n].y, vr[n].z, vr[n].w};
-            float vf[8];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                vf[2 * e] = bf16lo_to_f32(ww[e]);
-                vf[2 * e + 1] = bf16hi_to_f32(ww[e]);
-            }
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float pn = __shfl_sync(0xffffffffu, p[g], src);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pn, vf[e], acc[g][e]);
-            }
-        }
-    }
-
-    // row sum of each slot
-#pragma unroll
-    for (int off = LPK / 2; off >= 1; off /= 2)
-#pragma unroll
-        for (int g = 0; g < G; ++g) lsum[g] += __shfl_xor_sync(0xffffffffu, lsum[g], off);
-
-    // merge the (warp, slot) partial states of the CTA through shared memory
-    constexpr int NPART = kDecodeWarps * SLOTS;
-    float* sm_m = sm_dec;                       // [NPART][G]
-    float* sm_l = sm_m + NPART * G;             // [NPART][G]
-    float* sm_o = sm_l + NPART * G;             // [NPART][G][D]
-    const int part_id = warp * SLOTS + r;
-    if (c == 0) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-            sm_m[part_id * G + g] = m[g];
-            sm_l[part_id * G + g] = lsum[g];
-        }
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sm_o[(part_id * G + g) * D + c * 8 + e] = acc[g][e];
     __syncthreads();
 
-    for (int w = threadIdx.x; w < G * D; w += blockDim.x) {
-        const int g = w / D, d = w % D;
-        float M = -INFINITY;
-        for (int pi = 0; pi < NPART; ++pi) M = fmaxf(M, sm_m[pi * G + g]);
-        float Ls = 0.f, Od = 0.f;
-        if (M != -INFINITY) {
-            for (int pi = 0; pi < NPART; ++pi) {
-                const float mp = sm_m[pi * G + g];
-                if (mp == -INFINITY) continue;
-                const float wgt = fast_exp2(mp - M);
-                Ls = fmaf(sm_l[pi * G + g], wgt, Ls);
-                Od = fmaf(sm_o[(pi * G + g) * D + d], wgt, Od);
+    const int Hq = Hkv * group;
+    const int g = lane >> 2, t4 = lane & 3;    // MMA fragment coordinates: row g, column pair t4
+    float m_run = -INFINITY, l_run = 0.f, l_mma = 0.f;   // state of head row g (this lane's share)
+    float o_acc[ND][4];                                   // O rows g (c0,c1) and g+8 (padding)
+#pragma unroll
+    for (int nd = 0; nd < ND; ++nd)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o_acc[nd][e] = 0.f;
+
+    if (warp == kDecodeConsumerWarps) {
+        // ------------------------------- TMA producer ----------------------------------
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();   // the cache is streamed once
+            int issued = 0;
+            for (int t = 0; t < ntiles; ++t) {
+                const int s = t % kDecodeStages;
+                if (!mbar_wait(bar_empty + s, ((t / kDecodeStages) & 1) ^ 1)) break;
+                mbar_arrive_expect_tx(bar_full + s, C::STAGE_BYTES);
+                uint8_t* st = ring + s * C::STAGE_BYTES;
+#pragma unroll
+                for (int bx = 0; bx < C::NBOX; ++bx) {
+                    tma_load_4d(&tm_k, bar_full + s, st + bx * C::BOX_BYTES, bx * 64, kvh, kbeg + t * C::TK, b, pol);
+                    tma_load_4d(&tm_v, bar_full + s, st + C::TILE_BYTES + bx * C::BOX_BYTES, bx * 64, kvh,
+                                kbeg + t * C::TK, b, pol);
+                }
+                issued = t + 1;
+            }
+            // no copy may still be landing when the ring is reused below
+            for (int t = issued - kDecodeStages > 0 ? issued - kDecodeStages : 0; t < issued; ++t)
+                mbar_wait(bar_full + t % kDecodeStages, (t / kDecodeStages) & 1);
+        }
+    } else {
+        // ------------------------------- consumers -------------------------------------
+        // A fragments of Q (rows = heads; rows >= GC and the padding rows 8-15 are zero)
+        uint32_t qa[KS][2];
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk) {
+            qa[kk][0] = 0;
+            qa[kk][1] = 0;
+            if (g < GC) {
+                const uint32_t* qrow = reinterpret_cast<const uint32_t*>(q + (static_cast<long>(b) * Hq + h0 + g) * D);
+                qa[kk][0] = qrow[(kk * 16 + 2 * t4) >> 1];
+                qa[kk][1] = qrow[(kk * 16 + 8 + 2 * t4) >> 1];
             }
         }
-        const long hq = static_cast<long>(b) * Hq + h0 + g;
+        bool ok = true;
+        for (int t = 0; t < ntiles; ++t) {
+            const int s = t % kDecodeStages;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_full + s, (t / kDecodeStages) & 1))) { ok = false; break; }
+            const uint32_t sK = smem_u32(ring + s * C::STAGE_BYTES);
+            const uint32_t sV = sK + C::TILE_BYTES;
+            const int r0 = warp * KW;                     // first tile row of this warp
+            const int key0 = kbeg + t * C::TK + r0;       // its key index
+            const int nvalid = kend - key0;               // keys [key0, key0 + nvalid) are real
+            if (nvalid < KW) {
+                // rows past the split end may hold anything (other data, NaN): zero their V so
+                // that P = 0 times V stays 0 in the MMA
+                uint8_t* vt = ring + s * C::STAGE_BYTES + C::TILE_BYTES;
+                for (int idx = lane; idx < KW * (D / 8); idx += 32) {
+                    const int rr = idx / (D / 8), ch = idx % (D / 8);
+                    if (rr >= nvalid) *reinterpret_cast<uint4*>(vt + dec_chunk<D>(r0 + rr, ch)) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();   // ordered before the stage's next TMA fill
+                __syncwarp();
+            }
+            // S = Q K^T for this warp's KW keys: NT column blocks of 8 keys
+            float sacc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < KS; kk += 2) {
+                    // matrices: (keys, dims 16kk+0..7), (.., +8..15), (.., 16kk+16..23), (.., +24..31)
+                    const int row = r0 + nt * 8 + (lane & 7);
+                    const int ch = 2 * kk + (lane >> 3);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(sK + dec_chunk<D>(row, ch), b0, b1, b2, b3);
+                    mma_bf16_16816(sacc[nt], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+                    mma_bf16_16816(sacc[nt], qa[kk + 1][0], 0u, qa[kk + 1][1], 0u, b2, b3);
+                }
+            }
+            // online softmax for head row g over the keys of this slice
+            float mx = -INFINITY;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int kidx = nt * 8 + 2 * t4 + e;
+                    const float v = kidx < nvalid ? sacc[nt][e] * scale_log2 : -INFINITY;
+                    sacc[nt][e] = v;
+                    mx = fmaxf(mx, v);
+                }
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float mn = fmaxf(m_run, mx);
+            const float corr = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - mn);
+            m_run = mn;
+            const float mu = (mn == -INFINITY) ? 0.f : mn;
+            l_run *= corr;
+            l_mma *= corr;
+#pragma unroll
+            for (int nd = 0; nd < ND; ++nd) {
+                o_acc[nd][0] *= corr;
+                o_acc[nd][1] *= corr;
+            }
+            uint32_t pa[NT];   // bf16 pairs of P for row g: keys (8nt + 2t4, +1)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const float p0 = fast_exp2(sacc[nt][0] - mu);
+                const float p1 = fast_exp2(sacc[nt][1] - mu);
+                l_run += p0 + p1;
+                pa[nt] = pack_bf16x2(p0, p1);
+                l_mma += bf16lo_to_f32(pa[nt]) + bf16hi_to_f32(pa[nt]);
+            }
+            // O += P V: k steps of 16 keys, dim columns of 8
+#pragma unroll
+            for (int ks = 0; ks < NKS; ++ks) {
+#pragma unroll
+                for (int nd = 0; nd < ND; nd += 2) {
+                    // matrices (transposed): (keys 16ks+0..7, dims 8nd..), (keys +8..15, ..),
+                    //                        (keys 16ks+0..7, dims 8nd+8..), (keys +8..15, ..)
+                    const int row = r0 + ks * 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
+                    const int ch = nd + (lane >> 4);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(sV + dec_chunk<D>(row, ch), b0, b1, b2, b3);
+                    mma_bf16_16816(o_acc[nd], pa[2 * ks], 0u, pa[2 * ks + 1], 0u, b0, b1);
+                    mma_bf16_16816(o_acc[nd + 1], pa[2 * ks], 0u, pa[2 * ks + 1], 0u, b2, b3);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_empty + s);
+        }
+        (void)ok;
+        // row sums of head row g: add the four lanes t4 = 0..3
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+        l_mma += __shfl_xor_sync(0xffffffffu, l_mma, 1);
+        l_mma += __shfl_xor_sync(0xffffffffu, l_mma, 2);
+    }
+    __syncthreads();   // every tile consumed, no copy in flight: the ring is reused for the merge
+
+    // merge the four consumer warps' states per head row
+    constexpr int NW = kDecodeConsumerWarps;
+    float* sm_m = reinterpret_cast<float*>(ring);          // [NW][16]
+    float* sm_l = sm_m + NW * kDecodeMaxHeads;             // [NW][16]
+    float* sm_lm = sm_l + NW * kDecodeMaxHeads;            // [NW][16]
+    float* sm_o = sm_lm + NW * kDecodeMaxHeads;            // [NW][16][D]
+    static_assert((3 * NW * kDecodeMaxHeads + NW * kDecodeMaxHeads * D) * 4 <= C::RING_BYTES, "merge area");
+    if (warp < NW) {
+        if (t4 == 0) {
+            sm_m[warp * kDecodeMaxHeads + g] = m_run;
+            sm_l[warp * kDecodeMaxHeads + g] = l_run;
+            sm_lm[warp * kDecodeMaxHeads + g] = l_mma;
+        }
+#pragma unroll
+        for (int nd = 0; nd < ND; ++nd) {
+            sm_o[(warp * kDecodeMaxHeads + g) * D + nd * 8 + 2 * t4] = o_acc[nd][0];
+            sm_o[(warp * kDecodeMaxHeads + g) * D + nd * 8 + 2 * t4 + 1] = o_acc[nd][1];
+        }
+    }
+    __syncthreads();
+    for (int w = threadIdx.x; w < GC * D; w += blockDim.x) {
+        const int hh = w / D, d = w % D;
+        float M = -INFINITY;
+        for (int pi = 0; pi < NW; ++pi) M = fmaxf(M, sm_m[pi * kDecodeMaxHeads + hh]);
+        float Ls = 0.f, Lm = 0.f, Od = 0.f;
+        if (M != -INFINITY) {
+            for (int pi = 0; pi < NW; ++pi) {
+                const float mp = sm_m[pi * kDecodeMaxHeads + hh];
+                if (mp == -INFINITY) continue;
+                const float wgt = fast_exp2(mp - M);
+                Ls = fmaf(sm_l[pi * kDecodeMaxHeads + hh], wgt, Ls);
+                Lm = fmaf(sm_lm[pi * kDecodeMaxHeads + hh], wgt, Lm);
+                Od = fmaf(sm_o[(pi * kDecodeMaxHeads + hh) * D + d], wgt, Od);
+            }
+        }
+        const long hq = static_cast<long>(b) * Hq + h0 + hh;
         const long slot = hq * max_splits + split;
-        o_part[slot * D + d] = Ls > 0.f ? Od / Ls : 0.f;
+        // normalised by the sum of the rounded weights the MMA used; lse from the fp32 sum
+        o_part[slot * D + d] = Lm > 0.f ? Od / Lm : 0.f;
         if (d == 0) lse_part[slot] = Ls > 0.f ? (M + fast_log2(Ls)) * 0.69314718055994531f : -INFINITY;
     }
 }
 
-// One warp per (sequence, q head): out = sum_s exp(lse_s - lse) o_s over splits with finite lse,
-// lse = max + ln sum exp(lse_s - max).
+// One CTA of 8 warps per (sequence, q head): out = sum_s exp(lse_s - lse) o_s over splits with
+// finite lse, lse = max + ln sum exp(lse_s - max).  Warp w accumulates splits s = w (mod 8), then
+// the eight partial sums are added through shared memory.
+constexpr int kCombineWarps = 8;
+
 template <int D>
-__global__ void __launch_bounds__(128) decode_combine_kernel(
+__global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part,
     const int32_t* __restrict__ seqlens, __nv_bfloat16* __restrict__ o, float* __restrict__ o_f32,
     float* __restrict__ lse, int B, int Hq, int Smax, int max_splits) {
     constexpr int DPL = D / 32;   // dims per lane
-    const int warp_global = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (warp_global >= B * Hq) return;
-    const int b = warp_global / Hq;
+    __shared__ float sm_acc[kCombineWarps][D];
+    __shared__ float sm_tot[kCombineWarps];
+    const int bh = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = bh / Hq;
     int L = seqlens[b];
     if (L < 1) L = 1;
     if (L > Smax) L = Smax;
     const int nsplit = decode_num_splits(L, max_splits);
-    const long slot0 = static_cast<long>(warp_global) * max_splits;
+    const long slot0 = static_cast<long>(bh) * max_splits;
 
     float M = -INFINITY;
     for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, lse_part[slot0 + s]);
@@ -279,27 +351,42 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
     for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
     float total = 0.f;
     if (M != -INFINITY) {
-        for (int s = 0; s < nsplit; ++s) {
+#pragma unroll 4
+        for (int s = warp; s < nsplit; s += kCombineWarps) {
             const float ls = lse_part[slot0 + s];
-            if (ls == -INFINITY) continue;
-            const float w = __expf(ls - M);
+            const float w = (ls == -INFINITY) ? 0.f : __expf(ls - M);
             total += w;
 #pragma unroll
             for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, o_part[(slot0 + s) * D + lane * DPL + e], acc[e]);
         }
     }
-    const float inv = total > 0.f ? 1.f / total : 0.f;
-    if (o_f32 != nullptr) {
-        float* orow = o_f32 + static_cast<long>(warp_global) * D + lane * DPL;
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) orow[e] = acc[e] * inv;
-    } else {
-        __nv_bfloat16* orow = o + static_cast<long>(warp_global) * D + lane * DPL;
+    for (int e = 0; e < DPL; ++e) sm_acc[warp][lane * DPL + e] = acc[e];
+    if (lane == 0) sm_tot[warp] = total;
+    __syncthreads();
+    if (warp != 0) return;
+    float tot = 0.f;
 #pragma unroll
-        for (int e = 0; e < DPL; e += 2)
-            *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+    for (int w = 0; w < kCombineWarps; ++w) tot += sm_tot[w];
+    const float inv = tot > 0.f ? 1.f / tot : 0.f;
+    float out[DPL];
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) {
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCombineWarps; ++w) a += sm_acc[w][lane * DPL + e];
+        out[e] = a * inv;
     }
-    if (lse != nullptr && lane == 0) lse[warp_global] = total > 0.f ? M + logf(total) : -INFINITY;
+    if (o_f32 != nullptr) {
+        float* orow = o_f32 + static_cast<long>(bh) * D + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) orow[e] = out[e];
+    } else {
+        __nv_bfloat16* orow = o + static_cast<long>(bh) * D + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; e += 2) *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(out[e], out[e + 1]);
+    }
+    if (lse != nullptr && lane == 0) lse[bh] = tot > 0.f ? M + logf(tot) : -INFINITY;
 }
 
 }  // namespace attn
