@@ -45,8 +45,8 @@ constexpr int kTcThreads = 384;
 // the two softmax warpgroups take them.  The launch must provide kTcThreads * kTcLaunchRegsMin
 // registers, which covers 128 * kRegsControl + 256 * kRegsSoftmax; the host checks the compiled
 // register count before every launch.  Per sub-partition (warps w, w+4, w+8 share one):
-// (64 + 2 * 208) * 32 = 15360 <= 16384 registers.
-constexpr int kRegsControl = 64;
+// (72 + 2 * 208) * 32 = 15616 <= 16384 registers.
+constexpr int kRegsControl = 72;
 constexpr int kRegsSoftmax = 208;
 constexpr int kTcLaunchRegsMin = (128 * kRegsControl + 256 * kRegsSoftmax + kTcThreads - 1) / kTcThreads;
 constexpr float kRescaleThreshold = 8.0f;
@@ -268,31 +268,38 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             const int ni = i ? tile[1].nkv : tile[0].nkv;
             bool ok = mbar_wait(ROPE ? bar_q_ready : bar_q_full, 0);
             tc_fence_after();
+            // Descriptors: the high words are constants, the low words advance with the start
+            // address (16-byte units), so an MMA costs one add and the instruction itself.
+            constexpr uint32_t hiK = desc_sw128_hi(1024);
+            const uint32_t qlo = desc_sw128_lo(sQi, 16);
+            const uint32_t kvlo0 = desc_sw128_lo(smem_u32(sKV), 16);
+            const uint32_t vlo0 = desc_sw128_lo(smem_u32(sKV) + C::K_TILES * C::TILE_BYTES, C::TILE_BYTES / C::NBOX);
             auto issue_s = [&](int j) {
-                const uint32_t sK = smem_u32(sKV + (j % C::STAGES) * C::STAGE_BYTES);
+                const uint32_t klo = kvlo0 + ((j % C::STAGES) * C::STAGE_BYTES >> 4);
                 // chains: (Qh,Kh) [+ (Qh,Kl) + (Ql,Kh) with RoPE]
                 constexpr int NCHAIN = ROPE ? 3 : 1;
 #pragma unroll
                 for (int ch = 0; ch < NCHAIN; ++ch) {
-                    const uint32_t qa = sQi + (ch == 2 ? C::TILE_BYTES : 0);
-                    const uint32_t kb = sK + (ch == 1 ? C::TILE_BYTES : 0);
+                    const uint32_t qa = qlo + (ch == 2 ? (C::TILE_BYTES >> 4) : 0);
+                    const uint32_t kb = klo + (ch == 1 ? (C::TILE_BYTES >> 4) : 0);
 #pragma unroll
                     for (int kk = 0; kk < C::KSTEPS; ++kk) {
                         // K step kk: box kk/4, 32-byte column offset (kk%4) inside the 128-byte row
-                        const uint32_t off = (kk >> 2) * (C::TILE_BYTES / C::NBOX) + (kk & 3) * 32;
-                        mma_ss(dS, smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                               idesc_qk, (ch > 0 || kk > 0) ? 1u : 0u);
+                        constexpr uint32_t box16 = (C::TILE_BYTES / C::NBOX) >> 4;
+                        const uint32_t off = (kk >> 2) * box16 + (kk & 3) * 2;
+                        mma_ss(dS, desc_join(qa + off, hiK), desc_join(kb + off, hiK), idesc_qk,
+                               (ch > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
                 mma_commit(s_full);
             };
             auto issue_pv = [&](int j) {
-                const uint32_t sV = smem_u32(sKV + (j % C::STAGES) * C::STAGE_BYTES) + C::K_TILES * C::TILE_BYTES;
+                const uint32_t vlo = vlo0 + ((j % C::STAGES) * C::STAGE_BYTES >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     // keys [16kk, 16kk+16): 16 rows of 128 B in every 64-wide D box
-                    const uint64_t db = smem_desc_sw128(sV + kk * 2048, C::TILE_BYTES / C::NBOX, 1024);
-                    mma_ts(dO, aP + kk * 8, db, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_ts(dO, aP + kk * 8, desc_join(vlo + kk * (2048 >> 4), hiK), idesc_pv,
+                           (j > 0 || kk > 0) ? 1u : 0u);
                 }
                 mma_commit(pv_done);
             };
