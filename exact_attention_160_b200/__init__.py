@@ -31,7 +31,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 # symbols the library exports (kept in step with include/attn_b200.h)
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
            "attn_decode_workspace_size", "attn_decode_noalloc", "rope_apply", "attn_status_string",
-           "attn_last_error", "attn_read_device_status")
+           "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status")
 
 _lib = None
 
@@ -67,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_status_string.argtypes = [I]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_read_device_status.argtypes = [P]
+    lib.attn_selftest_wait_timeout.argtypes = [I, P]
+    lib.attn_selftest_wait_timeout.restype = I
     lib.attn_last_error.argtypes = []
     lib.attn_last_error.restype = ctypes.c_char_p
     for f in (lib.attn_fwd, lib.attn_fwd_ex, lib.attn_decode, lib.rope_apply, lib.attn_read_device_status):

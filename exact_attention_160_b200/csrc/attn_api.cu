@@ -260,7 +260,7 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
                                                       scale * 1.4426950408889634f);
     attn_status s = launch_status("decode_split_kernel");
     if (s != ATTN_OK) return s;
-    decode_combine_kernel<D><<<B * Hq, kCombineWarps * 32, 0, st>>>(
+    decode_combine_kernel<D><<<B * Hq, kCombineThreads, 0, st>>>(
         o_part, lse_part, seqlens, o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
         o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Hq, Smax, num_splits);
     return launch_status("decode_combine_kernel");
@@ -427,6 +427,13 @@ attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float b
         rope_apply_kernel<float><<<grid, 128, smem, st>>>(static_cast<float*>(x), pos, T, H, D,
                                                           static_cast<double>(base));
     return launch_status("rope_apply_kernel");
+}
+
+attn_status attn_selftest_wait_timeout(int timeout_us, attn_stream_t stream) {
+    if (timeout_us < 1 || timeout_us > 1000000) return ATTN_ERR_INVALID_ARG;
+    wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint64_t>(timeout_us) * 1000ull);
+    return launch_status("wait_timeout_selftest_kernel");
 }
 
 const char* attn_last_error(void) { return g_last_error; }

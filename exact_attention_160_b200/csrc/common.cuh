@@ -76,7 +76,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Returns false (and records a
 // timeout) if that does not happen within kWaitTimeoutNs.  A caller that gets false must stop
 // issuing work and head for the kernel's exit path.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = kWaitTimeoutNs) {
     const uint32_t a = smem_u32(bar);
     if (mbar_try_wait(a, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
@@ -84,11 +84,23 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait(a, parity)) return true;
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        if (globaltimer_ns() - t0 > timeout_ns) {
             record_error(ATTN_DEVICE_ERR_TIMEOUT);
             return false;
         }
     }
+}
+
+// A kernel whose single wait can never complete (nothing arrives on the barrier): the bounded
+// wait gives up after timeout_ns, records ATTN_DEVICE_ERR_TIMEOUT and the kernel returns.
+__global__ void wait_timeout_selftest_kernel(uint64_t timeout_ns) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, timeout_ns);
 }
 
 // ------------------------------------------------------------------------------------------

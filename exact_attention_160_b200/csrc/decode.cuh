@@ -17,7 +17,7 @@
 // kernel run at memory speed.  The S accumulators, exponentiated and rounded to bf16, are the A
 // operand of O += P V directly (no shuffles).
 //
-// Combine kernel: eight warps per (sequence, q head) merge the splits by logsumexp.
+// Combine kernel: one CTA per (sequence, q head) merges the splits by logsumexp.
 #pragma once
 
 #include "common.cuh"
@@ -319,21 +319,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_split_kernel(
     }
 }
 
-// One CTA of 8 warps per (sequence, q head): out = sum_s exp(lse_s - lse) o_s over splits with
-// finite lse, lse = max + ln sum exp(lse_s - max).  Warp w accumulates splits s = w (mod 8), then
-// the eight partial sums are added through shared memory.
-constexpr int kCombineWarps = 8;
+// One CTA of 256 threads per (sequence, q head): out = sum_s exp(lse_s - lse) o_s over splits
+// with finite lse, lse = max + ln sum exp(lse_s - max) (the weights and their max go through
+// shared memory; splits are handled kCombineChunk at a time).  Thread (d, g) accumulates output
+// dim d over the splits s = g (mod 256/D), issuing independent coalesced loads, and the partial
+// sums of the groups are added through shared memory.
+constexpr int kCombineThreads = 256;
+constexpr int kCombineChunk = 1024;
 
 template <int D>
-__global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(
+__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(
     const float* __restrict__ o_part, const float* __restrict__ lse_part,
     const int32_t* __restrict__ seqlens, __nv_bfloat16* __restrict__ o, float* __restrict__ o_f32,
     float* __restrict__ lse, int B, int Hq, int Smax, int max_splits) {
-    constexpr int DPL = D / 32;   // dims per lane
-    __shared__ float sm_acc[kCombineWarps][D];
-    __shared__ float sm_tot[kCombineWarps];
+    constexpr int NG = kCombineThreads / D;       // split groups
+    __shared__ float sm_w[kCombineChunk];
+    __shared__ float sm_red[kCombineThreads];
+    __shared__ float sm_acc[NG][D];
     const int bh = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tid = threadIdx.x;
     const int b = bh / Hq;
     int L = seqlens[b];
     if (L < 1) L = 1;
@@ -341,52 +345,52 @@ __global__ void __launch_bounds__(kCombineWarps * 32) decode_combine_kernel(
     const int nsplit = decode_num_splits(L, max_splits);
     const long slot0 = static_cast<long>(bh) * max_splits;
 
+    // global max of the split lse values
     float M = -INFINITY;
-    for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, lse_part[slot0 + s]);
-#pragma unroll
-    for (int off = 16; off >= 1; off /= 2) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-
-    float acc[DPL];
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-    float total = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-        for (int s = warp; s < nsplit; s += kCombineWarps) {
-            const float ls = lse_part[slot0 + s];
-            const float w = (ls == -INFINITY) ? 0.f : __expf(ls - M);
-            total += w;
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) acc[e] = fmaf(w, o_part[(slot0 + s) * D + lane * DPL + e], acc[e]);
-        }
-    }
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) sm_acc[warp][lane * DPL + e] = acc[e];
-    if (lane == 0) sm_tot[warp] = total;
+    for (int s = tid; s < nsplit; s += kCombineThreads) M = fmaxf(M, lse_part[slot0 + s]);
+    sm_red[tid] = M;
     __syncthreads();
-    if (warp != 0) return;
-    float tot = 0.f;
-#pragma unroll
-    for (int w = 0; w < kCombineWarps; ++w) tot += sm_tot[w];
-    const float inv = tot > 0.f ? 1.f / tot : 0.f;
-    float out[DPL];
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) {
-        float a = 0.f;
-#pragma unroll
-        for (int w = 0; w < kCombineWarps; ++w) a += sm_acc[w][lane * DPL + e];
-        out[e] = a * inv;
+    for (int w = kCombineThreads / 2; w >= 1; w /= 2) {
+        if (tid < w) sm_red[tid] = fmaxf(sm_red[tid], sm_red[tid + w]);
+        __syncthreads();
     }
+    M = sm_red[0];
+    __syncthreads();
+
+    const int d = tid % D, g = tid / D;
+    float acc = 0.f, wsum = 0.f;
+    for (int c0 = 0; c0 < nsplit; c0 += kCombineChunk) {
+        const int cn = min(kCombineChunk, nsplit - c0);
+        for (int s = tid; s < cn; s += kCombineThreads) {
+            const float ls = lse_part[slot0 + c0 + s];
+            sm_w[s] = (M == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - M);
+        }
+        __syncthreads();
+#pragma unroll 8
+        for (int s = g; s < cn; s += NG) {
+            const float w = sm_w[s];
+            acc = fmaf(w, o_part[(slot0 + c0 + s) * D + d], acc);
+            wsum += w;
+        }
+        __syncthreads();
+    }
+    sm_acc[g][d] = acc;
+    sm_red[tid] = wsum;
+    __syncthreads();
+    if (tid >= D) return;
+    float a = 0.f, total = 0.f;
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+        a += sm_acc[k][d];
+        total += sm_red[k * D + d];   // group k's weight sum (equal for every d of the group)
+    }
+    const float out = total > 0.f ? a / total : 0.f;
     if (o_f32 != nullptr) {
-        float* orow = o_f32 + static_cast<long>(bh) * D + lane * DPL;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) orow[e] = out[e];
+        o_f32[static_cast<long>(bh) * D + d] = out;
     } else {
-        __nv_bfloat16* orow = o + static_cast<long>(bh) * D + lane * DPL;
-#pragma unroll
-        for (int e = 0; e < DPL; e += 2) *reinterpret_cast<uint32_t*>(orow + e) = pack_bf16x2(out[e], out[e + 1]);
+        o[static_cast<long>(bh) * D + d] = __float2bfloat16_rn(out);
     }
-    if (lse != nullptr && lane == 0) lse[bh] = tot > 0.f ? M + logf(tot) : -INFINITY;
+    if (lse != nullptr && d == 0) lse[bh] = total > 0.f ? M + logf(total) : -INFINITY;
 }
 
 }  // namespace attn

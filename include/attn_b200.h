@@ -168,6 +168,16 @@ const char* attn_status_string(attn_status s);
 const char* attn_last_error(void);
 
 /*
+ * attn_selftest_wait_timeout -- check of the kernels' failure reporting: launches one tiny
+ * kernel whose only wait (an mbarrier nothing arrives on) can never complete.  The wait gives up
+ * after timeout_us microseconds (1 .. 1e6), sets bit 1 in the device status word and the kernel
+ * returns normally; attn_read_device_status then reports it.  The same bounded wait guards every
+ * wait in the attention kernels (with a 2 s bound), so a logic or hardware stall ends with a
+ * status bit rather than a hung GPU.
+ */
+attn_status attn_selftest_wait_timeout(int timeout_us, attn_stream_t stream);
+
+/*
  * Read and clear the device status word (bit 1: a bounded wait gave up; bit 2: a decode
  * sequence length was clamped; bit 4: tensor memory allocation failed).  Synchronises
  * `stream` first.  Returns the bits, or -1 if the read itself failed.

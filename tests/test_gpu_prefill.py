@@ -49,6 +49,9 @@ BF16_CASES = [
     P("rope_gqa_causal", "bf16", 1, 8, 2, 300, 300, 64, True, rope_base=10000.0),
     P("rope_mha_chunked", "bf16", 1, 2, 2, 90, 400, 64, True, rope_base=10000.0, q_pos0=310),
     P("rope_d128", "bf16", 1, 2, 2, 140, 140, 128, True, rope_base=500000.0),
+    # Whisper encoder self-attention shape (whisper-apr attention_generated.rs: 1500 frames,
+    # 6 heads of 64, non-causal)
+    P("whisper_encoder_s1500_h6", "bf16", 1, 6, 6, 1500, 1500, 64, False),
 ]
 
 F32_CASES = [
