@@ -84,29 +84,56 @@ def barrier(dist, device):
 # ------------------------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock and clock-event reasons sampled every millisecond through NVML (read-only
+    queries), so that even a timed region of a few milliseconds gets several samples; falls back
+    to nvidia-smi every 200 ms where NVML is unavailable."""
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
-    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_s: float = 0.001):
         self.idx = gpu_index
-        self.samples = []
+        self.period = period_s
+        self.samples = []          # (sm_mhz, max_mhz, set of reason names)
         self._stop = threading.Event()
         self._t = threading.Thread(target=self._run, daemon=True)
+        self._nvml = None
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self._nvml = pynvml
+        except Exception:
+            self._nvml = None
 
     def _query(self):
+        if self._nvml is not None:
+            n = self._nvml
+            sm = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+            mx = n.nvmlDeviceGetMaxClockInfo(self._h, n.NVML_CLOCK_SM)
+            bits = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            masks = (n.nvmlClocksEventReasonHwSlowdown, n.nvmlClocksEventReasonHwThermalSlowdown,
+                     n.nvmlClocksEventReasonSwThermalSlowdown, n.nvmlClocksEventReasonSwPowerCap)
+            return float(sm), float(mx), {name for name, m in zip(self.NAMES, masks) if bits & m}
         out = subprocess.run(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}",
                               "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-        return [x.strip() for x in out.stdout.strip().split(",")]
+        f = [x.strip() for x in out.stdout.strip().split(",")]
+        return (float(f[0]), float(f[1]),
+                {name for name, v in zip(self.NAMES, f[2:]) if v.lower() == "active"})
 
     def _run(self):
+        period = self.period if self._nvml is not None else 0.2
         while not self._stop.is_set():
             try:
                 self.samples.append(self._query())
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(period)
 
     def __enter__(self):
         self._t.start()
@@ -124,46 +151,30 @@ class ClockSampler:
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
         reasons = set()
-        for s in self.samples:
-            for name, val in zip(self.NAMES, s[2:]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(self.samples)}
+        for _, _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples),
+                "sm_max_mhz": max(s[1] for s in self.samples), "reasons": sorted(reasons),
+                "samples": len(self.samples), "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
-# ------------------------------------------------------------------------------------------
-# peaks and profile evidence
-# ------------------------------------------------------------------------------------------
+def make_l2_flush(torch, device):
+    """Cold-cache preparation run before every timed step, outside its events: write a buffer
+    larger than L2 (evicting the step's inputs), then read another one of the same size so that
+    L2 holds clean lines only and the step does not pay the write-back of the flush."""
+    wbuf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    rbuf = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    sink = torch.empty((), dtype=torch.float32, device=device)
 
-def load_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d, "measured"
-    return dict(FALLBACK_PEAKS), "fallback"
-
-
-def profile_traffic(name: str):
-    """Per-launch DRAM bytes recorded in profiles/<name>.md ('traffic_bytes_per_launch: N'), if the
-    summary is current; None otherwise."""
-    p = os.path.join(ROOT, "profiles", name + ".md")
-    if not os.path.exists(p):
-        return None
-    for line in open(p):
-        if line.strip().startswith("traffic_bytes_per_launch:"):
-            v = line.split(":", 1)[1].strip()
-            return None if v in ("null", "") else float(v)
-    return None
+    def flush():
+        wbuf.zero_()
+        torch.sum(rbuf, out=sink)
+    return flush
 
 
-# ------------------------------------------------------------------------------------------
-# GPU measurement
-# ------------------------------------------------------------------------------------------
+L2_NOTE = "flushed before every timed step (256 MB written, then 256 MB of other data read)"
+
 
 def dev_bf16(bits, torch):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
@@ -200,13 +211,10 @@ def bench_prefill_gpu(w: si.Prefill, args, torch, ea, dist, device):
     ws = None
     if w.rope_base > 0:
         ws = torch.empty(ea.fwd_workspace_bytes(q, k, w.rope_base, w.q_pos0), dtype=torch.uint8, device=device)
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = make_l2_flush(torch, device)
 
     def step():
         ea.attn_fwd_ex(q, k, v, w.scale, w.causal, w.rope_base, w.q_pos0, o=o, lse=lse, workspace=ws)
-
-    def flush():
-        flush_buf.zero_()
 
     launches_per_step = 1 if w.rope_base <= 0 else 3
     with ClockSampler(device.index) as clk:
@@ -243,12 +251,12 @@ def bench_decode_gpu(w: si.Decode, args, torch, ea, dist, device, steps=None):
     o = torch.empty(q.shape, dtype=torch.float32, device=device)
     lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=device)
     ws = torch.empty(ea.decode_workspace_bytes(w.B, w.Hq, w.D, w.num_splits), dtype=torch.uint8, device=device)
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    flush = make_l2_flush(torch, device)
 
     def step():
         ea.attn_decode(q, kc, vc, sl, w.scale, w.num_splits, o=o, lse=lse, workspace=ws)
 
-    ms = time_steps(step, steps or args.steps, args.warmup, lambda: flush_buf.zero_(), torch, dist, device)
+    ms = time_steps(step, steps or args.steps, args.warmup, flush, torch, dist, device)
     if ea.read_device_status() != 0:
         raise RuntimeError("device status set after decode timing")
     kv_bytes = si.decode_kv_bytes(d["seqlens"], w.Hkv, w.D)
@@ -337,7 +345,7 @@ def run_gpu(args):
         launches = r["launches_per_step"] * args.steps
         config = {"workload": w.name, "global_batch": w.B * world, "seq_len": w.Sq, "heads_q": w.Hq,
                   "heads_kv": w.Hkv, "head_dim": w.D, "causal": w.causal, "rope_base": w.rope_base,
-                  "parallelism": f"replicas{world}", "l2": "flushed before every timed step",
+                  "parallelism": f"replicas{world}", "l2": L2_NOTE,
                   "inputs": "seeded synthetic N(0,1) rounded to bf16 (seeded_inputs)"}
     else:
         with ClockSampler(device.index) as clk:
@@ -354,7 +362,7 @@ def run_gpu(args):
         launches = 2 * args.steps
         config = {"workload": w.name, "global_batch": w.B * world, "heads_q": w.Hq, "heads_kv": w.Hkv,
                   "head_dim": w.D, "smax": w.Smax, "num_splits": w.num_splits,
-                  "parallelism": f"replicas{world}", "l2": "flushed before every timed step (cache > L2)"}
+                  "parallelism": f"replicas{world}", "l2": L2_NOTE + "; the cache is also larger than L2"}
 
     out = {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",

@@ -260,9 +260,24 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
                                                       scale * 1.4426950408889634f);
     attn_status s = launch_status("decode_split_kernel");
     if (s != ATTN_OK) return s;
-    decode_combine_kernel<D><<<B * Hq, kCombineThreads, 0, st>>>(
-        o_part, lse_part, seqlens, o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
-        o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Hq, Smax, num_splits);
+    // The combine is a programmatic dependent launch: its CTAs may be scheduled while the last
+    // split CTAs finish, which hides the launch gap; it waits (griddepcontrol.wait) for the
+    // split grid to complete before reading the partials.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(B) * static_cast<unsigned>(Hq));
+    cfg.blockDim = dim3(kCombineThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, static_cast<const float*>(o_part),
+                                             static_cast<const float*>(lse_part), seqlens,
+                                             o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
+                                             o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Hq, Smax, num_splits);
+    if (e != cudaSuccess) return cuda_failure("decode_combine_kernel launch", cudaGetErrorString(e));
     return launch_status("decode_combine_kernel");
 }
 

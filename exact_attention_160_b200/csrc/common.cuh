@@ -91,6 +91,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// Programmatic dependent launch.  A grid launched with programmatic stream serialisation may be
+// scheduled before the grid ahead of it in the stream has finished: once every CTA of that grid
+// has called griddep_launch_dependents (or exited).  griddep_wait blocks until the grid ahead
+// has completed and its memory writes are visible, so everything after it may read them.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // A kernel whose single wait can never complete (nothing arrives on the barrier): the bounded
 // wait gives up after timeout_ns, records ATTN_DEVICE_ERR_TIMEOUT and the kernel returns.
 __global__ void wait_timeout_selftest_kernel(uint64_t timeout_ns) {

@@ -317,6 +317,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 3) decode_split_kernel(
         o_part[slot * D + d] = Lm > 0.f ? Od / Lm : 0.f;
         if (d == 0) lse_part[slot] = Ls > 0.f ? (M + fast_log2(Ls)) * 0.69314718055994531f : -INFINITY;
     }
+    // this CTA's partials are written: the combine grid may be scheduled (it still waits for
+    // the whole grid to finish before it reads them)
+    griddep_launch_dependents();
 }
 
 // One CTA of 256 threads per (sequence, q head): out = sum_s exp(lse_s - lse) o_s over splits
@@ -344,6 +347,9 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(
     if (L > Smax) L = Smax;
     const int nsplit = decode_num_splits(L, max_splits);
     const long slot0 = static_cast<long>(bh) * max_splits;
+    // launched as a programmatic dependent of the split kernel: its partials are complete and
+    // visible only after this wait
+    griddep_wait();
 
     // global max of the split lse values
     float M = -INFINITY;
