@@ -159,6 +159,36 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
+# ------------------------------------------------------------------------------------------
+# peaks and profile evidence
+# ------------------------------------------------------------------------------------------
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def profile_traffic(name: str):
+    """Per-launch DRAM bytes recorded in profiles/<name>.md ('traffic_bytes_per_launch: N'), if the
+    summary is current; None otherwise."""
+    p = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(p):
+        return None
+    for line in open(p):
+        if line.strip().startswith("traffic_bytes_per_launch:"):
+            v = line.split(":", 1)[1].strip()
+            return None if v in ("null", "") else float(v)
+    return None
+
+
+# ------------------------------------------------------------------------------------------
+# GPU measurement
+# ------------------------------------------------------------------------------------------
+
 def make_l2_flush(torch, device):
     """Cold-cache preparation run before every timed step, outside its events: write a buffer
     larger than L2 (evicting the step's inputs), then read another one of the same size so that
@@ -260,8 +290,26 @@ def bench_decode_gpu(w: si.Decode, args, torch, ea, dist, device, steps=None):
     if ea.read_device_status() != 0:
         raise RuntimeError("device status set after decode timing")
     kv_bytes = si.decode_kv_bytes(d["seqlens"], w.Hkv, w.D)
+
+    # the fused cache append of the same decode step (one new token per sequence, RoPE on the
+    # new key and query): timed on its own, lengths kept below the capacity for every call
+    n_app = (steps or args.steps) + args.warmup
+    sl_app = torch.from_numpy(np.minimum(d["seqlens"], w.Smax - n_app - 1).astype(np.int32)).to(device)
+    kn = torch.zeros((w.B, 1, w.Hkv, w.D), dtype=torch.bfloat16, device=device)
+    vn = torch.zeros_like(kn)
+    qn = torch.zeros((w.B, 1, w.Hq, w.D), dtype=torch.bfloat16, device=device)
+
+    def step_append():
+        ea.kv_append(kc, vc, sl_app, kn, vn, q=qn, rope_base=10000.0)
+
+    ms_app = time_steps(step_append, steps or args.steps, args.warmup, flush, torch, dist, device)
+    if ea.read_device_status() != 0:
+        raise RuntimeError("device status set after the append timing")
+    app_bytes = w.B * (2 * 2 * w.Hkv * w.D * 2 + 2 * w.Hq * w.D * 2)   # k,v read+write; q read+write
     return {"ms": statistics.mean(ms), "kv_bytes": kv_bytes,
-            "qo_bytes": 2 * w.B * w.Hq * w.D * 2 + 4 * w.B * w.Hq}
+            "qo_bytes": 2 * w.B * w.Hq * w.D * 2 + 4 * w.B * w.Hq,
+            "append": {"us_per_call": round(statistics.mean(ms_app) * 1e3, 2), "bytes_per_call": app_bytes,
+                       "what": "attn_kv_append: one token per sequence, RoPE on k and q, cache write, length advance"}}
 
 
 def cpu_baseline_prefill(w: si.Prefill, max_seconds: float = 30.0):
@@ -338,7 +386,7 @@ def run_gpu(args):
         roof = roofline_prefill(w, r["ms"], peaks, how, profile_traffic("prefill_tc_" + w.name.split("_")[0]))
         extra = {"decode": {"workload": dec_w.name, "value": round(whole_job_rate(dec["kv_bytes"], dec_ms, world) / 1e9, 1),
                             "unit": "GB/s", "ms_per_call": round(dec_ms, 4),
-                            "roofline": roofline_decode(dec, peaks, how)}}
+                            "roofline": roofline_decode(dec, peaks, how), "append": dec["append"]}}
         clocks = r["clocks"]
         e2e = {"value": round(value_e2e, 3), "unit": unit, "h2d_bytes_per_step": r["h2d"],
                "d2h_bytes_per_step": r["d2h"], "ms_per_step": round(ms_e2e, 4)}
@@ -356,7 +404,7 @@ def run_gpu(args):
         unit = "GB/s"
         roof = roofline_decode(dec, peaks, how)
         roof["traffic"] = profile_traffic("decode_split_" + w.name.split("_")[0])
-        extra = {}
+        extra = {"append": dec["append"]}
         clocks = clk.summary()
         e2e = None
         launches = 2 * args.steps

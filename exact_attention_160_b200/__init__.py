@@ -31,7 +31,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 # symbols the library exports (kept in step with include/attn_b200.h)
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
            "attn_decode_workspace_size", "attn_decode_noalloc", "rope_apply", "attn_status_string",
-           "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status")
+           "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status", "attn_kv_append")
 
 _lib = None
 
@@ -67,6 +67,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_status_string.argtypes = [I]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_read_device_status.argtypes = [P]
+    lib.attn_kv_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
+    lib.attn_kv_append.restype = I
     lib.attn_selftest_wait_timeout.argtypes = [I, P]
     lib.attn_selftest_wait_timeout.restype = I
     lib.attn_last_error.argtypes = []
@@ -189,6 +191,27 @@ def rope_apply(x, pos, base: float, stream=None):
     st = lib.rope_apply(_ptr(x), _ptr(pos), T, H, D, float(base), _dtype_code(x), _stream(stream))
     _check(st, "rope_apply")
     return x
+
+
+def kv_append(kcache, vcache, seqlens, k_new, v_new, q=None, rope_base: float = 0.0, stream=None):
+    """Append k_new/v_new [B, T, Hkv, D] (bf16) to the caches [B, Smax, Hkv, D] after each
+    sequence's length, rotating keys (and q [B, T, Hq, D], in place) at positions L_b + t when
+    rope_base > 0; advances seqlens [B] (int32, device).  Overflowing sequences are skipped and
+    flagged in the device status word."""
+    lib = load_library()
+    _need_cuda(kcache, vcache, seqlens, k_new, v_new, q)
+    for t in (kcache, vcache, k_new, v_new, q):
+        if t is not None and t.dtype != torch.bfloat16:
+            raise TypeError("kv_append takes bf16 tensors")
+    if seqlens.dtype != torch.int32:
+        raise TypeError("seqlens must be int32")
+    B, Smax, Hkv, D = kcache.shape
+    T = k_new.shape[1]
+    Hq = q.shape[2] if q is not None else Hkv
+    st = lib.attn_kv_append(_ptr(kcache), _ptr(vcache), _ptr(seqlens), _ptr(k_new), _ptr(v_new), _ptr(q), B, T,
+                            Hq, Hkv, Smax, D, float(rope_base), _stream(stream))
+    _check(st, "attn_kv_append")
+    return kcache, vcache, seqlens
 
 
 def read_device_status(stream=None) -> int:

@@ -444,6 +444,25 @@ attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float b
     return launch_status("rope_apply_kernel");
 }
 
+attn_status attn_kv_append(void* kcache, void* vcache, int32_t* seqlens, const void* k_new, const void* v_new,
+                           void* q, int B, int T, int Hq, int Hkv, int Smax, int D, float rope_base,
+                           attn_stream_t stream) {
+    if (B <= 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Smax <= 0 || D <= 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_ERR_DIM_MISMATCH;
+    if (D % 8 != 0) return ATTN_ERR_DIM_MISMATCH;   // value rows move as 16-byte vectors; RoPE needs D even
+    if (!kcache || !vcache || !seqlens || !k_new || !v_new) return ATTN_ERR_INVALID_ARG;
+    if (!isfinite(rope_base)) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(kcache) || !aligned16(vcache) || !aligned16(k_new) || !aligned16(v_new) ||
+        (q != nullptr && !aligned16(q)))
+        return ATTN_ERR_INVALID_ARG;
+    if (B > 65535 * 32) return ATTN_ERR_UNSUPPORTED;
+    kv_append_kernel<<<B, 256, (D / 2) * sizeof(float2), static_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint32_t*>(kcache), static_cast<uint4*>(vcache), seqlens, static_cast<const uint32_t*>(k_new),
+        static_cast<const uint4*>(v_new), static_cast<uint32_t*>(q), T, Hq, Hkv, Smax, D,
+        rope_base > 0.f ? static_cast<double>(rope_base) : 0.0);
+    return launch_status("kv_append_kernel");
+}
+
 attn_status attn_selftest_wait_timeout(int timeout_us, attn_stream_t stream) {
     if (timeout_us < 1 || timeout_us > 1000000) return ATTN_ERR_INVALID_ARG;
     wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(

@@ -21,6 +21,7 @@ enum : int {
     ATTN_DEVICE_ERR_TIMEOUT = 1,      // an mbarrier wait gave up
     ATTN_DEVICE_ERR_SEQLEN = 2,       // a decode sequence length was outside [1, Smax] (clamped)
     ATTN_DEVICE_ERR_TMEM = 4,         // tensor memory allocation returned an unusable address
+    ATTN_DEVICE_ERR_OVERFLOW = 8,     // a cache append would pass the cache capacity (skipped)
 };
 
 // Defined here: the library is a single translation unit (attn_api.cu includes every header).

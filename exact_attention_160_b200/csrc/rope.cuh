@@ -87,4 +87,70 @@ __global__ void rope_split_kv_kernel(const uint32_t* __restrict__ k, uint32_t* _
     }
 }
 
+// Decode-step cache update, fused (scirs2-neural 0.4.4 grouped_query_attention.rs,
+// forward_with_cache: new keys/values go after the cached ones and new Q/K are rotated at the
+// cache offset; whisper-apr 0.3.1 lfm2 KvCache: appending past the capacity is an error).
+// One block per sequence b, so the block alone reads and advances seqlens[b]:
+//   L = seqlens[b]; if L < 0 or L + T > Smax: set ATTN_DEVICE_ERR_OVERFLOW, leave b untouched.
+//   for t < T: kcache[b, L+t] = rope(k_new[b, t], L+t); vcache[b, L+t] = v_new[b, t];
+//              q[b, t] = rope(q[b, t], L+t) in place (q may be null);
+//   seqlens[b] = L + T.
+// All tensors bf16, rows of H*D contiguous elements; rope_base <= 0 copies without rotating.
+__global__ void kv_append_kernel(uint32_t* __restrict__ kcache, uint4* __restrict__ vcache,
+                                 int32_t* __restrict__ seqlens, const uint32_t* __restrict__ k_new,
+                                 const uint4* __restrict__ v_new, uint32_t* __restrict__ q, int T, int Hq,
+                                 int Hkv, int Smax, int D, double base) {
+    extern __shared__ float2 cs[];   // [D/2] cos, sin of the current position
+    __shared__ int s_len;
+    const int b = blockIdx.x;
+    const int half = D / 2;
+    if (threadIdx.x == 0) {
+        const int L = seqlens[b];
+        const bool fits = L >= 0 && static_cast<long>(L) + T <= Smax;
+        if (!fits) record_error(ATTN_DEVICE_ERR_OVERFLOW);
+        s_len = fits ? L : -1;
+    }
+    __syncthreads();
+    const int L = s_len;
+    if (L < 0) return;
+    const bool rot = base > 0.0;
+    const int kpairs = Hkv * half;            // bf16 pairs in one key row
+    const int vvec = Hkv * D / 8;             // 16-byte vectors in one value row
+    const int qpairs = Hq * half;
+    for (int t = 0; t < T; ++t) {
+        const long pos = static_cast<long>(L) + t;
+        if (rot) {
+            for (int i = threadIdx.x; i < half; i += blockDim.x) {
+                double sn, c;
+                sincos(rope_theta(static_cast<double>(pos), i, D, base), &sn, &c);
+                cs[i] = make_float2(static_cast<float>(c), static_cast<float>(sn));
+            }
+            __syncthreads();
+        }
+        const long src_row = static_cast<long>(b) * T + t;
+        const long dst_row = static_cast<long>(b) * Smax + pos;
+        for (int w = threadIdx.x; w < kpairs; w += blockDim.x) {
+            uint32_t v = k_new[src_row * kpairs + w];
+            if (rot) {
+                const float2 r = cs[w % half];
+                const float x0 = bf16lo_to_f32(v), x1 = bf16hi_to_f32(v);
+                v = pack_bf16x2(x0 * r.x - x1 * r.y, x0 * r.y + x1 * r.x);
+            }
+            kcache[dst_row * kpairs + w] = v;
+        }
+        for (int w = threadIdx.x; w < vvec; w += blockDim.x) vcache[dst_row * vvec + w] = v_new[src_row * vvec + w];
+        if (q != nullptr && rot) {
+            for (int w = threadIdx.x; w < qpairs; w += blockDim.x) {
+                uint32_t* pq = q + src_row * qpairs + w;
+                const float2 r = cs[w % half];
+                const uint32_t v = *pq;
+                const float x0 = bf16lo_to_f32(v), x1 = bf16hi_to_f32(v);
+                *pq = pack_bf16x2(x0 * r.x - x1 * r.y, x0 * r.y + x1 * r.x);
+            }
+        }
+        __syncthreads();   // cs is rewritten for the next position
+    }
+    if (threadIdx.x == 0) seqlens[b] = L + T;
+}
+
 }  // namespace attn

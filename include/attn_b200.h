@@ -15,6 +15,8 @@
  *                (flash_decode_tile, combine_tile_outputs, flash_decode_single_head);
  *                whisper-apr 0.3.1 src/model/lfm2/gqa.rs (attention_cached).
  *   rope_apply   the rotation alone, in place.  RotaryPositionEmbedding::apply as above.
+ *   attn_kv_append  decode-step cache append with the new keys and queries rotated at their
+ *                positions.  grouped_query_attention.rs (forward_with_cache); whisper-apr KvCache.
  *
  * Conventions shared by every entry point:
  *   - All tensor pointers are DEVICE pointers (CUDA global memory), row-major and contiguous in
@@ -160,6 +162,28 @@ attn_status attn_decode_noalloc(const void* q, const void* kcache, const void* v
 attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float base, attn_dtype dtype,
                        attn_stream_t stream);
 
+/*
+ * attn_kv_append -- the decode step's cache update, fused into one launch: rotate the new keys
+ * with RoPE at their positions and write them, with the new values, into the cache right after
+ * each sequence's current length; rotate the new queries at the same positions; advance the
+ * lengths.  scirs2-neural 0.4.4 grouped_query_attention.rs (forward_with_cache: new K/V follow
+ * the cached ones, new Q and K are rotated at the cache offset); whisper-apr 0.3.1
+ * src/model/lfm2 KvCache (an append past the capacity is an error).
+ *   kcache, vcache [B, Smax, Hkv, D]  bf16   rows [L_b, L_b + T) written (K rotated)
+ *   seqlens [B]                       int32  device; read as L_b, advanced to L_b + T
+ *   k_new, v_new   [B, T, Hkv, D]     bf16   read
+ *   q              [B, T, Hq, D]      bf16   rotated in place at positions L_b + t; may be NULL
+ *   rope_base > 0: token t of sequence b is rotated at position L_b + t (angles in double, as in
+ *   rope_apply); rope_base <= 0: keys and queries are copied / left unrotated.
+ * Overflow: a sequence with L_b < 0 or L_b + T > Smax is left untouched (cache rows, length and
+ * its q rows) and bit 8 of the device status word is set; the other sequences are appended.
+ * D must be a multiple of 8 (DIM_MISMATCH), all pointers 16-byte aligned.  After the call,
+ * attn_decode with the same seqlens lets each new query see the cache including its own key.
+ */
+attn_status attn_kv_append(void* kcache, void* vcache, int32_t* seqlens, const void* k_new, const void* v_new,
+                           void* q, int B, int T, int Hq, int Hkv, int Smax, int D, float rope_base,
+                           attn_stream_t stream);
+
 /* Static description of a status code.                                                     */
 const char* attn_status_string(attn_status s);
 
@@ -179,7 +203,8 @@ attn_status attn_selftest_wait_timeout(int timeout_us, attn_stream_t stream);
 
 /*
  * Read and clear the device status word (bit 1: a bounded wait gave up; bit 2: a decode
- * sequence length was clamped; bit 4: tensor memory allocation failed).  Synchronises
+ * sequence length was clamped; bit 4: tensor memory allocation failed; bit 8: a cache append
+ * would have passed the capacity and was skipped).  Synchronises
  * `stream` first.  Returns the bits, or -1 if the read itself failed.
  */
 int attn_read_device_status(attn_stream_t stream);

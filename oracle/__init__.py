@@ -167,3 +167,37 @@ def decode_split(q, kcache, vcache, seqlens, scale: float, num_tiles: int):
                                            _ptr(lse), B, Hq, Hkv, Smax, D, float(scale),
                                            int(num_tiles)))
     return o, lse
+
+
+def kv_append(kcache, vcache, seqlens, k_new, v_new, q=None, rope_base: float = 0.0):
+    """The decode step's cache update (scirs2-neural 0.4.4 grouped_query_attention.rs,
+    forward_with_cache / concat_cache: the new keys and values follow the cached ones and the new
+    queries and keys are rotated at the cache offset; whisper-apr 0.3.1 lfm2 KvCache: an append
+    past the capacity is an error).
+
+    kcache/vcache [B,Smax,Hkv,D], seqlens [B], k_new/v_new [B,T,Hkv,D], q [B,T,Hq,D] or None.
+    For each sequence b with L = seqlens[b]: if 0 <= L and L + T <= Smax, rows [L, L+T) take
+    k_new[b] rotated at positions L..L+T-1 (rope_base > 0; unrotated otherwise) and v_new[b];
+    q[b] is rotated at the same positions; the length becomes L + T.  Otherwise sequence b is
+    left as it is and reported.  Returns float64 copies (kcache, vcache, seqlens, q, overflow[B]).
+    """
+    kc = np.array(kcache, dtype=np.float64)
+    vc = np.array(vcache, dtype=np.float64)
+    sl = np.array(seqlens, dtype=np.int64)
+    kn, vn = np.asarray(k_new, dtype=np.float64), np.asarray(v_new, dtype=np.float64)
+    qo = None if q is None else np.array(q, dtype=np.float64)
+    B, Smax = kc.shape[0], kc.shape[1]
+    T = kn.shape[1]
+    overflow = np.zeros(B, dtype=bool)
+    for b in range(B):
+        L = int(sl[b])
+        if L < 0 or L + T > Smax:
+            overflow[b] = True
+            continue
+        pos = np.arange(L, L + T, dtype=np.int32)
+        kc[b, L:L + T] = rope(kn[b], pos, rope_base) if rope_base > 0 else kn[b]
+        vc[b, L:L + T] = vn[b]
+        if qo is not None and rope_base > 0:
+            qo[b] = rope(qo[b], pos, rope_base)
+        sl[b] = L + T
+    return kc, vc, sl, qo, overflow

@@ -150,7 +150,17 @@ C4 = Decode("c4_bf16_decode_B16_Hq32_Hkv8_D64_Smax32768", 16, 32, 8, 64, 32768, 
 C5 = Prefill("c5_bf16_mha_causal_B1_H16_S16384_D128_peaked", "bf16", 1, 16, 16, 16384, 16384, 128,
              True, 1.0 / np.sqrt(128.0), qk_std=3.0, seed=1005)
 
-WORKLOADS = {w.name: w for w in (C1, C2, C3, C4, C5)}
+# Beyond the five configurations: the pages' second prefill workload and the cache-offset case.
+# Whisper encoder self-attention (whisper-apr: 1500 audio frames, 6 heads of 64, no mask), and a
+# chunked prefill -- 512 new query rows at positions 3584..4095 against a 4096-key cache,
+# bottom-right causal, GQA 32/8 with RoPE (scirs2-neural grouped_query_attention.rs
+# forward_with_cache: the cache offset shifts both the mask and the query positions).
+F2_WHISPER = Prefill("f2_bf16_whisper_encoder_B1_H6_S1500_D64", "bf16", 1, 6, 6, 1500, 1500, 64, False,
+                     1.0 / 8.0, seed=1006)
+F2_CHUNK = Prefill("f2_bf16_chunked_prefill_gqa32x8_rope_B2_Sq512_Skv4096_D64", "bf16", 2, 32, 8, 512, 4096,
+                   64, True, 1.0 / 8.0, rope_base=10000.0, q_pos0=3584, seed=1007)
+
+WORKLOADS = {w.name: w for w in (C1, C2, C3, C4, C5, F2_WHISPER, F2_CHUNK)}
 
 
 def prefill_inputs(w: Prefill):

@@ -441,4 +441,97 @@ def pin_sampled_rows_match_full():
         _close(ls[r], lse[b, h, i], 0.0, "sampled LSE")
 
 
+def _append_case(seed, B=3, Smax=12, Hkv=2, G=2, D=8, T=3):
+    kc = normal_f32(seed, 0, (B, Smax, Hkv, D))
+    vc = normal_f32(seed, 1, (B, Smax, Hkv, D))
+    kn = normal_f32(seed, 2, (B, T, Hkv, D))
+    vn = normal_f32(seed, 3, (B, T, Hkv, D))
+    q = normal_f32(seed, 4, (B, T, Hkv * G, D))
+    return kc, vc, kn, vn, q
+
+
+def pin_kv_append_positions_and_copy():
+    """Rows [L, L+T) receive the new tokens; a token at cache position 0 is unrotated (RoPE at
+    position 0 is the identity); values and untouched rows are copied exactly; lengths advance."""
+    kc, vc, kn, vn, q = _append_case(61)
+    sl = np.array([0, 4, 9], dtype=np.int32)
+    k2, v2, s2, q2, ovf = oracle.kv_append(kc, vc, sl, kn, vn, q, rope_base=10000.0)
+    assert not ovf.any() and list(s2) == [3, 7, 12]
+    _close(k2[0, 0], kn[0, 0], 0.0, "position 0 is the identity")
+    _close(q2[0, 0], q[0, 0], 0.0, "query at position 0 unrotated")
+    for b, L in enumerate(sl):
+        _close(v2[b, L:L + 3], vn[b], 0.0, "values copied to rows [L, L+T)")
+        _close(np.delete(v2[b], range(L, L + 3), axis=0), np.delete(vc[b], range(L, L + 3), axis=0), 0.0,
+               "other rows untouched")
+        _close(np.delete(k2[b], range(L, L + 3), axis=0), np.delete(kc[b], range(L, L + 3), axis=0), 0.0,
+               "other key rows untouched")
+    # without RoPE the keys are copied too and q is left alone
+    k3, _, _, q3, _ = oracle.kv_append(kc, vc, sl, kn, vn, q, rope_base=0.0)
+    _close(k3[1, 4:7], kn[1], 0.0, "plain append")
+    _close(q3, q, 0.0, "q untouched without RoPE")
+
+
+def pin_kv_append_same_position_dot():
+    """Query and key of the same new token are rotated by the same angles: their dot product is
+    the unrotated one (closed form, any position)."""
+    kc, vc, kn, vn, q = _append_case(62, G=1)
+    sl = np.array([0, 5, 8], dtype=np.int32)
+    k2, _, _, q2, _ = oracle.kv_append(kc, vc, sl, kn, vn, q, rope_base=500.0)
+    for b, L in enumerate(sl):
+        for t in range(3):
+            got = np.sum(q2[b, t] * k2[b, L + t], axis=-1)
+            ref = np.sum(q[b, t].astype(np.float64) * kn[b, t].astype(np.float64), axis=-1)
+            _close(got, ref, 1e-12, "same-position dot product")
+    # and the rotation is not the identity away from position 0
+    assert np.max(np.abs(k2[1, 5] - kn[1, 0])) > 1e-3
+
+
+def pin_kv_append_chunks_compose():
+    """Appending T tokens at once equals appending them in two chunks."""
+    kc, vc, kn, vn, q = _append_case(63, T=5)
+    sl = np.array([1, 0, 6], dtype=np.int32)
+    a = oracle.kv_append(kc, vc, sl, kn, vn, q, rope_base=10000.0)
+    k1, v1, s1, q1, _ = oracle.kv_append(kc, vc, sl, kn[:, :2], vn[:, :2], q[:, :2], rope_base=10000.0)
+    k2, v2, s2, q2, _ = oracle.kv_append(k1.astype(np.float32), v1.astype(np.float32), s1, kn[:, 2:], vn[:, 2:],
+                                         q[:, 2:], rope_base=10000.0)
+    assert list(s2) == list(a[2])
+    _close(k2, a[0], 2e-6, "keys (the first chunk's rows went through float32 once more)")
+    _close(v2, a[1], 0.0, "values")
+    _close(np.concatenate([q1, q2], axis=1), a[3], 0.0, "queries")
+
+
+def pin_kv_append_then_decode_is_causal_prefill_row():
+    """Append a whole sequence token by token into an empty cache (rotating each new q), decode
+    the last query: equal to the last row of causal prefill with RoPE on the full sequence -- two
+    independent paths of the oracle (append + decode against attn_fwd's own RoPE)."""
+    B, S, Hkv, G, D, Smax = 2, 7, 2, 2, 8, 10
+    kall = normal_f32(64, 0, (B, S, Hkv, D))
+    vall = normal_f32(64, 1, (B, S, Hkv, D))
+    qall = normal_f32(64, 2, (B, S, Hkv * G, D))
+    kc = np.zeros((B, Smax, Hkv, D), dtype=np.float32)
+    vc = np.zeros((B, Smax, Hkv, D), dtype=np.float32)
+    sl = np.zeros(B, dtype=np.int32)
+    for t in range(S):
+        kc, vc, sl, qt, _ = oracle.kv_append(kc, vc, sl, kall[:, t:t + 1], vall[:, t:t + 1], qall[:, t:t + 1],
+                                             rope_base=100.0)
+        kc, vc = kc.astype(np.float32), vc.astype(np.float32)
+    o_dec, l_dec = oracle.decode(qt[:, 0], kc, vc, sl, 0.4)
+    o_pf, l_pf = oracle.attn_fwd(qall, kall, vall, 0.4, True, rope_base=100.0, q_pos0=0)
+    _close(o_dec, o_pf[:, S - 1], 1e-6, "decode after append = last causal row (O)")
+    _close(l_dec, l_pf[:, :, S - 1], 1e-6, "decode after append = last causal row (LSE)")
+
+
+def pin_kv_append_overflow():
+    """A sequence whose append would pass Smax (or with a negative length) is left untouched and
+    reported; the others are appended."""
+    kc, vc, kn, vn, q = _append_case(65)
+    sl = np.array([9, 10, -1], dtype=np.int32)          # Smax 12, T 3: 9 fits, 10 and -1 do not
+    k2, v2, s2, q2, ovf = oracle.kv_append(kc, vc, sl, kn, vn, q, rope_base=10000.0)
+    assert list(ovf) == [False, True, True] and list(s2) == [12, 10, -1]
+    for b in (1, 2):
+        _close(k2[b], kc[b], 0.0, "overflowing sequence keys untouched")
+        _close(v2[b], vc[b], 0.0, "overflowing sequence values untouched")
+        _close(q2[b], q[b], 0.0, "overflowing sequence queries untouched")
+
+
 ALL_PINS = [obj for name, obj in sorted(globals().items()) if name.startswith("pin_")]

@@ -54,3 +54,31 @@ def test_whole_job_rate_counts_all_replicas():
     # 2 replicas of 17.19 GFLOP each, slowest rank 0.06 ms -> 2 * 17.19e9 / 6e-5 FLOP/s
     assert bench.whole_job_rate(17.19e9, 0.06, 2) == pytest.approx(2 * 17.19e9 / 0.06e-3)
     assert bench.whole_job_rate(1.0, 1.0, 1) == pytest.approx(1e3)
+
+
+def test_bench_helpers_read_peaks_and_profile_traffic():
+    """bench.py's host helpers: measured peaks are found, each committed ncu summary gives a
+    per-launch traffic figure, and the module defines every name its GPU path uses."""
+    import ast
+    import builtins
+    import bench
+    peaks, how = bench.load_peaks()
+    assert how in ("measured", "fallback") and peaks["hbm_gbs"] > 0 and peaks["bf16_tflops"] > 0
+    assert bench.profile_traffic("prefill_tc_c2") > 0
+    assert bench.profile_traffic("decode_split_c4") > 0
+    assert bench.profile_traffic("no_such_profile") is None
+    tree = ast.parse(open(bench.__file__).read())
+    defined = set(dir(builtins)) | {"__file__"}
+    for node in ast.walk(tree):
+        if isinstance(node, (ast.FunctionDef, ast.ClassDef)):
+            defined.add(node.name)
+        elif isinstance(node, (ast.Import, ast.ImportFrom)):
+            defined.update((a.asname or a.name).split(".")[0] for a in node.names)
+        elif isinstance(node, ast.Name) and isinstance(node.ctx, (ast.Store, ast.Del)):
+            defined.add(node.id)
+        elif isinstance(node, ast.arg):
+            defined.add(node.arg)
+        elif isinstance(node, ast.ExceptHandler) and node.name:
+            defined.add(node.name)
+    used = {n.id for n in ast.walk(tree) if isinstance(n, ast.Name) and isinstance(n.ctx, ast.Load)}
+    assert not (used - defined), sorted(used - defined)

@@ -39,6 +39,23 @@ def test_full_size_prefill(w):
     assert np.max(np.abs(lg[:, :, 0] - s0)) <= TOL_BF16_LSE
 
 
+@pytest.mark.parametrize("w", [si.F2_WHISPER, si.F2_CHUNK], ids=lambda w: w.name)
+def test_full_size_f2_prefill(w):
+    """Whisper-encoder shape (non-causal) and chunked prefill (Sq < Skv, bottom-right causal,
+    RoPE at the cache offset): sampled rows against the oracle, every output finite."""
+    x, dev = make_prefill(w)
+    o, lse = ea.attn_fwd_ex(dev["q"], dev["k"], dev["v"], w.scale, w.causal, w.rope_base, w.q_pos0,
+                            out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ea.read_device_status() == 0
+    og, lg = to_host_f64(o), to_host_f64(lse)
+    assert np.isfinite(og).all() and np.isfinite(lg).all()
+    rows = sample_rows(w, 400, seed=2)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.rope_base, w.q_pos0, rows=rows)
+    go, gl = gather_rows(og, lg, rows, w)
+    compare(go, ro, gl, rl, TOL_BF16_O, TOL_BF16_LSE, w.name)
+
+
 def test_full_size_decode():
     w = si.C4
     d = si.decode_inputs(w)      # rows past each length hold NaN

@@ -60,3 +60,40 @@ def test_pins_reject_planted_mistake(name, orig, planted, tmp_path):
     finally:
         oracle.swap_library(None)
     assert failed, f"planted mistake {name!r} passed every pin"
+
+
+# Planted mistakes in the Python-level cache append (oracle.kv_append): each is a source edit of
+# the function, applied to a copy that temporarily replaces it.
+import inspect
+import textwrap
+
+APPEND_MUTANTS = [
+    ("append_position_off_by_one", "pos = np.arange(L, L + T, dtype=np.int32)",
+     "pos = np.arange(L + 1, L + T + 1, dtype=np.int32)"),
+    ("append_rows_shifted", "kc[b, L:L + T] = rope(", "kc[b, L + 1:L + T + 1] = rope("),
+    ("append_length_not_advanced", "sl[b] = L + T", "sl[b] = L"),
+    ("append_q_not_rotated", "qo[b] = rope(qo[b], pos, rope_base)", "pass"),
+    ("append_overflow_ignored", "if L < 0 or L + T > Smax:", "if L < 0:"),
+    ("append_positions_from_zero", "pos = np.arange(L, L + T, dtype=np.int32)",
+     "pos = np.arange(0, T, dtype=np.int32)"),
+]
+
+
+@pytest.mark.parametrize("name,orig,planted", APPEND_MUTANTS, ids=[m[0] for m in APPEND_MUTANTS])
+def test_pins_reject_planted_append_mistake(name, orig, planted):
+    src = textwrap.dedent(inspect.getsource(oracle.kv_append))
+    assert src.count(orig) == 1, f"mutation site for {name} not found"
+    ns = dict(vars(oracle))
+    exec(src.replace(orig, planted, 1), ns)
+    real = oracle.kv_append
+    oracle.kv_append = ns["kv_append"]
+    failed = []
+    try:
+        for pin in ALL_PINS:
+            try:
+                pin()
+            except (AssertionError, oracle.OracleError, FloatingPointError, ValueError, IndexError):
+                failed.append(pin.__name__)
+    finally:
+        oracle.kv_append = real
+    assert failed, f"planted mistake {name!r} passed every pin"
