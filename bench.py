@@ -199,7 +199,7 @@ def make_l2_flush(torch, device):
 
     def flush():
         wbuf.zero_()
-        torch.sum(rbuf, out=sink)
+        torch.sum(rbuf, dim=0, out=sink)
     return flush
 
 
