@@ -286,7 +286,8 @@ def bench_decode_gpu(w: si.Decode, args, torch, ea, dist, device, steps=None):
     def step():
         ea.attn_decode(q, kc, vc, sl, w.scale, w.num_splits, o=o, lse=lse, workspace=ws)
 
-    ms = time_steps(step, steps or args.steps, args.warmup, flush, torch, dist, device)
+    # the cache (~0.5 GB) is larger than L2, so decode calls run back to back without a flush
+    ms = time_steps(step, steps or args.steps, args.warmup, lambda: None, torch, dist, device)
     if ea.read_device_status() != 0:
         raise RuntimeError("device status set after decode timing")
     kv_bytes = si.decode_kv_bytes(d["seqlens"], w.Hkv, w.D)
@@ -384,7 +385,8 @@ def run_gpu(args):
         dec_ms = max_over_ranks(dec["ms"], dist, device)
         dec["ms"] = dec_ms
         roof = roofline_prefill(w, r["ms"], peaks, how, profile_traffic("prefill_tc_" + w.name.split("_")[0]))
-        extra = {"decode": {"workload": dec_w.name, "value": round(whole_job_rate(dec["kv_bytes"], dec_ms, world) / 1e9, 1),
+        extra = {"decode": {"workload": dec_w.name, "l2": "not flushed: the cache is larger than L2",
+                            "value": round(whole_job_rate(dec["kv_bytes"], dec_ms, world) / 1e9, 1),
                             "unit": "GB/s", "ms_per_call": round(dec_ms, 4),
                             "roofline": roofline_decode(dec, peaks, how), "append": dec["append"]}}
         clocks = r["clocks"]
@@ -410,7 +412,7 @@ def run_gpu(args):
         launches = 2 * args.steps
         config = {"workload": w.name, "global_batch": w.B * world, "heads_q": w.Hq, "heads_kv": w.Hkv,
                   "head_dim": w.D, "smax": w.Smax, "num_splits": w.num_splits,
-                  "parallelism": f"replicas{world}", "l2": L2_NOTE + "; the cache is also larger than L2"}
+                  "parallelism": f"replicas{world}", "l2": "not flushed: the cache is larger than L2 (the append timing flushes: " + L2_NOTE + ")"}
 
     out = {"metric": METRIC, "value": round(value, 3), "unit": unit, "n_gpus": world, "steps": args.steps,
            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
