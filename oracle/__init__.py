@@ -45,8 +45,9 @@ def _bind(path: str):
         lib.oracle_attn_fwd_tiled_f64.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Dd, I, I, I]
         lib.oracle_decode_f64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, Dd]
         lib.oracle_decode_split_f64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, Dd, I]
+        lib.oracle_attn_bwd_f64.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
         for f in (lib.oracle_rope_f64, lib.oracle_attn_fwd_f64, lib.oracle_attn_fwd_tiled_f64,
-                  lib.oracle_decode_f64, lib.oracle_decode_split_f64):
+                  lib.oracle_decode_f64, lib.oracle_decode_split_f64, lib.oracle_attn_bwd_f64):
             f.restype = I
     return lib
 
@@ -167,6 +168,23 @@ def decode_split(q, kcache, vcache, seqlens, scale: float, num_tiles: int):
                                            _ptr(lse), B, Hq, Hkv, Smax, D, float(scale),
                                            int(num_tiles)))
     return o, lse
+
+
+def attn_bwd(q, k, v, dout, scale: float, causal: bool, rope_base: float = 0.0, q_pos0: int = 0):
+    """Gradients (dq [B,Sq,Hq,D], dk, dv [B,Skv,Hkv,D], float64) of the forward's o for the
+    upstream gradient dout [B,Sq,Hq,D] -- the definition, see oracle_attn_bwd_f64."""
+    q, k, v, dout = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    if k.shape != (B, Skv, Hkv, D) or v.shape != k.shape or dout.shape != q.shape:
+        raise OracleError("dimension mismatch")
+    dq = np.empty((B, Sq, Hq, D), dtype=np.float64)
+    dk = np.empty((B, Skv, Hkv, D), dtype=np.float64)
+    dv = np.empty((B, Skv, Hkv, D), dtype=np.float64)
+    _check(_load().oracle_attn_bwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
+                                       B, Hq, Hkv, Sq, Skv, D, float(scale), int(bool(causal)),
+                                       float(rope_base), int(q_pos0)))
+    return dq, dk, dv
 
 
 def kv_append(kcache, vcache, seqlens, k_new, v_new, q=None, rope_base: float = 0.0):

@@ -455,3 +455,117 @@ int oracle_decode_split_f64(const float* q, const float* kc, const float* vc,
     }
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Backward                                                                                    */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Gradients of the forward above with respect to q, k and v for an upstream gradient dout of o,
+ * written from the definition (the backward of [P1] flash_backward_head, FA-2's Algorithm 4,
+ * without its blocking; [P2] GQA backward: a kv head's gradients are summed over the q heads of
+ * its group and the RoPE rotation is undone on dq and dk).  For every (b, q head, row i), with
+ * s_j and p_j the scores and probabilities of attn_row (p_j = 0 for masked keys):
+ *   dP_j  = sum_d dout_d V_jd
+ *   Dsum  = sum_j p_j dP_j
+ *   dS_j  = p_j (dP_j - Dsum)
+ *   dq_r  = scale * sum_j dS_j K_j          (K, q as rotated in the forward)
+ *   dk_r[j] += scale * dS_j q_r,   dv[j] += p_j dout
+ * and finally dq = R(-theta) dq_r, dk = R(-theta) dk_r: the transpose of a rotation is the
+ * rotation by the negated angle.  A row with no visible key contributes nothing.
+ * q, dout [B,Sq,Hq,D]; k, v [B,Skv,Hkv,D] (float32 values); dq [B,Sq,Hq,D], dk, dv [B,Skv,Hkv,D]
+ * (double).                                                                                  */
+int oracle_attn_bwd_f64(const float* q, const float* k, const float* v, const float* dout,
+                        double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Sq, int Skv,
+                        int D, double scale, int causal, double rope_base, int q_pos0) {
+    int st = check_dims(B, Hq, Hkv, Sq, Skv, D);
+    if (st) return st;
+    if (rope_base > 0.0 && D % 2) return ORACLE_ERR_INVALID_ARG;
+    const int g = Hq / Hkv;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+    for (int b = 0; b < B; ++b) {
+        for (int kvh = 0; kvh < Hkv; ++kvh) {
+            double* Kd = (double*)malloc(sizeof(double) * (size_t)Skv * D);
+            double* Vd = (double*)malloc(sizeof(double) * (size_t)Skv * D);
+            double* dKr = (double*)calloc((size_t)Skv * D, sizeof(double));
+            double* dVa = (double*)calloc((size_t)Skv * D, sizeof(double));
+            double* s = (double*)malloc(sizeof(double) * (size_t)Skv);
+            double* p = (double*)malloc(sizeof(double) * (size_t)Skv);
+            double* dP = (double*)malloc(sizeof(double) * (size_t)Skv);
+            double* qd = (double*)malloc(sizeof(double) * (size_t)D);
+            double* go = (double*)malloc(sizeof(double) * (size_t)D);
+            double* dqr = (double*)malloc(sizeof(double) * (size_t)D);
+            if (!Kd || !Vd || !dKr || !dVa || !s || !p || !dP || !qd || !go || !dqr) {
+#pragma omp atomic write
+                fail = 1;
+            } else {
+                gather_head(k, b, kvh, Skv, Hkv, D, rope_base, Kd);
+                gather_head(v, b, kvh, Skv, Hkv, D, 0.0, Vd);
+                for (int hg = 0; hg < g; ++hg) {
+                    const int hq = kvh * g + hg;
+                    for (int i = 0; i < Sq; ++i) {
+                        const long qoff = (((long)b * Sq + i) * Hq + hq) * D;
+                        double* dqo = dq + qoff;
+                        const int nvis = visible_keys(i, Sq, Skv, causal);
+                        if (nvis <= 0) {
+                            for (int d = 0; d < D; ++d) dqo[d] = 0.0;
+                            continue;
+                        }
+                        for (int d = 0; d < D; ++d) qd[d] = (double)q[qoff + d];
+                        if (rope_base > 0.0) rope_vec(qd, (double)q_pos0 + (double)i, D, rope_base);
+                        for (int d = 0; d < D; ++d) go[d] = (double)dout[qoff + d];
+                        /* scores and the three-pass softmax over the visible keys */
+                        double m = -INFINITY;
+                        for (int j = 0; j < nvis; ++j) {
+                            double dot = 0.0;
+                            for (int d = 0; d < D; ++d) dot += qd[d] * Kd[(long)j * D + d];
+                            s[j] = scale * dot;
+                            if (s[j] > m) m = s[j];
+                        }
+                        double l = 0.0;
+                        for (int j = 0; j < nvis; ++j) l += exp(s[j] - m);
+                        double Dsum = 0.0;
+                        for (int j = 0; j < nvis; ++j) {
+                            p[j] = exp(s[j] - m) / l;
+                            double dot = 0.0;
+                            for (int d = 0; d < D; ++d) dot += go[d] * Vd[(long)j * D + d];
+                            dP[j] = dot;
+                            Dsum += p[j] * dP[j];
+                        }
+                        for (int d = 0; d < D; ++d) dqr[d] = 0.0;
+                        for (int j = 0; j < nvis; ++j) {
+                            const double dS = p[j] * (dP[j] - Dsum);
+                            for (int d = 0; d < D; ++d) {
+                                dqr[d] += scale * dS * Kd[(long)j * D + d];
+                                dKr[(long)j * D + d] += scale * dS * qd[d];
+                                dVa[(long)j * D + d] += p[j] * go[d];
+                            }
+                        }
+                        if (rope_base > 0.0) rope_vec(dqr, -((double)q_pos0 + (double)i), D, rope_base);
+                        for (int d = 0; d < D; ++d) dqo[d] = dqr[d];
+                    }
+                }
+                for (int j = 0; j < Skv; ++j) {
+                    double* dkr = dKr + (long)j * D;
+                    if (rope_base > 0.0) rope_vec(dkr, -(double)j, D, rope_base);
+                    const long koff = (((long)b * Skv + j) * Hkv + kvh) * D;
+                    for (int d = 0; d < D; ++d) {
+                        dk[koff + d] = dkr[d];
+                        dv[koff + d] = dVa[(long)j * D + d];
+                    }
+                }
+            }
+            free(Kd);
+            free(Vd);
+            free(dKr);
+            free(dVa);
+            free(s);
+            free(p);
+            free(dP);
+            free(qd);
+            free(go);
+            free(dqr);
+        }
+    }
+    return fail ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}

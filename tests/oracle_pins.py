@@ -534,4 +534,75 @@ def pin_kv_append_overflow():
         _close(q2[b], q[b], 0.0, "overflowing sequence queries untouched")
 
 
+def _grid(x, step=2.0 ** -12):
+    """Round to a 2^-12 grid so that x +- 2^-10 is exact in float32 (finite differences)."""
+    return (np.round(np.asarray(x, dtype=np.float64) / step) * step).astype(np.float32)
+
+
+def _fd_grads(q, k, v, g, scale, causal, rope_base=0.0, q_pos0=0, eps=2.0 ** -10):
+    """Central differences of L = sum(o * g) through the forward oracle, every input element."""
+    def loss(qq, kk, vv):
+        o, _ = oracle.attn_fwd(qq, kk, vv, scale, causal, rope_base, q_pos0)
+        return float(np.sum(o * g.astype(np.float64)))
+    out = []
+    for which in range(3):
+        xs = [q.copy(), k.copy(), v.copy()]
+        grad = np.zeros(xs[which].shape, dtype=np.float64)
+        flat = xs[which].reshape(-1)
+        for idx in range(flat.size):
+            x0 = flat[idx]
+            flat[idx] = x0 + np.float32(eps)
+            lp = loss(*xs)
+            flat[idx] = x0 - np.float32(eps)
+            lm = loss(*xs)
+            flat[idx] = x0
+            grad.reshape(-1)[idx] = (lp - lm) / (2 * eps)
+        out.append(grad)
+    return out
+
+
+def pin_backward_matches_finite_differences():
+    """dq, dk, dv of the backward oracle equal central differences of the *forward* oracle's
+    L = sum(o * dout) -- non-causal MHA, bottom-right causal GQA with Sq < Skv and a fully
+    masked row (Sq > Skv), and RoPE with a query offset."""
+    cases = [
+        dict(B=1, Sq=4, Skv=5, Hq=2, Hkv=2, D=4, scale=0.7, causal=False),
+        dict(B=2, Sq=3, Skv=5, Hq=4, Hkv=2, D=4, scale=0.5, causal=True),
+        dict(B=1, Sq=5, Skv=3, Hq=2, Hkv=1, D=4, scale=0.9, causal=True),       # row 0, 1 fully masked
+        dict(B=1, Sq=3, Skv=4, Hq=2, Hkv=1, D=6, scale=0.6, causal=True, rope_base=50.0, q_pos0=1),
+    ]
+    for n, c in enumerate(cases):
+        q = _grid(normal_f32(81 + n, 0, (c["B"], c["Sq"], c["Hq"], c["D"])))
+        k = _grid(normal_f32(81 + n, 1, (c["B"], c["Skv"], c["Hkv"], c["D"])))
+        v = _grid(normal_f32(81 + n, 2, (c["B"], c["Skv"], c["Hkv"], c["D"])))
+        g = _grid(normal_f32(81 + n, 3, (c["B"], c["Sq"], c["Hq"], c["D"])))
+        rb, qp = c.get("rope_base", 0.0), c.get("q_pos0", 0)
+        dq, dk, dv = oracle.attn_bwd(q, k, v, g, c["scale"], c["causal"], rb, qp)
+        fq, fk, fv = _fd_grads(q, k, v, g, c["scale"], c["causal"], rb, qp)
+        for name, a, b in (("dq", dq, fq), ("dk", dk, fk), ("dv", dv, fv)):
+            _close(a, b, 2e-6 * max(1.0, float(np.max(np.abs(b)))), f"case {n} {name} vs finite differences")
+
+
+def pin_backward_invariants():
+    """Without RoPE each row's dS sums to zero, so the key gradients of a (b, kv head) sum to
+    zero; each row's probabilities sum to one, so the value gradients sum to the sum of dout over
+    rows with a visible key; GQA gradients equal MHA gradients on repeated kv heads, with the
+    kv-head gradients summed over the group."""
+    B, Sq, Skv, Hq, Hkv, D = 2, 7, 9, 4, 2, 8
+    q = normal_f32(91, 0, (B, Sq, Hq, D))
+    k = normal_f32(91, 1, (B, Skv, Hkv, D))
+    v = normal_f32(91, 2, (B, Skv, Hkv, D))
+    g = normal_f32(91, 3, (B, Sq, Hq, D))
+    dq, dk, dv = oracle.attn_bwd(q, k, v, g, 0.4, True)
+    _close(np.sum(dk, axis=1), np.zeros((B, Hkv, D)), 1e-12, "sum over keys of dk")
+    G = Hq // Hkv
+    gsum = np.sum(g.astype(np.float64).reshape(B, Sq, Hkv, G, D), axis=(1, 3))
+    _close(np.sum(dv, axis=1), gsum, 1e-12, "sum over keys of dv = sum of dout")
+    kr, vr = np.repeat(k, G, axis=2), np.repeat(v, G, axis=2)
+    mq, mk, mv = oracle.attn_bwd(q, kr, vr, g, 0.4, True)
+    _close(dq, mq, 1e-12, "GQA dq = MHA dq")
+    _close(dk, mk.reshape(B, Skv, Hkv, G, D).sum(axis=3), 1e-12, "GQA dk = summed MHA dk")
+    _close(dv, mv.reshape(B, Skv, Hkv, G, D).sum(axis=3), 1e-12, "GQA dv = summed MHA dv")
+
+
 ALL_PINS = [obj for name, obj in sorted(globals().items()) if name.startswith("pin_")]

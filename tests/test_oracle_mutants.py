@@ -36,6 +36,15 @@ MUTANTS = [
     ("split_drops_remainder", "int len = base + (t < rem ? 1 : 0);", "int len = base;"),
     ("tiled_no_correction", "for (int d = 0; d < D; ++d) acc[(long)i * D + d] *= c;", ""),
     ("decode_drops_last_key", "attn_row(qq, Kd, Vd, L, D, L, scale", "attn_row(qq, Kd, Vd, L, D, L - 1, scale"),
+    # backward
+    ("bwd_dq_no_scale", "dqr[d] += scale * dS * Kd[(long)j * D + d];", "dqr[d] += dS * Kd[(long)j * D + d];"),
+    ("bwd_no_dsum", "const double dS = p[j] * (dP[j] - Dsum);", "const double dS = p[j] * dP[j];"),
+    ("bwd_dv_from_ds", "dVa[(long)j * D + d] += p[j] * go[d];", "dVa[(long)j * D + d] += p[j] * dP[j] * go[d];"),
+    ("bwd_dk_rope_not_undone", "if (rope_base > 0.0) rope_vec(dkr, -(double)j, D, rope_base);",
+     "if (rope_base > 0.0) rope_vec(dkr, (double)j, D, rope_base);"),
+    ("bwd_dq_rope_not_undone", "if (rope_base > 0.0) rope_vec(dqr, -((double)q_pos0 + (double)i), D, rope_base);", ""),
+    ("bwd_dp_from_keys", "for (int d = 0; d < D; ++d) dot += go[d] * Vd[(long)j * D + d];",
+     "for (int d = 0; d < D; ++d) dot += go[d] * Kd[(long)j * D + d];"),
 ]
 
 
