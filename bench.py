@@ -313,6 +313,30 @@ def bench_decode_gpu(w: si.Decode, args, torch, ea, dist, device, steps=None):
                        "what": "attn_kv_append: one token per sequence, RoPE on k and q, cache write, length advance"}}
 
 
+def bench_backward_gpu(w: si.Prefill, args, torch, ea, dist, device, steps=None):
+    """attn_bwd on the same workload: bf16 inputs, the forward's o and lse, fp32 gradients; L2
+    flushed before every call.  Algorithmic work: 10 D FLOP per unmasked (query, key) pair -- the
+    method recomputes S (2D) and forms dP, dV, dQ, dK (2D each)."""
+    x = si.prefill_inputs(w)
+    q, k, v = (dev_bf16(x[n + "_bits"], torch) for n in ("q", "k", "v"))
+    dout = dev_bf16(si.bf16_normal(w.seed, 7, (w.B, w.Sq, w.Hq, w.D))[0], torch)
+    ws_f = None
+    if w.rope_base > 0:
+        ws_f = torch.empty(ea.fwd_workspace_bytes(q, k, w.rope_base, w.q_pos0), dtype=torch.uint8, device=device)
+    o, lse = ea.attn_fwd_ex(q, k, v, w.scale, w.causal, w.rope_base, w.q_pos0, workspace=ws_f)
+    ws = torch.empty(ea.bwd_workspace_bytes(q, k, w.rope_base, w.q_pos0), dtype=torch.uint8, device=device)
+    flush = make_l2_flush(torch, device)
+
+    def step():
+        ea.attn_bwd(q, k, v, o, lse, dout, w.scale, w.causal, w.rope_base, w.q_pos0, grad_dtype=torch.float32,
+                    workspace=ws)
+
+    ms = time_steps(step, steps or args.steps, args.warmup, flush, torch, dist, device)
+    if ea.read_device_status() != 0:
+        raise RuntimeError("device status set after the backward timing")
+    return {"ms": statistics.mean(ms), "flop": 2.5 * w.flops}
+
+
 def cpu_baseline_prefill(w: si.Prefill, max_seconds: float = 30.0):
     """The fp64 oracle on a bounded sample of the workload's rows (all (b, h), every r-th row)."""
     import oracle
@@ -385,7 +409,18 @@ def run_gpu(args):
         dec_ms = max_over_ranks(dec["ms"], dist, device)
         dec["ms"] = dec_ms
         roof = roofline_prefill(w, r["ms"], peaks, how, profile_traffic("prefill_tc_" + w.name.split("_")[0]))
-        extra = {"decode": {"workload": dec_w.name, "l2": "not flushed: the cache is larger than L2",
+        bwd = bench_backward_gpu(w, args, torch, ea, dist, device, steps=max(5, args.steps // 3))
+        bwd_ms = max_over_ranks(bwd["ms"], dist, device)
+        fma_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12   # fp32 FFMA, TFLOP/s
+        bwd_tf = whole_job_rate(bwd["flop"], bwd_ms, world) / 1e12
+        extra_bwd = {"workload": w.name, "what": "attn_bwd: dq, dk, dv (fp32) from bf16 q, k, v, o, dout and lse",
+                     "value": round(bwd_tf, 2), "unit": "TFLOP/s", "ms_per_call": round(bwd_ms, 4),
+                     "algorithmic_flop_per_call": bwd["flop"],
+                     "roofline": {"bound": "alu", "achieved": round(bwd_tf / world, 2), "peak": round(fma_peak, 1),
+                                  "unit": "TFLOP/s", "frac": round(bwd_tf / world / fma_peak, 4),
+                                  "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 FLOP at the maximum SM clock"}}
+        extra = {"backward": extra_bwd,
+                 "decode": {"workload": dec_w.name, "l2": "not flushed: the cache is larger than L2",
                             "value": round(whole_job_rate(dec["kv_bytes"], dec_ms, world) / 1e9, 1),
                             "unit": "GB/s", "ms_per_call": round(dec_ms, 4),
                             "roofline": roofline_decode(dec, peaks, how), "append": dec["append"]}}

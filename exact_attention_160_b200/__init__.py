@@ -31,7 +31,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 # symbols the library exports (kept in step with include/attn_b200.h)
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
            "attn_decode_workspace_size", "attn_decode_noalloc", "rope_apply", "attn_status_string",
-           "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status", "attn_kv_append")
+           "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status", "attn_kv_append",
+           "attn_bwd", "attn_bwd_workspace_size")
 
 _lib = None
 
@@ -67,6 +68,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_status_string.argtypes = [I]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_read_device_status.argtypes = [P]
+    lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
+    lib.attn_bwd.restype = I
+    lib.attn_bwd_workspace_size.argtypes = [I, I, I, I, I, I, F, I]
+    lib.attn_bwd_workspace_size.restype = Z
     lib.attn_kv_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_kv_append.restype = I
     lib.attn_selftest_wait_timeout.argtypes = [I, P]
@@ -191,6 +196,38 @@ def rope_apply(x, pos, base: float, stream=None):
     st = lib.rope_apply(_ptr(x), _ptr(pos), T, H, D, float(base), _dtype_code(x), _stream(stream))
     _check(st, "rope_apply")
     return x
+
+
+def bwd_workspace_bytes(q, k, rope_base: float = 0.0, q_pos0: int = 0) -> int:
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    return int(load_library().attn_bwd_workspace_size(B, Hq, Hkv, Sq, Skv, D, float(rope_base), int(q_pos0)))
+
+
+def attn_bwd(q, k, v, o, lse, dout, scale: float, causal: bool, rope_base: float = 0.0, q_pos0: int = 0,
+             grad_dtype=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of the forward for the upstream gradient dout.  o and lse are the
+    forward's outputs.  grad_dtype: torch.float32 to take a bf16 problem's gradients in fp32
+    (default: q's dtype)."""
+    lib = load_library()
+    _need_cuda(q, k, v, o, lse, dout, workspace)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    gd = q.dtype if grad_dtype is None else grad_dtype
+    if q.dtype == torch.float32 and gd != torch.float32:
+        raise TypeError("fp32 inputs take fp32 gradients")
+    code = ATTN_FP32 if q.dtype == torch.float32 else (ATTN_BF16_OUT_F32 if gd == torch.float32 else ATTN_BF16)
+    dq = torch.empty(q.shape, dtype=gd, device=q.device)
+    dk = torch.empty(k.shape, dtype=gd, device=q.device)
+    dv = torch.empty(v.shape, dtype=gd, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(bwd_workspace_bytes(q, k, rope_base, q_pos0), 1), dtype=torch.uint8,
+                                device=q.device)
+    st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq,
+                      Hkv, Sq, Skv, D, float(scale), int(bool(causal)), code, float(rope_base), int(q_pos0),
+                      _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "attn_bwd")
+    return dq, dk, dv
 
 
 def kv_append(kcache, vcache, seqlens, k_new, v_new, q=None, rope_base: float = 0.0, stream=None):

@@ -15,6 +15,7 @@
 #include "prefill_f32.cuh"
 #include "prefill_tc.cuh"
 #include "rope.cuh"
+#include "backward.cuh"
 
 using namespace attn;
 
@@ -281,7 +282,140 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
     return launch_status("decode_combine_kernel");
 }
 
+// Layout of the attn_bwd workspace: rope table (with RoPE), fp32 copies of rotated q, dO,
+// rotated k, v, then D_i = dO . O per row.
+struct BwdWorkspace {
+    size_t tab_off, q_off, do_off, k_off, v_off, d_off, total;
+    int positions;
+};
+
+BwdWorkspace bwd_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, bool rope, int q_pos0) {
+    BwdWorkspace w{};
+    const long pq = static_cast<long>(q_pos0) + Sq;
+    w.positions = rope ? static_cast<int>(pq > Skv ? pq : Skv) : 0;
+    const size_t tab = static_cast<size_t>(w.positions) * (D / 2) * sizeof(float2);
+    const size_t qb = static_cast<size_t>(B) * Sq * Hq * D * sizeof(float);
+    const size_t kb = static_cast<size_t>(B) * Skv * Hkv * D * sizeof(float);
+    w.tab_off = 0;
+    w.q_off = round_up(tab, 256);
+    w.do_off = round_up(w.q_off + qb, 256);
+    w.k_off = round_up(w.do_off + qb, 256);
+    w.v_off = round_up(w.k_off + kb, 256);
+    w.d_off = round_up(w.v_off + kb, 256);
+    w.total = round_up(w.d_off + static_cast<size_t>(B) * Hq * Sq * sizeof(float), 256);
+    return w;
+}
+
+template <int D, typename T>
+attn_status launch_bwd(const T* q, const T* k, const T* v, const T* o, const float* lse, const T* dout, void* dq,
+                       void* dk, void* dv, bool g_f32, int B, int Hq, int Hkv, int Sq, int Skv, float scale,
+                       int causal, const float2* tab, int q_pos0, uint8_t* ws, const BwdWorkspace& w,
+                       cudaStream_t st) {
+    float* Qf = reinterpret_cast<float*>(ws + w.q_off);
+    float* dOf = reinterpret_cast<float*>(ws + w.do_off);
+    float* Kf = reinterpret_cast<float*>(ws + w.k_off);
+    float* Vf = reinterpret_cast<float*>(ws + w.v_off);
+    float* Dvec = reinterpret_cast<float*>(ws + w.d_off);
+    const long nq = static_cast<long>(B) * Sq * Hq, nk = static_cast<long>(B) * Skv * Hkv;
+    bwd_prep_q_kernel<T><<<static_cast<unsigned>((nq * 32 + 255) / 256), 256, 0, st>>>(q, o, dout, Qf, dOf, Dvec, tab,
+                                                                                      nq, Sq, Hq, D, q_pos0);
+    attn_status s = launch_status("bwd_prep_q_kernel");
+    if (s != ATTN_OK) return s;
+    bwd_prep_kv_kernel<T><<<static_cast<unsigned>((nk * 32 + 255) / 256), 256, 0, st>>>(k, v, Kf, Vf, tab, nk, Skv,
+                                                                                       Hkv, D);
+    if ((s = launch_status("bwd_prep_kv_kernel")) != ATTN_OK) return s;
+    BwdParams p{};
+    p.Qf = Qf;
+    p.Kf = Kf;
+    p.Vf = Vf;
+    p.dOf = dOf;
+    p.lse = lse;
+    p.Dvec = Dvec;
+    p.tab = tab;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sq = Sq;
+    p.Skv = Skv;
+    p.q_pos0 = q_pos0;
+    p.causal = causal;
+    p.scale = scale;
+    const size_t smem_dq = 2 * kBwdTile * D * sizeof(float);
+    const size_t smem_dkdv = (2 * kBwdTile * D + 2 * kBwdTile) * sizeof(float);
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem_dq));
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem_dkdv));
+        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(bwd kernels)", cudaGetErrorString(e));
+        attr_set = true;
+    }
+    p.g_f32 = g_f32 ? static_cast<float*>(dq) : nullptr;
+    p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq);
+    bwd_dq_kernel<D><<<dim3((Sq + kBwdRows - 1) / kBwdRows, Hq, B), kBwdThreads, smem_dq, st>>>(p);
+    if ((s = launch_status("bwd_dq_kernel")) != ATTN_OK) return s;
+    p.g_f32 = g_f32 ? static_cast<float*>(dk) : nullptr;
+    p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
+    bwd_dkdv_kernel<D><<<dim3((Skv + kBwdRows - 1) / kBwdRows, Hkv, B), kBwdThreads, smem_dkdv, st>>>(
+        p, g_f32 ? static_cast<float*>(dv) : nullptr, g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv));
+    return launch_status("bwd_dkdv_kernel");
+}
+
 }  // namespace
+
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, float rope_base, int q_pos0) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0 || q_pos0 < 0) return 0;
+    return bwd_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                     int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
+                     size_t workspace_bytes, attn_stream_t stream) {
+    attn_status s = check_common(B, Hq, Hkv, Sq, Skv, D, scale, causal);
+    if (s != ATTN_OK) return s;
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv))
+        return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP32 && dtype != ATTN_BF16_OUT_F32) return ATTN_ERR_INVALID_ARG;
+    const bool rope = rope_base > 0.f;
+    if (rope && !isfinite(rope_base)) return ATTN_ERR_INVALID_ARG;
+    if (q_pos0 < 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq > 65535 || B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+    const BwdWorkspace w = bwd_workspace(B, Hq, Hkv, Sq, Skv, D, rope, q_pos0);
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const float2* tab = nullptr;
+    if (rope) {
+        float2* t = reinterpret_cast<float2*>(ws + w.tab_off);
+        const long n = static_cast<long>(w.positions) * (D / 2);
+        rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, st>>>(
+            t, w.positions, D, static_cast<double>(rope_base));
+        if ((s = launch_status("rope_table_kernel")) != ATTN_OK) return s;
+        tab = t;
+    }
+    const bool g_f32 = dtype != ATTN_BF16;
+    if (dtype == ATTN_FP32) {
+        const float *qf = static_cast<const float*>(q), *kf = static_cast<const float*>(k),
+                    *vf = static_cast<const float*>(v), *of = static_cast<const float*>(o),
+                    *gf = static_cast<const float*>(dout);
+        return D == 64 ? launch_bwd<64>(qf, kf, vf, of, lse, gf, dq, dk, dv, true, B, Hq, Hkv, Sq, Skv, scale, causal,
+                                        tab, q_pos0, ws, w, st)
+                       : launch_bwd<128>(qf, kf, vf, of, lse, gf, dq, dk, dv, true, B, Hq, Hkv, Sq, Skv, scale,
+                                         causal, tab, q_pos0, ws, w, st);
+    }
+    using bf = __nv_bfloat16;
+    const bf *qb = static_cast<const bf*>(q), *kb = static_cast<const bf*>(k), *vb = static_cast<const bf*>(v),
+             *ob = static_cast<const bf*>(o), *gb = static_cast<const bf*>(dout);
+    return D == 64 ? launch_bwd<64>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale, causal,
+                                    tab, q_pos0, ws, w, st)
+                   : launch_bwd<128>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale, causal,
+                                     tab, q_pos0, ws, w, st);
+}
 
 // ------------------------------------------------------------------------------------------
 // Built-in decode scratch for callers that cannot allocate device memory.

@@ -15,6 +15,8 @@
  *                (flash_decode_tile, combine_tile_outputs, flash_decode_single_head);
  *                whisper-apr 0.3.1 src/model/lfm2/gqa.rs (attention_cached).
  *   rope_apply   the rotation alone, in place.  RotaryPositionEmbedding::apply as above.
+ *   attn_bwd     gradients of the forward wrt q, k, v.  flash_attention.rs (flash_backward_head);
+ *                grouped_query_attention.rs (backward).
  *   attn_kv_append  decode-step cache append with the new keys and queries rotated at their
  *                positions.  grouped_query_attention.rs (forward_with_cache); whisper-apr KvCache.
  *
@@ -161,6 +163,31 @@ attn_status attn_decode_noalloc(const void* q, const void* kcache, const void* v
  */
 attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float base, attn_dtype dtype,
                        attn_stream_t stream);
+
+/*
+ * attn_bwd -- gradients of attn_fwd / attn_fwd_ex with respect to q, k and v.
+ *   scirs2-neural 0.4.3 flash_attention.rs (flash_backward_head: FA-2's backward, recomputing the
+ *   probabilities from the saved row statistics); scirs2-neural 0.4.4 grouped_query_attention.rs
+ *   (backward: kv-head gradients summed over the group, RoPE undone on dq and dk).
+ *   q, o, dout [B, Sq, Hq, D]   read (o: the forward's output; dout: gradient of the loss wrt o)
+ *   k, v       [B, Skv, Hkv, D] read
+ *   lse        [B, Hq, Sq] fp32 read: the forward's logsumexp (-inf for rows without a key)
+ *   dq         [B, Sq, Hq, D]   written;  dk, dv [B, Skv, Hkv, D] written
+ *   dtype: ATTN_FP32 (all fp32), ATTN_BF16 (inputs and gradients bf16), ATTN_BF16_OUT_F32
+ *   (bf16 inputs, fp32 gradients).  scale, causal, rope_base, q_pos0: as passed to the forward.
+ *   workspace: >= attn_bwd_workspace_size(...) bytes of device scratch, contents overwritten.
+ * All arithmetic is fp32 (CUDA cores): with fp32 gradients the result matches the definition to
+ * about 1e-6 relative when o and lse are exact; o from the bf16 forward carries its own error
+ * into D_i = dout . o.
+ */
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                     int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
+                     size_t workspace_bytes, attn_stream_t stream);
+
+/* Bytes of workspace attn_bwd needs (fp32 copies of rotated q and k, dout, v, the row sums
+ * D_i and, with RoPE, the angle table); 0 for invalid sizes.                               */
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, float rope_base, int q_pos0);
 
 /*
  * attn_kv_append -- the decode step's cache update, fused into one launch: rotate the new keys
