@@ -70,7 +70,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_read_device_status.argtypes = [P]
     lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
     lib.attn_bwd.restype = I
-    lib.attn_bwd_workspace_size.argtypes = [I, I, I, I, I, I, F, I]
+    lib.attn_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I, F, I]
     lib.attn_bwd_workspace_size.restype = Z
     lib.attn_kv_append.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, F, P]
     lib.attn_kv_append.restype = I
@@ -201,7 +201,8 @@ def rope_apply(x, pos, base: float, stream=None):
 def bwd_workspace_bytes(q, k, rope_base: float = 0.0, q_pos0: int = 0) -> int:
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
-    return int(load_library().attn_bwd_workspace_size(B, Hq, Hkv, Sq, Skv, D, float(rope_base), int(q_pos0)))
+    code = ATTN_FP32 if q.dtype == torch.float32 else ATTN_BF16
+    return int(load_library().attn_bwd_workspace_size(B, Hq, Hkv, Sq, Skv, D, code, float(rope_base), int(q_pos0)))
 
 
 def attn_bwd(q, k, v, o, lse, dout, scale: float, causal: bool, rope_base: float = 0.0, q_pos0: int = 0,

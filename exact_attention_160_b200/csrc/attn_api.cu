@@ -16,6 +16,7 @@
 #include "prefill_tc.cuh"
 #include "rope.cuh"
 #include "backward.cuh"
+#include "backward_mma.cuh"
 
 using namespace attn;
 
@@ -363,11 +364,102 @@ attn_status launch_bwd(const T* q, const T* k, const T* v, const T* o, const flo
     return launch_status("bwd_dkdv_kernel");
 }
 
+// Layout of the bf16 (tensor-core) attn_bwd workspace: rope table, D_i, and with RoPE the
+// rotated q and k as hi/lo bf16 pairs.
+struct BmWorkspace {
+    size_t tab_off, d_off, qh_off, ql_off, kh_off, kl_off, total;
+    int positions;
+};
+
+BmWorkspace bm_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, bool rope, int q_pos0) {
+    BmWorkspace w{};
+    const long pq = static_cast<long>(q_pos0) + Sq;
+    w.positions = rope ? static_cast<int>(pq > Skv ? pq : Skv) : 0;
+    const size_t tab = static_cast<size_t>(w.positions) * (D / 2) * sizeof(float2);
+    const size_t qb = rope ? static_cast<size_t>(B) * Sq * Hq * D * 2 : 0;
+    const size_t kb = rope ? static_cast<size_t>(B) * Skv * Hkv * D * 2 : 0;
+    w.tab_off = 0;
+    w.d_off = round_up(tab, 256);
+    w.qh_off = round_up(w.d_off + static_cast<size_t>(B) * Hq * Sq * sizeof(float), 256);
+    w.ql_off = round_up(w.qh_off + qb, 256);
+    w.kh_off = round_up(w.ql_off + qb, 256);
+    w.kl_off = round_up(w.kh_off + kb, 256);
+    w.total = round_up(w.kl_off + kb, 256);
+    return w;
+}
+
+template <int D, bool ROPE>
+attn_status launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                           const __nv_bfloat16* o, const float* lse, const __nv_bfloat16* dout, void* dq, void* dk,
+                           void* dv, bool g_f32, int B, int Hq, int Hkv, int Sq, int Skv, float scale, int causal,
+                           const float2* tab, int q_pos0, uint8_t* ws, const BmWorkspace& w, cudaStream_t st) {
+    float* Dvec = reinterpret_cast<float*>(ws + w.d_off);
+    const long nq = static_cast<long>(B) * Sq * Hq;
+    bwd_rowdot_kernel<<<static_cast<unsigned>((nq * 32 + 255) / 256), 256, 0, st>>>(o, dout, Dvec, nq, Sq, Hq, D);
+    attn_status s = launch_status("bwd_rowdot_kernel");
+    if (s != ATTN_OK) return s;
+    BmParams p{};
+    p.q = q;
+    p.k = k;
+    if (ROPE) {
+        uint32_t* qh = reinterpret_cast<uint32_t*>(ws + w.qh_off);
+        uint32_t* ql = reinterpret_cast<uint32_t*>(ws + w.ql_off);
+        uint32_t* kh = reinterpret_cast<uint32_t*>(ws + w.kh_off);
+        uint32_t* kl = reinterpret_cast<uint32_t*>(ws + w.kl_off);
+        const long nqp = nq * (D / 2), nkp = static_cast<long>(B) * Skv * Hkv * (D / 2);
+        bwd_rope_split_kernel<<<static_cast<unsigned>(min((nqp + 255) / 256, 148L * 64)), 256, 0, st>>>(
+            reinterpret_cast<const uint32_t*>(q), qh, ql, tab, nqp, Sq, Hq, D, q_pos0);
+        if ((s = launch_status("bwd_rope_split_kernel(q)")) != ATTN_OK) return s;
+        bwd_rope_split_kernel<<<static_cast<unsigned>(min((nkp + 255) / 256, 148L * 64)), 256, 0, st>>>(
+            reinterpret_cast<const uint32_t*>(k), kh, kl, tab, nkp, Skv, Hkv, D, 0);
+        if ((s = launch_status("bwd_rope_split_kernel(k)")) != ATTN_OK) return s;
+        p.q = reinterpret_cast<const __nv_bfloat16*>(qh);
+        p.ql = reinterpret_cast<const __nv_bfloat16*>(ql);
+        p.k = reinterpret_cast<const __nv_bfloat16*>(kh);
+        p.kl = reinterpret_cast<const __nv_bfloat16*>(kl);
+    }
+    p.v = v;
+    p.dout = dout;
+    p.lse = lse;
+    p.Dvec = Dvec;
+    p.tab = tab;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.Sq = Sq;
+    p.Skv = Skv;
+    p.q_pos0 = q_pos0;
+    p.causal = causal;
+    p.scale = scale;
+    using C = BmCfg<D, ROPE>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(bwd_dq_mma_kernel<D, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(bwd_dkdv_mma_kernel<D, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM);
+        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(bwd mma kernels)", cudaGetErrorString(e));
+        attr_set = true;
+    }
+    p.g_f32 = g_f32 ? static_cast<float*>(dq) : nullptr;
+    p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq);
+    bwd_dq_mma_kernel<D, ROPE><<<dim3((Sq + kBmRows - 1) / kBmRows, Hq, B), kBmThreads, C::SMEM, st>>>(p);
+    if ((s = launch_status("bwd_dq_mma_kernel")) != ATTN_OK) return s;
+    p.g_f32 = g_f32 ? static_cast<float*>(dk) : nullptr;
+    p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
+    p.g2_f32 = g_f32 ? static_cast<float*>(dv) : nullptr;
+    p.g2_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
+    bwd_dkdv_mma_kernel<D, ROPE><<<dim3((Skv + kBmRows - 1) / kBmRows, Hkv, B), kBmThreads, C::SMEM, st>>>(p);
+    return launch_status("bwd_dkdv_mma_kernel");
+}
+
 }  // namespace
 
-size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, float rope_base, int q_pos0) {
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
+                               int q_pos0) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0 || q_pos0 < 0) return 0;
-    return bwd_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
+    if (dtype == ATTN_FP32) return bwd_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
+    return bm_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
 }
 
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
@@ -386,12 +478,14 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     if (q_pos0 < 0) return ATTN_ERR_INVALID_ARG;
     if (Hq > 65535 || B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
     const BwdWorkspace w = bwd_workspace(B, Hq, Hkv, Sq, Skv, D, rope, q_pos0);
-    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+    const BmWorkspace wm = bm_workspace(B, Hq, Hkv, Sq, Skv, D, rope, q_pos0);
+    const size_t need = dtype == ATTN_FP32 ? w.total : wm.total;
+    if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const float2* tab = nullptr;
     if (rope) {
-        float2* t = reinterpret_cast<float2*>(ws + w.tab_off);
+        float2* t = reinterpret_cast<float2*>(ws + w.tab_off);   // offset 0 in both layouts
         const long n = static_cast<long>(w.positions) * (D / 2);
         rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, st>>>(
             t, w.positions, D, static_cast<double>(rope_base));
@@ -411,10 +505,15 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     using bf = __nv_bfloat16;
     const bf *qb = static_cast<const bf*>(q), *kb = static_cast<const bf*>(k), *vb = static_cast<const bf*>(v),
              *ob = static_cast<const bf*>(o), *gb = static_cast<const bf*>(dout);
-    return D == 64 ? launch_bwd<64>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale, causal,
-                                    tab, q_pos0, ws, w, st)
-                   : launch_bwd<128>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale, causal,
-                                     tab, q_pos0, ws, w, st);
+    if (D == 64)
+        return rope ? launch_bwd_mma<64, true>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
+                                               causal, tab, q_pos0, ws, wm, st)
+                    : launch_bwd_mma<64, false>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
+                                                causal, tab, q_pos0, ws, wm, st);
+    return rope ? launch_bwd_mma<128, true>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
+                                            causal, tab, q_pos0, ws, wm, st)
+                : launch_bwd_mma<128, false>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
+                                             causal, tab, q_pos0, ws, wm, st);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -1,0 +1,372 @@
+// backward_mma.cuh -- the bf16 backward on the tensor cores (m16n8k16 bf16 MMA, fp32 accumulation).
+//
+// Same method as backward.cuh (FA-2's backward, scirs2-neural 0.4.3 flash_attention.rs
+// flash_backward_head; GQA sums and RoPE undo from grouped_query_attention.rs): every product
+// of the recurrence is a dense 16x8x16 MMA tile --
+//   dq kernel   (4 warps x 16 query rows):   S = Q K^T, dP = dO V^T, dQ += dS K
+//   dkdv kernel (4 warps x 16 keys):       S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q
+// with the probabilities and dS formed in the accumulator registers and reused, rounded to
+// bf16, as the A operand of the next product (no shared-memory round trip).  Tiles of 64 rows
+// of Q, dO, K and V are staged in shared memory with a 16-byte XOR swizzle so that ldmatrix
+// reads are conflict-free.  With RoPE the scores are recomputed from the rotated q and k carried
+// as hi + lo bf16 pairs (S = Qh Kh^T + Qh Kl^T + Ql Kh^T, as in the forward), so P matches the
+// forward's logsumexp; the gradient products use the hi halves.
+#pragma once
+
+#include "common.cuh"
+#include "backward.cuh"
+
+namespace attn {
+
+constexpr int kBmThreads = 128;   // 4 warps x 16 rows = 64 rows per CTA
+constexpr int kBmRows = 64;
+constexpr int kBmTile = 64;       // keys (dq) / query rows (dkdv) per step
+constexpr float kLog2e = 1.4426950408889634f;
+
+// Byte offset of 16-byte chunk ch (8 bf16) of row r in a tile of rows of D bf16, with the low
+// three chunk bits XOR-ed by the row: eight consecutive rows at one chunk hit eight banks groups.
+template <int D>
+__device__ __forceinline__ uint32_t bsw(int r, int ch) {
+    return static_cast<uint32_t>(r * (D * 2) + (((ch & 7) ^ (r & 7)) | (ch & ~7)) * 16);
+}
+
+// Copy 64 rows (row r at src + r*stride elements; rows >= nvalid become zero) into a swizzled tile.
+template <int D>
+__device__ __forceinline__ void stage_rows(uint8_t* tile, const __nv_bfloat16* src, long stride, int nvalid) {
+    for (int idx = threadIdx.x; idx < kBmTile * (D / 8); idx += kBmThreads) {
+        const int r = idx / (D / 8), ch = idx % (D / 8);
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (r < nvalid) v = *reinterpret_cast<const uint4*>(src + r * stride + ch * 8);
+        *reinterpret_cast<uint4*>(tile + bsw<D>(r, ch)) = v;
+    }
+}
+
+struct BmParams {
+    const __nv_bfloat16* q;     // [B, Sq, Hq, D]  (rotated hi half with RoPE)
+    const __nv_bfloat16* ql;    // rotated lo half (RoPE only)
+    const __nv_bfloat16* k;     // [B, Skv, Hkv, D] (rotated hi half with RoPE)
+    const __nv_bfloat16* kl;    // rotated lo half (RoPE only)
+    const __nv_bfloat16* v;
+    const __nv_bfloat16* dout;  // [B, Sq, Hq, D]
+    const float* lse;           // [B, Hq, Sq]
+    const float* Dvec;          // [B, Hq, Sq]
+    const float2* tab;          // (cos, sin) per [position][D/2] (RoPE only)
+    float* g_f32;               // gradient output, fp32 or
+    __nv_bfloat16* g_bf16;      // bf16
+    float* g2_f32;              // dv (dkdv kernel)
+    __nv_bfloat16* g2_bf16;
+    int Hq, Hkv, Sq, Skv, q_pos0, causal;
+    float scale;
+};
+
+// Store a 16-row x D accumulator fragment set (rows g, g+8 of the warp) with optional RoPE undo.
+template <int D>
+__device__ __forceinline__ void bm_store(float (&acc)[D / 8][4], float* f32, __nv_bfloat16* bf16, long row_off0,
+                                         long row_off8, bool live0, bool live8, const float2* cs0, const float2* cs8,
+                                         int t4) {
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd) {
+        float x0 = acc[nd][0], x1 = acc[nd][1], y0 = acc[nd][2], y1 = acc[nd][3];
+        const int pair = nd * 4 + t4;   // dims (8nd + 2t4, +1)
+        if (cs0 != nullptr) rot_pair(x0, x1, cs0[pair], -1.f);
+        if (cs8 != nullptr) rot_pair(y0, y1, cs8[pair], -1.f);
+        const int d = nd * 8 + 2 * t4;
+        if (f32 != nullptr) {
+            if (live0) *reinterpret_cast<float2*>(f32 + row_off0 + d) = make_float2(x0, x1);
+            if (live8) *reinterpret_cast<float2*>(f32 + row_off8 + d) = make_float2(y0, y1);
+        } else {
+            if (live0) *reinterpret_cast<uint32_t*>(bf16 + row_off0 + d) = pack_bf16x2(x0, x1);
+            if (live8) *reinterpret_cast<uint32_t*>(bf16 + row_off8 + d) = pack_bf16x2(y0, y1);
+        }
+    }
+}
+
+// A fragments (16 rows x 16 dims, k step kk) of a swizzled tile, rows r0.. of the warp.
+template <int D>
+__device__ __forceinline__ void lda(uint32_t tile, int r0, int kk, int lane, uint32_t (&a)[4]) {
+    const int m = lane >> 3;
+    ldsm_x4(tile + bsw<D>(r0 + (m & 1) * 8 + (lane & 7), 2 * kk + (m >> 1)), a[0], a[1], a[2], a[3]);
+}
+
+// acc[nt] (16 x 8 for 8 rows nt of `tile`) += A(16 x D) * tile^T, over all k steps.
+template <int D>
+__device__ __forceinline__ void mma_rows_t(float (&acc)[8][4], uint32_t atile, int ar0, uint32_t btile, int lane) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; kk += 2) {
+        uint32_t a0[4], a1[4];
+        lda<D>(atile, ar0, kk, lane, a0);
+        lda<D>(atile, ar0, kk + 1, lane, a1);
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(btile + bsw<D>(nt * 8 + (lane & 7), 2 * kk + (lane >> 3)), b0, b1, b2, b3);
+            mma_bf16_16816(acc[nt], a0[0], a0[1], a0[2], a0[3], b0, b1);
+            mma_bf16_16816(acc[nt], a1[0], a1[1], a1[2], a1[3], b2, b3);
+        }
+    }
+}
+
+// acc (16 x D) += A(16 x 64, given as bf16 fragments per 16-column step) * tile (64 x D).
+template <int D>
+__device__ __forceinline__ void mma_p_tile(float (&acc)[D / 8][4], const uint32_t (&pa)[4][4], uint32_t btile, int lane) {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+#pragma unroll
+        for (int nd = 0; nd < D / 8; nd += 2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(btile + bsw<D>(ks * 16 + ((lane >> 3) & 1) * 8 + (lane & 7), nd + (lane >> 4)), b0, b1, b2, b3);
+            mma_bf16_16816(acc[nd], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b0, b1);
+            mma_bf16_16816(acc[nd + 1], pa[ks][0], pa[ks][1], pa[ks][2], pa[ks][3], b2, b3);
+        }
+    }
+}
+
+// Round 16 x 64 fp32 accumulators (8 column blocks of 8) to the bf16 A fragments of 4 k steps.
+__device__ __forceinline__ void to_afrag(const float (&x)[8][4], uint32_t (&pa)[4][4]) {
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+        pa[ks][0] = pack_bf16x2(x[2 * ks][0], x[2 * ks][1]);
+        pa[ks][1] = pack_bf16x2(x[2 * ks][2], x[2 * ks][3]);
+        pa[ks][2] = pack_bf16x2(x[2 * ks + 1][0], x[2 * ks + 1][1]);
+        pa[ks][3] = pack_bf16x2(x[2 * ks + 1][2], x[2 * ks + 1][3]);
+    }
+}
+
+template <int D, bool ROPE>
+struct BmCfg {
+    static constexpr int TILE = kBmTile * D * 2;                 // bytes of one 64-row bf16 tile
+    // dq kernel: Q, Ql, dO, K, Kl, V.  dkdv kernel: K, Kl, V, Q, Ql, dO (+ lse, D rows)
+    static constexpr int SMEM = (ROPE ? 6 : 4) * TILE + 2 * kBmTile * 4 + 128;
+};
+
+// dQ: CTA (64 query rows, q head h, batch b).
+template <int D, bool ROPE>
+__global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p) {
+    using C = BmCfg<D, ROPE>;
+    extern __shared__ __align__(128) uint8_t bm_smem[];
+    uint8_t* sQ = bm_smem;
+    uint8_t* sQl = sQ + C::TILE;
+    uint8_t* sG = sQl + (ROPE ? C::TILE : 0);
+    uint8_t* sK = sG + C::TILE;
+    uint8_t* sKl = sK + C::TILE;
+    uint8_t* sV = sKl + (ROPE ? C::TILE : 0);
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int kvh = h / (p.Hq / p.Hkv);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int i0 = blockIdx.x * kBmRows;
+    const long qstride = static_cast<long>(p.Hq) * D, kstride = static_cast<long>(p.Hkv) * D;
+    const long qbase = ((static_cast<long>(b) * p.Sq + i0) * p.Hq + h) * D;
+    const int qvalid = min(kBmRows, p.Sq - i0);
+    stage_rows<D>(sQ, p.q + qbase, qstride, qvalid);
+    if (ROPE) stage_rows<D>(sQl, p.ql + qbase, qstride, qvalid);
+    stage_rows<D>(sG, p.dout + qbase, qstride, qvalid);
+    // this thread's two rows: r_a = warp*16 + g, r_b = r_a + 8
+    const int ra = i0 + warp * 16 + g, rb = ra + 8;
+    const long off_c = static_cast<long>(p.Skv) - p.Sq;
+    auto row_state = [&](int i, float& lse2, float& dv, long& nvis) {
+        if (i >= p.Sq) { lse2 = 0.f; dv = 0.f; nvis = 0; return; }
+        const long srow = (static_cast<long>(b) * p.Hq + h) * p.Sq + i;
+        const float l = p.lse[srow];
+        lse2 = l * kLog2e;
+        dv = p.Dvec[srow];
+        long n = p.causal ? static_cast<long>(i) + off_c + 1 : p.Skv;
+        n = n < 0 ? 0 : (n > p.Skv ? p.Skv : n);
+        nvis = (l == -INFINITY) ? 0 : n;
+    };
+    float lse_a, lse_b, d_a, d_b;
+    long nv_a, nv_b;
+    row_state(ra, lse_a, d_a, nv_a);
+    row_state(rb, lse_b, d_b, nv_b);
+    float dq[D / 8][4];
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dq[nd][e] = 0.f;
+    const long last_row = static_cast<long>(i0) + kBmRows - 1;
+    long kmax = p.causal ? last_row + off_c + 1 : p.Skv;
+    kmax = kmax < 0 ? 0 : (kmax > p.Skv ? p.Skv : kmax);
+    const float sl2 = p.scale * kLog2e;
+    const uint32_t uQ = smem_u32(sQ), uQl = smem_u32(sQl), uG = smem_u32(sG);
+    const uint32_t uK = smem_u32(sK), uKl = smem_u32(sKl), uV = smem_u32(sV);
+    for (long k0 = 0; k0 < kmax; k0 += kBmTile) {
+        __syncthreads();
+        const long kbase = ((static_cast<long>(b) * p.Skv + k0) * p.Hkv + kvh) * D;
+        const int kvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Skv - k0));
+        stage_rows<D>(sK, p.k + kbase, kstride, kvalid);
+        if (ROPE) stage_rows<D>(sKl, p.kl + kbase, kstride, kvalid);
+        stage_rows<D>(sV, p.v + kbase, kstride, kvalid);
+        __syncthreads();
+        float s[8][4], dp[8][4];
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
+        mma_rows_t<D>(s, uQ, warp * 16, uK, lane);
+        if (ROPE) {
+            mma_rows_t<D>(s, uQ, warp * 16, uKl, lane);
+            mma_rows_t<D>(s, uQl, warp * 16, uK, lane);
+        }
+        mma_rows_t<D>(dp, uG, warp * 16, uV, lane);
+        // dS * scale in place of s
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const long key = k0 + nt * 8 + 2 * t4 + (e & 1);
+                const bool top = e < 2;
+                const bool vis = key < (top ? nv_a : nv_b);
+                const float pr = vis ? fast_exp2(s[nt][e] * sl2 - (top ? lse_a : lse_b)) : 0.f;
+                s[nt][e] = pr * (dp[nt][e] - (top ? d_a : d_b)) * p.scale;
+            }
+        }
+        uint32_t pa[4][4];
+        to_afrag(s, pa);
+        mma_p_tile<D>(dq, pa, uK, lane);
+    }
+    const bool live_a = ra < p.Sq, live_b = rb < p.Sq;
+    const long oa = ((static_cast<long>(b) * p.Sq + ra) * p.Hq + h) * D;
+    const long ob = ((static_cast<long>(b) * p.Sq + rb) * p.Hq + h) * D;
+    const float2* ca = (ROPE && live_a) ? p.tab + static_cast<long>(p.q_pos0 + ra) * (D / 2) : nullptr;
+    const float2* cb = (ROPE && live_b) ? p.tab + static_cast<long>(p.q_pos0 + rb) * (D / 2) : nullptr;
+    bm_store<D>(dq, p.g_f32, p.g_bf16, oa, ob, live_a, live_b, ca, cb, t4);
+}
+
+// dK, dV: CTA (64 keys, kv head, batch b); loops over the group's q heads and the query tiles.
+template <int D, bool ROPE>
+__global__ void __launch_bounds__(kBmThreads) bwd_dkdv_mma_kernel(const BmParams p) {
+    using C = BmCfg<D, ROPE>;
+    extern __shared__ __align__(128) uint8_t bm_smem[];
+    uint8_t* sK = bm_smem;
+    uint8_t* sKl = sK + C::TILE;
+    uint8_t* sV = sKl + (ROPE ? C::TILE : 0);
+    uint8_t* sQ = sV + C::TILE;
+    uint8_t* sQl = sQ + C::TILE;
+    uint8_t* sG = sQl + (ROPE ? C::TILE : 0);
+    float* sL = reinterpret_cast<float*>(sG + C::TILE);   // [64] lse * log2(e)
+    float* sD = sL + kBmTile;                             // [64] D
+    const int kvh = blockIdx.y, b = blockIdx.z;
+    const int G = p.Hq / p.Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, t4 = lane & 3;
+    const int j0 = blockIdx.x * kBmRows;
+    const long qstride = static_cast<long>(p.Hq) * D, kstride = static_cast<long>(p.Hkv) * D;
+    const long kbase = ((static_cast<long>(b) * p.Skv + j0) * p.Hkv + kvh) * D;
+    const int kvalid = min(kBmRows, p.Skv - j0);
+    stage_rows<D>(sK, p.k + kbase, kstride, kvalid);
+    if (ROPE) stage_rows<D>(sKl, p.kl + kbase, kstride, kvalid);
+    stage_rows<D>(sV, p.v + kbase, kstride, kvalid);
+    const int ja = j0 + warp * 16 + g, jb = ja + 8;    // this thread's two keys
+    const long off_c = static_cast<long>(p.Skv) - p.Sq;
+    float dk[D / 8][4], dv[D / 8][4];
+#pragma unroll
+    for (int nd = 0; nd < D / 8; ++nd)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dk[nd][e] = dv[nd][e] = 0.f;
+    long i_lo = p.causal ? static_cast<long>(j0) - off_c : 0;
+    i_lo = i_lo < 0 ? 0 : i_lo;
+    const long i_start = (i_lo / kBmTile) * kBmTile;
+    const float sl2 = p.scale * kLog2e;
+    const uint32_t uQ = smem_u32(sQ), uQl = smem_u32(sQl), uG = smem_u32(sG);
+    const uint32_t uK = smem_u32(sK), uKl = smem_u32(sKl), uV = smem_u32(sV);
+    for (int hg = 0; hg < G; ++hg) {
+        const int h = kvh * G + hg;
+        for (long i0 = i_start; i0 < p.Sq; i0 += kBmTile) {
+            __syncthreads();
+            const long qbase = ((static_cast<long>(b) * p.Sq + i0) * p.Hq + h) * D;
+            const int qvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Sq - i0));
+            stage_rows<D>(sQ, p.q + qbase, qstride, qvalid);
+            if (ROPE) stage_rows<D>(sQl, p.ql + qbase, qstride, qvalid);
+            stage_rows<D>(sG, p.dout + qbase, qstride, qvalid);
+            for (int w = threadIdx.x; w < kBmTile; w += kBmThreads) {
+                const long srow = (static_cast<long>(b) * p.Hq + h) * p.Sq + i0 + w;
+                const bool in = w < qvalid;
+                sL[w] = in ? p.lse[srow] * kLog2e : -INFINITY;
+                sD[w] = in ? p.Dvec[srow] : 0.f;
+            }
+            __syncthreads();
+            float s[8][4], dp[8][4];
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
+            mma_rows_t<D>(s, uK, warp * 16, uQ, lane);        // S^T = K Q^T
+            if (ROPE) {
+                mma_rows_t<D>(s, uK, warp * 16, uQl, lane);
+                mma_rows_t<D>(s, uKl, warp * 16, uQ, lane);
+            }
+            mma_rows_t<D>(dp, uV, warp * 16, uG, lane);       // dP^T = V dO^T
+            // s <- P^T, dp <- dS^T * scale
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int qi = nt * 8 + 2 * t4 + (e & 1);   // query row within the tile
+                    const long key = (e < 2) ? ja : jb;
+                    const float l2 = sL[qi];
+                    const bool vis = key < p.Skv && l2 != -INFINITY &&
+                                     (!p.causal || key <= i0 + qi + off_c);
+                    const float pr = vis ? fast_exp2(s[nt][e] * sl2 - l2) : 0.f;
+                    dp[nt][e] = pr * (dp[nt][e] - sD[qi]) * p.scale;
+                    s[nt][e] = pr;
+                }
+            }
+            uint32_t pa[4][4];
+            to_afrag(s, pa);
+            mma_p_tile<D>(dv, pa, uG, lane);                   // dV += P^T dO
+            to_afrag(dp, pa);
+            mma_p_tile<D>(dk, pa, uQ, lane);                   // dK += dS^T Q
+        }
+    }
+    const bool live_a = ja < p.Skv, live_b = jb < p.Skv;
+    const long oa = ((static_cast<long>(b) * p.Skv + ja) * p.Hkv + kvh) * D;
+    const long ob = ((static_cast<long>(b) * p.Skv + jb) * p.Hkv + kvh) * D;
+    const float2* ca = (ROPE && live_a) ? p.tab + static_cast<long>(ja) * (D / 2) : nullptr;
+    const float2* cb = (ROPE && live_b) ? p.tab + static_cast<long>(jb) * (D / 2) : nullptr;
+    bm_store<D>(dk, p.g_f32, p.g_bf16, oa, ob, live_a, live_b, ca, cb, t4);
+    bm_store<D>(dv, p.g2_f32, p.g2_bf16, oa, ob, live_a, live_b, nullptr, nullptr, t4);
+}
+
+// Rotated q/k for the MMA path: hi = bf16(x'), lo = bf16(x' - hi), x' the rotation in fp32.
+__global__ void bwd_rope_split_kernel(const uint32_t* __restrict__ x, uint32_t* __restrict__ hi,
+                                      uint32_t* __restrict__ lo, const float2* __restrict__ tab, long npairs,
+                                      int S, int H, int D, int pos0) {
+    const int half = D / 2;
+    for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < npairs;
+         idx += static_cast<long>(gridDim.x) * blockDim.x) {
+        const int i = static_cast<int>(idx % half);
+        const long row = idx / half;                 // (b*S + s)*H + h
+        const int sidx = static_cast<int>((row / H) % S);
+        const float2 r = tab[static_cast<long>(pos0 + sidx) * half + i];
+        const uint32_t v = x[idx];
+        float x0 = bf16lo_to_f32(v), x1 = bf16hi_to_f32(v);
+        rot_pair(x0, x1, r, 1.f);
+        const uint32_t h = pack_bf16x2(x0, x1);
+        hi[idx] = h;
+        lo[idx] = pack_bf16x2(x0 - bf16lo_to_f32(h), x1 - bf16hi_to_f32(h));
+    }
+}
+
+// D_i = dO . O per row for the bf16 path (one warp per row).
+__global__ void bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                                  float* __restrict__ Dvec, long nrows, int Sq, int Hq, int D) {
+    const int lane = threadIdx.x & 31;
+    const long row = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    if (row >= nrows) return;
+    const int h = static_cast<int>(row % Hq);
+    const int i = static_cast<int>((row / Hq) % Sq);
+    const long b = row / (static_cast<long>(Hq) * Sq);
+    const uint32_t* op = reinterpret_cast<const uint32_t*>(o + row * D);
+    const uint32_t* gp = reinterpret_cast<const uint32_t*>(dout + row * D);
+    float acc = 0.f;
+    for (int w = lane; w < D / 2; w += 32) {
+        const uint32_t a = op[w], c = gp[w];
+        acc = fmaf(bf16lo_to_f32(a), bf16lo_to_f32(c), acc);
+        acc = fmaf(bf16hi_to_f32(a), bf16hi_to_f32(c), acc);
+    }
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+    if (lane == 0) Dvec[(b * Hq + h) * Sq + i] = acc;
+}
+
+}  // namespace attn

@@ -176,18 +176,22 @@ attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float b
  *   dtype: ATTN_FP32 (all fp32), ATTN_BF16 (inputs and gradients bf16), ATTN_BF16_OUT_F32
  *   (bf16 inputs, fp32 gradients).  scale, causal, rope_base, q_pos0: as passed to the forward.
  *   workspace: >= attn_bwd_workspace_size(...) bytes of device scratch, contents overwritten.
- * All arithmetic is fp32 (CUDA cores): with fp32 gradients the result matches the definition to
- * about 1e-6 relative when o and lse are exact; o from the bf16 forward carries its own error
- * into D_i = dout . o.
+ * ATTN_FP32 runs in fp32 on the CUDA cores (matches the definition to ~1e-6 relative when o and
+ * lse are exact).  The bf16 dtypes run the products on the tensor cores (bf16 operands, fp32
+ * accumulation; P and dS are rounded to bf16 as operands, ~2^-9 relative each); with RoPE the
+ * scores are recomputed from hi + lo bf16 halves of the rotated q and k, as in the forward.
+ * o from the bf16 forward carries its own rounding into D_i = dout . o.
  */
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
                      int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
                      size_t workspace_bytes, attn_stream_t stream);
 
-/* Bytes of workspace attn_bwd needs (fp32 copies of rotated q and k, dout, v, the row sums
+/* Bytes of workspace attn_bwd needs for these sizes and dtype (fp32: fp32 copies of rotated q
+ * and k, dout, v; bf16: the rotated q and k as hi/lo bf16 pairs with RoPE; both: the row sums
  * D_i and, with RoPE, the angle table); 0 for invalid sizes.                               */
-size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, float rope_base, int q_pos0);
+size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
+                               int q_pos0);
 
 /*
  * attn_kv_append -- the decode step's cache update, fused into one launch: rotate the new keys

@@ -3,8 +3,9 @@ differences of the forward oracle).
 
 Tolerances, as a fraction of the largest reference gradient of each tensor:
   * fp32 inputs, o and lse exact to fp32: 2e-5 (fp32 accumulation over <= a few thousand keys);
-  * bf16 inputs: o is stored in bf16, so D_i = dout . o carries o's rounding (2^-9 relative per
-    element) into every dS of the row: 1e-2;
+  * bf16 inputs (tensor-core products): o is stored in bf16, so D_i = dout . o carries o's
+    rounding (2^-9 relative per element) into every dS of the row, and P and dS are rounded to
+    bf16 as MMA operands: 1e-2;
   * the whole chain (the library's bf16 forward, then its backward): 2e-2.
 """
 import numpy as np
@@ -48,6 +49,10 @@ CASES = [
     P("masked_rows", "fp32", 1, 2, 2, 150, 100, 64, True, 0.125, seed=205),
     P("bf16_gqa_rope", "bf16", 1, 8, 2, 160, 160, 64, True, 0.125, rope_base=10000.0, seed=206),
     P("bf16_d128", "bf16", 2, 2, 2, 140, 140, 128, True, 0.0884, seed=207),
+    P("bf16_d128_rope_offset_gqa", "bf16", 1, 4, 2, 100, 170, 128, True, 0.0884, rope_base=500000.0, q_pos0=70,
+      seed=209),
+    P("bf16_noncausal_masked_mqa", "bf16", 2, 4, 1, 77, 200, 64, False, 0.125, seed=210),
+    P("bf16_causal_sq_gt_skv", "bf16", 1, 2, 2, 150, 90, 64, True, 0.125, seed=211),
 ]
 
 
