@@ -411,14 +411,15 @@ def run_gpu(args):
         roof = roofline_prefill(w, r["ms"], peaks, how, profile_traffic("prefill_tc_" + w.name.split("_")[0]))
         bwd = bench_backward_gpu(w, args, torch, ea, dist, device, steps=max(5, args.steps // 3))
         bwd_ms = max_over_ranks(bwd["ms"], dist, device)
-        fma_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12   # fp32 FFMA, TFLOP/s
         bwd_tf = whole_job_rate(bwd["flop"], bwd_ms, world) / 1e12
+        tpk = float(peaks["bf16_tflops"])
         extra_bwd = {"workload": w.name, "what": "attn_bwd: dq, dk, dv (fp32) from bf16 q, k, v, o, dout and lse",
                      "value": round(bwd_tf, 2), "unit": "TFLOP/s", "ms_per_call": round(bwd_ms, 4),
                      "algorithmic_flop_per_call": bwd["flop"],
-                     "roofline": {"bound": "alu", "achieved": round(bwd_tf / world, 2), "peak": round(fma_peak, 1),
-                                  "unit": "TFLOP/s", "frac": round(bwd_tf / world / fma_peak, 4),
-                                  "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 FLOP at the maximum SM clock"}}
+                     "roofline": {"bound": "tensor", "achieved": round(bwd_tf / world, 2), "peak": tpk,
+                                  "unit": "TFLOP/s", "frac": round(bwd_tf / world / tpk, 4),
+                                  "peak_source": how + " bf16_tflops (burst, cuBLAS bf16 GEMM); the backward "
+                                                 "issues m16n8k16 mma.sync, not tcgen05"}}
         extra = {"backward": extra_bwd,
                  "decode": {"workload": dec_w.name, "l2": "not flushed: the cache is larger than L2",
                             "value": round(whole_job_rate(dec["kv_bytes"], dec_ms, world) / 1e9, 1),

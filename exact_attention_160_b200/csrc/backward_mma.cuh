@@ -30,14 +30,26 @@ __device__ __forceinline__ uint32_t bsw(int r, int ch) {
     return static_cast<uint32_t>(r * (D * 2) + (((ch & 7) ^ (r & 7)) | (ch & ~7)) * 16);
 }
 
-// Copy 64 rows (row r at src + r*stride elements; rows >= nvalid become zero) into a swizzled tile.
+// Asynchronous copies global -> shared (cp.async, 16 or 4 bytes; a zero source size fills zeros).
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(valid ? 4 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// stage_rows with cp.async: rows >= nvalid are zero-filled (their source address is row 0).
 template <int D>
-__device__ __forceinline__ void stage_rows(uint8_t* tile, const __nv_bfloat16* src, long stride, int nvalid) {
+__device__ __forceinline__ void stage_rows_async(uint32_t tile, const __nv_bfloat16* src, long stride, int nvalid) {
     for (int idx = threadIdx.x; idx < kBmTile * (D / 8); idx += kBmThreads) {
         const int r = idx / (D / 8), ch = idx % (D / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (r < nvalid) v = *reinterpret_cast<const uint4*>(src + r * stride + ch * 8);
-        *reinterpret_cast<uint4*>(tile + bsw<D>(r, ch)) = v;
+        const bool ok = r < nvalid;
+        cp_async16(tile + bsw<D>(r, ch), src + (ok ? r * stride : 0) + ch * 8, ok);
     }
 }
 
@@ -135,8 +147,10 @@ __device__ __forceinline__ void to_afrag(const float (&x)[8][4], uint32_t (&pa)[
 template <int D, bool ROPE>
 struct BmCfg {
     static constexpr int TILE = kBmTile * D * 2;                 // bytes of one 64-row bf16 tile
-    // dq kernel: Q, Ql, dO, K, Kl, V.  dkdv kernel: K, Kl, V, Q, Ql, dO (+ lse, D rows)
-    static constexpr int SMEM = (ROPE ? 6 : 4) * TILE + 2 * kBmTile * 4 + 128;
+    static constexpr int NT = ROPE ? 3 : 2;                       // streamed tiles per step (K,Kl,V / Q,Ql,dO)
+    static constexpr int STEP = NT * TILE + 2 * kBmTile * 4;      // + lse and D rows (dkdv)
+    // fixed: Q, Ql, dO (dq) or K, Kl, V (dkdv); two buffers of the streamed step
+    static constexpr int SMEM = NT * TILE + 2 * STEP + 128;
 };
 
 // dQ: CTA (64 query rows, q head h, batch b).
@@ -144,26 +158,40 @@ template <int D, bool ROPE>
 __global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p) {
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
-    uint8_t* sQ = bm_smem;
-    uint8_t* sQl = sQ + C::TILE;
-    uint8_t* sG = sQl + (ROPE ? C::TILE : 0);
-    uint8_t* sK = sG + C::TILE;
-    uint8_t* sKl = sK + C::TILE;
-    uint8_t* sV = sKl + (ROPE ? C::TILE : 0);
+    const uint32_t base = smem_u32(bm_smem);
+    const uint32_t uQ = base, uQl = base + C::TILE, uG = base + (C::NT - 1) * C::TILE;
+    auto uK = [&](int buf) { return base + C::NT * C::TILE + buf * C::STEP; };
+    auto uKl = [&](int buf) { return uK(buf) + C::TILE; };
+    auto uV = [&](int buf) { return uK(buf) + (C::NT - 1) * C::TILE; };
     const int h = blockIdx.y, b = blockIdx.z;
     const int kvh = h / (p.Hq / p.Hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t4 = lane & 3;
-    const int i0 = blockIdx.x * kBmRows;
+    // causal: the last row blocks see the most keys, so they are scheduled first
+    const int i0 = (p.causal ? static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x) : blockIdx.x) * kBmRows;
     const long qstride = static_cast<long>(p.Hq) * D, kstride = static_cast<long>(p.Hkv) * D;
     const long qbase = ((static_cast<long>(b) * p.Sq + i0) * p.Hq + h) * D;
     const int qvalid = min(kBmRows, p.Sq - i0);
-    stage_rows<D>(sQ, p.q + qbase, qstride, qvalid);
-    if (ROPE) stage_rows<D>(sQl, p.ql + qbase, qstride, qvalid);
-    stage_rows<D>(sG, p.dout + qbase, qstride, qvalid);
+    const long off_c = static_cast<long>(p.Skv) - p.Sq;
+    const long last_row = static_cast<long>(i0) + kBmRows - 1;
+    long kmax = p.causal ? last_row + off_c + 1 : p.Skv;
+    kmax = kmax < 0 ? 0 : (kmax > p.Skv ? p.Skv : kmax);
+    const int nsteps = static_cast<int>((kmax + kBmTile - 1) / kBmTile);
+    auto issue_step = [&](int t) {
+        const long k0 = static_cast<long>(t) * kBmTile;
+        const long kbase = ((static_cast<long>(b) * p.Skv + k0) * p.Hkv + kvh) * D;
+        const int kvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Skv - k0));
+        stage_rows_async<D>(uK(t & 1), p.k + kbase, kstride, kvalid);
+        if (ROPE) stage_rows_async<D>(uKl(t & 1), p.kl + kbase, kstride, kvalid);
+        stage_rows_async<D>(uV(t & 1), p.v + kbase, kstride, kvalid);
+    };
+    stage_rows_async<D>(uQ, p.q + qbase, qstride, qvalid);
+    if (ROPE) stage_rows_async<D>(uQl, p.ql + qbase, qstride, qvalid);
+    stage_rows_async<D>(uG, p.dout + qbase, qstride, qvalid);
+    if (nsteps > 0) issue_step(0);
+    cp_async_commit();
     // this thread's two rows: r_a = warp*16 + g, r_b = r_a + 8
     const int ra = i0 + warp * 16 + g, rb = ra + 8;
-    const long off_c = static_cast<long>(p.Skv) - p.Sq;
     auto row_state = [&](int i, float& lse2, float& dv, long& nvis) {
         if (i >= p.Sq) { lse2 = 0.f; dv = 0.f; nvis = 0; return; }
         const long srow = (static_cast<long>(b) * p.Hq + h) * p.Sq + i;
@@ -183,31 +211,26 @@ __global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p
     for (int nd = 0; nd < D / 8; ++nd)
 #pragma unroll
         for (int e = 0; e < 4; ++e) dq[nd][e] = 0.f;
-    const long last_row = static_cast<long>(i0) + kBmRows - 1;
-    long kmax = p.causal ? last_row + off_c + 1 : p.Skv;
-    kmax = kmax < 0 ? 0 : (kmax > p.Skv ? p.Skv : kmax);
     const float sl2 = p.scale * kLog2e;
-    const uint32_t uQ = smem_u32(sQ), uQl = smem_u32(sQl), uG = smem_u32(sG);
-    const uint32_t uK = smem_u32(sK), uKl = smem_u32(sKl), uV = smem_u32(sV);
-    for (long k0 = 0; k0 < kmax; k0 += kBmTile) {
+    for (int t = 0; t < nsteps; ++t) {
+        // the next step's tiles load while this one is computed
+        if (t + 1 < nsteps) issue_step(t + 1);
+        cp_async_commit();
+        cp_async_wait<1>();
         __syncthreads();
-        const long kbase = ((static_cast<long>(b) * p.Skv + k0) * p.Hkv + kvh) * D;
-        const int kvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Skv - k0));
-        stage_rows<D>(sK, p.k + kbase, kstride, kvalid);
-        if (ROPE) stage_rows<D>(sKl, p.kl + kbase, kstride, kvalid);
-        stage_rows<D>(sV, p.v + kbase, kstride, kvalid);
-        __syncthreads();
+        const long k0 = static_cast<long>(t) * kBmTile;
+        const int buf = t & 1;
         float s[8][4], dp[8][4];
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
-        mma_rows_t<D>(s, uQ, warp * 16, uK, lane);
+        mma_rows_t<D>(s, uQ, warp * 16, uK(buf), lane);
         if (ROPE) {
-            mma_rows_t<D>(s, uQ, warp * 16, uKl, lane);
-            mma_rows_t<D>(s, uQl, warp * 16, uK, lane);
+            mma_rows_t<D>(s, uQ, warp * 16, uKl(buf), lane);
+            mma_rows_t<D>(s, uQl, warp * 16, uK(buf), lane);
         }
-        mma_rows_t<D>(dp, uG, warp * 16, uV, lane);
+        mma_rows_t<D>(dp, uG, warp * 16, uV(buf), lane);
         // dS * scale in place of s
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
@@ -222,8 +245,10 @@ __global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p
         }
         uint32_t pa[4][4];
         to_afrag(s, pa);
-        mma_p_tile<D>(dq, pa, uK, lane);
+        mma_p_tile<D>(dq, pa, uK(buf), lane);
+        __syncthreads();   // buffer buf is refilled by the step after next
     }
+    cp_async_wait<0>();
     const bool live_a = ra < p.Sq, live_b = rb < p.Sq;
     const long oa = ((static_cast<long>(b) * p.Sq + ra) * p.Hq + h) * D;
     const long ob = ((static_cast<long>(b) * p.Sq + rb) * p.Hq + h) * D;
@@ -237,14 +262,12 @@ template <int D, bool ROPE>
 __global__ void __launch_bounds__(kBmThreads) bwd_dkdv_mma_kernel(const BmParams p) {
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
-    uint8_t* sK = bm_smem;
-    uint8_t* sKl = sK + C::TILE;
-    uint8_t* sV = sKl + (ROPE ? C::TILE : 0);
-    uint8_t* sQ = sV + C::TILE;
-    uint8_t* sQl = sQ + C::TILE;
-    uint8_t* sG = sQl + (ROPE ? C::TILE : 0);
-    float* sL = reinterpret_cast<float*>(sG + C::TILE);   // [64] lse * log2(e)
-    float* sD = sL + kBmTile;                             // [64] D
+    const uint32_t base = smem_u32(bm_smem);
+    const uint32_t uK = base, uKl = base + C::TILE, uV = base + (C::NT - 1) * C::TILE;
+    auto uQ = [&](int buf) { return base + C::NT * C::TILE + buf * C::STEP; };
+    auto uQl = [&](int buf) { return uQ(buf) + C::TILE; };
+    auto uG = [&](int buf) { return uQ(buf) + (C::NT - 1) * C::TILE; };
+    auto sLrow = [&](int buf) { return reinterpret_cast<float*>(bm_smem + C::NT * C::TILE + buf * C::STEP + C::NT * C::TILE); };
     const int kvh = blockIdx.y, b = blockIdx.z;
     const int G = p.Hq / p.Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -253,71 +276,87 @@ __global__ void __launch_bounds__(kBmThreads) bwd_dkdv_mma_kernel(const BmParams
     const long qstride = static_cast<long>(p.Hq) * D, kstride = static_cast<long>(p.Hkv) * D;
     const long kbase = ((static_cast<long>(b) * p.Skv + j0) * p.Hkv + kvh) * D;
     const int kvalid = min(kBmRows, p.Skv - j0);
-    stage_rows<D>(sK, p.k + kbase, kstride, kvalid);
-    if (ROPE) stage_rows<D>(sKl, p.kl + kbase, kstride, kvalid);
-    stage_rows<D>(sV, p.v + kbase, kstride, kvalid);
-    const int ja = j0 + warp * 16 + g, jb = ja + 8;    // this thread's two keys
     const long off_c = static_cast<long>(p.Skv) - p.Sq;
+    long i_lo = p.causal ? static_cast<long>(j0) - off_c : 0;
+    i_lo = i_lo < 0 ? 0 : i_lo;
+    const int t_start = static_cast<int>(i_lo / kBmTile);
+    const int t_per_head = (p.Sq + kBmTile - 1) / kBmTile - t_start;   // query tiles per q head
+    const int nsteps = t_per_head > 0 ? t_per_head * G : 0;
+    // step -> (group head, query tile); lse and D rows land after the step's tiles
+    auto issue_step = [&](int t) {
+        const int hg = t / t_per_head;
+        const long i0 = static_cast<long>(t_start + t % t_per_head) * kBmTile;
+        const int h = kvh * G + hg;
+        const long qbase = ((static_cast<long>(b) * p.Sq + i0) * p.Hq + h) * D;
+        const int qvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Sq - i0));
+        stage_rows_async<D>(uQ(t & 1), p.q + qbase, qstride, qvalid);
+        if (ROPE) stage_rows_async<D>(uQl(t & 1), p.ql + qbase, qstride, qvalid);
+        stage_rows_async<D>(uG(t & 1), p.dout + qbase, qstride, qvalid);
+        const uint32_t dl = smem_u32(sLrow(t & 1));
+        const long srow0 = (static_cast<long>(b) * p.Hq + h) * p.Sq + i0;
+        for (int w = threadIdx.x; w < 2 * kBmTile; w += kBmThreads) {
+            const int r = w % kBmTile;
+            const bool ok = r < qvalid;
+            const float* src = (w < kBmTile ? p.lse : p.Dvec) + srow0 + (ok ? r : 0);
+            cp_async4(dl + w * 4, src, ok);
+        }
+    };
+    stage_rows_async<D>(uK, p.k + kbase, kstride, kvalid);
+    if (ROPE) stage_rows_async<D>(uKl, p.kl + kbase, kstride, kvalid);
+    stage_rows_async<D>(uV, p.v + kbase, kstride, kvalid);
+    if (nsteps > 0) issue_step(0);
+    cp_async_commit();
+    const int ja = j0 + warp * 16 + g, jb = ja + 8;    // this thread's two keys
     float dk[D / 8][4], dv[D / 8][4];
 #pragma unroll
     for (int nd = 0; nd < D / 8; ++nd)
 #pragma unroll
         for (int e = 0; e < 4; ++e) dk[nd][e] = dv[nd][e] = 0.f;
-    long i_lo = p.causal ? static_cast<long>(j0) - off_c : 0;
-    i_lo = i_lo < 0 ? 0 : i_lo;
-    const long i_start = (i_lo / kBmTile) * kBmTile;
     const float sl2 = p.scale * kLog2e;
-    const uint32_t uQ = smem_u32(sQ), uQl = smem_u32(sQl), uG = smem_u32(sG);
-    const uint32_t uK = smem_u32(sK), uKl = smem_u32(sKl), uV = smem_u32(sV);
-    for (int hg = 0; hg < G; ++hg) {
-        const int h = kvh * G + hg;
-        for (long i0 = i_start; i0 < p.Sq; i0 += kBmTile) {
-            __syncthreads();
-            const long qbase = ((static_cast<long>(b) * p.Sq + i0) * p.Hq + h) * D;
-            const int qvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Sq - i0));
-            stage_rows<D>(sQ, p.q + qbase, qstride, qvalid);
-            if (ROPE) stage_rows<D>(sQl, p.ql + qbase, qstride, qvalid);
-            stage_rows<D>(sG, p.dout + qbase, qstride, qvalid);
-            for (int w = threadIdx.x; w < kBmTile; w += kBmThreads) {
-                const long srow = (static_cast<long>(b) * p.Hq + h) * p.Sq + i0 + w;
-                const bool in = w < qvalid;
-                sL[w] = in ? p.lse[srow] * kLog2e : -INFINITY;
-                sD[w] = in ? p.Dvec[srow] : 0.f;
-            }
-            __syncthreads();
-            float s[8][4], dp[8][4];
+    for (int t = 0; t < nsteps; ++t) {
+        if (t + 1 < nsteps) issue_step(t + 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+        const int buf = t & 1;
+        const long i0 = static_cast<long>(t_start + t % t_per_head) * kBmTile;
+        const int qvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Sq - i0));
+        const float* sL = sLrow(buf);
+        const float* sD = sL + kBmTile;
+        float s[8][4], dp[8][4];
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
-            mma_rows_t<D>(s, uK, warp * 16, uQ, lane);        // S^T = K Q^T
-            if (ROPE) {
-                mma_rows_t<D>(s, uK, warp * 16, uQl, lane);
-                mma_rows_t<D>(s, uKl, warp * 16, uQ, lane);
-            }
-            mma_rows_t<D>(dp, uV, warp * 16, uG, lane);       // dP^T = V dO^T
-            // s <- P^T, dp <- dS^T * scale
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int qi = nt * 8 + 2 * t4 + (e & 1);   // query row within the tile
-                    const long key = (e < 2) ? ja : jb;
-                    const float l2 = sL[qi];
-                    const bool vis = key < p.Skv && l2 != -INFINITY &&
-                                     (!p.causal || key <= i0 + qi + off_c);
-                    const float pr = vis ? fast_exp2(s[nt][e] * sl2 - l2) : 0.f;
-                    dp[nt][e] = pr * (dp[nt][e] - sD[qi]) * p.scale;
-                    s[nt][e] = pr;
-                }
-            }
-            uint32_t pa[4][4];
-            to_afrag(s, pa);
-            mma_p_tile<D>(dv, pa, uG, lane);                   // dV += P^T dO
-            to_afrag(dp, pa);
-            mma_p_tile<D>(dk, pa, uQ, lane);                   // dK += dS^T Q
+            for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
+        mma_rows_t<D>(s, uK, warp * 16, uQ(buf), lane);        // S^T = K Q^T
+        if (ROPE) {
+            mma_rows_t<D>(s, uK, warp * 16, uQl(buf), lane);
+            mma_rows_t<D>(s, uKl, warp * 16, uQ(buf), lane);
         }
+        mma_rows_t<D>(dp, uV, warp * 16, uG(buf), lane);       // dP^T = V dO^T
+        // s <- P^T, dp <- dS^T * scale
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int qi = nt * 8 + 2 * t4 + (e & 1);   // query row within the tile
+                const long key = (e < 2) ? ja : jb;
+                const float lse = sL[qi];
+                const bool vis = qi < qvalid && key < p.Skv && lse != -INFINITY &&
+                                 (!p.causal || key <= i0 + qi + off_c);
+                const float pr = vis ? fast_exp2(s[nt][e] * sl2 - lse * kLog2e) : 0.f;
+                dp[nt][e] = pr * (dp[nt][e] - sD[qi]) * p.scale;
+                s[nt][e] = pr;
+            }
+        }
+        uint32_t pa[4][4];
+        to_afrag(s, pa);
+        mma_p_tile<D>(dv, pa, uG(buf), lane);                   // dV += P^T dO
+        to_afrag(dp, pa);
+        mma_p_tile<D>(dk, pa, uQ(buf), lane);                   // dK += dS^T Q
+        __syncthreads();   // buffer buf is refilled by the step after next
     }
+    cp_async_wait<0>();
     const bool live_a = ja < p.Skv, live_b = jb < p.Skv;
     const long oa = ((static_cast<long>(b) * p.Skv + ja) * p.Hkv + kvh) * D;
     const long ob = ((static_cast<long>(b) * p.Skv + jb) * p.Hkv + kvh) * D;
