@@ -395,7 +395,7 @@ attn_status launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const
                            const float2* tab, int q_pos0, uint8_t* ws, const BmWorkspace& w, cudaStream_t st) {
     float* Dvec = reinterpret_cast<float*>(ws + w.d_off);
     const long nq = static_cast<long>(B) * Sq * Hq;
-    bwd_rowdot_kernel<<<static_cast<unsigned>((nq * 32 + 255) / 256), 256, 0, st>>>(o, dout, Dvec, nq, Sq, Hq, D);
+    bwd_rowdot_kernel<D><<<static_cast<unsigned>((nq * (D / 8) + 255) / 256), 256, 0, st>>>(o, dout, Dvec, nq, Sq, Hq);
     attn_status s = launch_status("bwd_rowdot_kernel");
     if (s != ATTN_OK) return s;
     BmParams p{};

@@ -386,26 +386,34 @@ __global__ void bwd_rope_split_kernel(const uint32_t* __restrict__ x, uint32_t* 
     }
 }
 
-// D_i = dO . O per row for the bf16 path (one warp per row).
+// D_i = dO . O per row for the bf16 path: D/8 lanes per row, one 16-byte load of o and of dO per
+// lane, the row's lanes reduced with shuffles.
+template <int D>
 __global__ void bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                                  float* __restrict__ Dvec, long nrows, int Sq, int Hq, int D) {
-    const int lane = threadIdx.x & 31;
-    const long row = (static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    if (row >= nrows) return;
-    const int h = static_cast<int>(row % Hq);
-    const int i = static_cast<int>((row / Hq) % Sq);
-    const long b = row / (static_cast<long>(Hq) * Sq);
-    const uint32_t* op = reinterpret_cast<const uint32_t*>(o + row * D);
-    const uint32_t* gp = reinterpret_cast<const uint32_t*>(dout + row * D);
+                                  float* __restrict__ Dvec, long nrows, int Sq, int Hq) {
+    constexpr int LPR = D / 8;                   // lanes per row (8 or 16)
+    const long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const long row = t / LPR;
+    const int part = static_cast<int>(t % LPR);
     float acc = 0.f;
-    for (int w = lane; w < D / 2; w += 32) {
-        const uint32_t a = op[w], c = gp[w];
-        acc = fmaf(bf16lo_to_f32(a), bf16lo_to_f32(c), acc);
-        acc = fmaf(bf16hi_to_f32(a), bf16hi_to_f32(c), acc);
+    if (row < nrows) {
+        const uint4 a = *reinterpret_cast<const uint4*>(o + row * D + part * 8);
+        const uint4 c = *reinterpret_cast<const uint4*>(dout + row * D + part * 8);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc = fmaf(bf16lo_to_f32(aw[e]), bf16lo_to_f32(cw[e]), acc);
+            acc = fmaf(bf16hi_to_f32(aw[e]), bf16hi_to_f32(cw[e]), acc);
+        }
     }
 #pragma unroll
-    for (int w = 16; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
-    if (lane == 0) Dvec[(b * Hq + h) * Sq + i] = acc;
+    for (int w = LPR / 2; w >= 1; w >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+    if (row < nrows && part == 0) {
+        const int h = static_cast<int>(row % Hq);
+        const int i = static_cast<int>((row / Hq) % Sq);
+        const long b = row / (static_cast<long>(Hq) * Sq);
+        Dvec[(b * Hq + h) * Sq + i] = acc;
+    }
 }
 
 }  // namespace attn
