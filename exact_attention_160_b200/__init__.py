@@ -57,7 +57,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.attn_fwd.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, P]
     lib.attn_fwd_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
-    lib.attn_fwd_ex_workspace_size.argtypes = [I, I, I, I, I, I, F, I]
+    lib.attn_fwd_ex_workspace_size.argtypes = [I, I, I, I, I, I, I, F, I]
     lib.attn_fwd_ex_workspace_size.restype = Z
     lib.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, Z, I, P]
     lib.attn_decode_workspace_size.argtypes = [I, I, I, I]
@@ -127,11 +127,13 @@ def attn_fwd(q, k, v, scale: float, causal: bool, o=None, lse=None, want_lse: bo
                        stream=stream)
 
 
-def fwd_workspace_bytes(q, k, rope_base: float, q_pos0: int) -> int:
+def fwd_workspace_bytes(q, k, rope_base: float, q_pos0: int, out_dtype=None) -> int:
     lib = load_library()
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
-    return int(lib.attn_fwd_ex_workspace_size(B, Hkv, Sq, Skv, D, _dtype_code(q), float(rope_base), int(q_pos0)))
+    code = _dtype_code(q) if out_dtype is None or q.dtype != torch.bfloat16 else (
+        ATTN_BF16_OUT_F32 if out_dtype == torch.float32 else ATTN_BF16)
+    return int(lib.attn_fwd_ex_workspace_size(B, Hq, Hkv, Sq, Skv, D, code, float(rope_base), int(q_pos0)))
 
 
 def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: int = 0, o=None, lse=None,
@@ -146,12 +148,12 @@ def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: i
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     ws_bytes = 0
-    if rope_base > 0:
-        need = fwd_workspace_bytes(q, k, rope_base, q_pos0)
+    need = fwd_workspace_bytes(q, k, rope_base, q_pos0, o.dtype)
+    if need > 0 or workspace is not None:
         if workspace is None:
-            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
         ws_bytes = workspace.numel() * workspace.element_size()
-    if rope_base > 0:
+    if rope_base > 0 or need > 0:
         st = lib.attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
                              float(scale), int(bool(causal)), _dtype_code(q, o), float(rope_base), int(q_pos0),
                              _ptr(workspace), ws_bytes, _stream(stream))
@@ -198,10 +200,11 @@ def rope_apply(x, pos, base: float, stream=None):
     return x
 
 
-def bwd_workspace_bytes(q, k, rope_base: float = 0.0, q_pos0: int = 0) -> int:
+def bwd_workspace_bytes(q, k, rope_base: float = 0.0, q_pos0: int = 0, grad_dtype=None) -> int:
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
-    code = ATTN_FP32 if q.dtype == torch.float32 else ATTN_BF16
+    code = ATTN_FP32 if q.dtype == torch.float32 else (
+        ATTN_BF16_OUT_F32 if grad_dtype == torch.float32 else ATTN_BF16)
     return int(load_library().attn_bwd_workspace_size(B, Hq, Hkv, Sq, Skv, D, code, float(rope_base), int(q_pos0)))
 
 
@@ -222,7 +225,7 @@ def attn_bwd(q, k, v, o, lse, dout, scale: float, causal: bool, rope_base: float
     dk = torch.empty(k.shape, dtype=gd, device=q.device)
     dv = torch.empty(v.shape, dtype=gd, device=q.device)
     if workspace is None:
-        workspace = torch.empty(max(bwd_workspace_bytes(q, k, rope_base, q_pos0), 1), dtype=torch.uint8,
+        workspace = torch.empty(max(bwd_workspace_bytes(q, k, rope_base, q_pos0, gd), 1), dtype=torch.uint8,
                                 device=q.device)
     st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, Hq,
                       Hkv, Sq, Skv, D, float(scale), int(bool(causal)), code, float(rope_base), int(q_pos0),

@@ -100,6 +100,28 @@ attn_status check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float s
     return ATTN_OK;
 }
 
+// Head dims other than 64 and 128 run at Dp = 64 (D < 64) or 128 (64 < D < 128) with q, k, v
+// (and dout) zero-padded in the workspace: padded dims add nothing to q.k, the caller's scale is
+// kept, RoPE keeps the frequencies of D (padding pairs rotate by the identity), and the outputs
+// are copied back without the padding.  D must be even (whole 32-bit words per bf16 row).
+bool native_dim(int D) { return D == 64 || D == 128; }
+int padded_dim(int D) { return D <= 64 ? 64 : 128; }
+bool paddable_dim(int D) { return D > 0 && D < 128 && !native_dim(D) && D % 2 == 0; }
+
+attn_status launch_pad(const void* src, void* dst, long rows, int src_bytes, int dst_bytes, bool unpad,
+                       cudaStream_t st) {
+    const int sw = src_bytes / 4, dw = dst_bytes / 4;
+    const long n = rows * dw;
+    const unsigned grid = static_cast<unsigned>((n + 255) / 256 < 148L * 32 ? (n + 255) / 256 : 148L * 32);
+    if (unpad)
+        unpad_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(src), static_cast<uint32_t*>(dst), rows,
+                                                sw, dw);
+    else
+        pad_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const uint32_t*>(src), static_cast<uint32_t*>(dst), rows, sw,
+                                              dw);
+    return launch_status(unpad ? "unpad_rows_kernel" : "pad_rows_kernel");
+}
+
 // Layout of the attn_fwd_ex workspace: rope table, then (bf16) rotated K as hi and lo halves.
 struct ExWorkspace {
     size_t tab_off, khi_off, klo_off, total;
@@ -187,7 +209,7 @@ attn_status launch_f32(const void* q, const void* k, const void* v, void* o, flo
 
 attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                      int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
-                     void* workspace, size_t workspace_bytes, cudaStream_t st) {
+                     void* workspace, size_t workspace_bytes, cudaStream_t st, int rope_dim) {
     attn_status s = check_common(B, Hq, Hkv, Sq, Skv, D, scale, causal);
     if (s != ATTN_OK) return s;
     if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
@@ -208,7 +230,7 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
         float2* t = reinterpret_cast<float2*>(ws + w.tab_off);
         const long n = static_cast<long>(w.positions) * (D / 2);
         rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, st>>>(
-            t, w.positions, D, static_cast<double>(rope_base));
+            t, w.positions, D, static_cast<double>(rope_base), rope_dim);
         if ((s = launch_status("rope_table_kernel")) != ATTN_OK) return s;
         tab = t;
     }
@@ -281,6 +303,50 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
                                              o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Hq, Smax, num_splits);
     if (e != cudaSuccess) return cuda_failure("decode_combine_kernel launch", cudaGetErrorString(e));
     return launch_status("decode_combine_kernel");
+}
+
+// Workspace of a padded forward: q, k, v and o at Dp, then the inner call's own workspace.
+struct PadFwd {
+    size_t q_off, k_off, v_off, o_off, inner_off, total;
+    int Dp;
+};
+
+PadFwd pad_fwd_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
+                         int q_pos0) {
+    PadFwd w{};
+    w.Dp = padded_dim(D);
+    const size_t es_in = dtype == ATTN_FP32 ? 4 : 2, es_out = dtype == ATTN_BF16 ? 2 : 4;
+    const size_t qe = static_cast<size_t>(B) * Sq * Hq * w.Dp, ke = static_cast<size_t>(B) * Skv * Hkv * w.Dp;
+    w.q_off = 0;
+    w.k_off = round_up(qe * es_in, 256);
+    w.v_off = round_up(w.k_off + ke * es_in, 256);
+    w.o_off = round_up(w.v_off + ke * es_in, 256);
+    w.inner_off = round_up(w.o_off + qe * es_out, 256);
+    w.total = w.inner_off + (rope_base > 0.f ? ex_workspace(B, Hkv, Sq, Skv, w.Dp, dtype, q_pos0).total : 0);
+    return w;
+}
+
+attn_status fwd_padded(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                       int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
+                       void* workspace, size_t workspace_bytes, cudaStream_t st) {
+    attn_status s = check_common(B, Hq, Hkv, Sq, Skv, 64, scale, causal);   // everything but D
+    if (s != ATTN_OK) return s;
+    if (!paddable_dim(D)) return ATTN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP32 && dtype != ATTN_BF16_OUT_F32) return ATTN_ERR_INVALID_ARG;
+    const PadFwd w = pad_fwd_workspace(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base, q_pos0);
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int es_in = dtype == ATTN_FP32 ? 4 : 2, es_out = dtype == ATTN_BF16 ? 2 : 4;
+    const long qrows = static_cast<long>(B) * Sq * Hq, krows = static_cast<long>(B) * Skv * Hkv;
+    if ((s = launch_pad(q, ws + w.q_off, qrows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    if ((s = launch_pad(k, ws + w.k_off, krows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    if ((s = launch_pad(v, ws + w.v_off, krows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    s = fwd_impl(ws + w.q_off, ws + w.k_off, ws + w.v_off, ws + w.o_off, lse, B, Hq, Hkv, Sq, Skv, w.Dp, scale,
+                 causal, dtype, rope_base, q_pos0, ws + w.inner_off, w.total - w.inner_off, st, D);
+    if (s != ATTN_OK) return s;
+    return launch_pad(ws + w.o_off, o, qrows, w.Dp * es_out, D * es_out, true, st);
 }
 
 // Layout of the attn_bwd workspace: rope table (with RoPE), fp32 copies of rotated q, dO,
@@ -455,17 +521,93 @@ attn_status launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const
 
 }  // namespace
 
+namespace {
+
+size_t bwd_inner_bytes(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base, int q_pos0) {
+    if (dtype == ATTN_FP32) return bwd_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
+    return bm_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
+}
+
+// Workspace of a padded backward: q, k, v, o, dout and dq, dk, dv at Dp, then the inner call's.
+struct PadBwd {
+    size_t q_off, k_off, v_off, o_off, g_off, dq_off, dk_off, dv_off, inner_off, total;
+    int Dp;
+};
+
+PadBwd pad_bwd_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
+                         int q_pos0) {
+    PadBwd w{};
+    w.Dp = padded_dim(D);
+    const size_t es_in = dtype == ATTN_FP32 ? 4 : 2, es_g = dtype == ATTN_BF16 ? 2 : 4;
+    const size_t qe = static_cast<size_t>(B) * Sq * Hq * w.Dp, ke = static_cast<size_t>(B) * Skv * Hkv * w.Dp;
+    w.q_off = 0;
+    w.k_off = round_up(qe * es_in, 256);
+    w.v_off = round_up(w.k_off + ke * es_in, 256);
+    w.o_off = round_up(w.v_off + ke * es_in, 256);
+    w.g_off = round_up(w.o_off + qe * es_in, 256);
+    w.dq_off = round_up(w.g_off + qe * es_in, 256);
+    w.dk_off = round_up(w.dq_off + qe * es_g, 256);
+    w.dv_off = round_up(w.dk_off + ke * es_g, 256);
+    w.inner_off = round_up(w.dv_off + ke * es_g, 256);
+    w.total = w.inner_off + bwd_inner_bytes(B, Hq, Hkv, Sq, Skv, w.Dp, dtype, rope_base, q_pos0);
+    return w;
+}
+
+attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                     int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
+                     size_t workspace_bytes, attn_stream_t stream, int rope_dim);
+
+}  // namespace
+
 size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
                                int q_pos0) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0 || q_pos0 < 0) return 0;
-    if (dtype == ATTN_FP32) return bwd_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
-    return bm_workspace(B, Hq, Hkv, Sq, Skv, D, rope_base > 0.f, q_pos0).total;
+    if (!native_dim(D)) return paddable_dim(D) ? pad_bwd_workspace(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base, q_pos0).total : 0;
+    return bwd_inner_bytes(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base, q_pos0);
 }
 
 attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
                      int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
                      size_t workspace_bytes, attn_stream_t stream) {
+    if (D <= 0 || native_dim(D))
+        return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base,
+                        q_pos0, workspace, workspace_bytes, stream, D);
+    attn_status s = check_common(B, Hq, Hkv, Sq, Skv, 64, scale, causal);   // everything but D
+    if (s != ATTN_OK) return s;
+    if (!paddable_dim(D)) return ATTN_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(dq) ||
+        !aligned16(dk) || !aligned16(dv))
+        return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_FP32 && dtype != ATTN_BF16_OUT_F32) return ATTN_ERR_INVALID_ARG;
+    const PadBwd w = pad_bwd_workspace(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base, q_pos0);
+    if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int es_in = dtype == ATTN_FP32 ? 4 : 2, es_g = dtype == ATTN_BF16 ? 2 : 4;
+    const long qrows = static_cast<long>(B) * Sq * Hq, krows = static_cast<long>(B) * Skv * Hkv;
+    if ((s = launch_pad(q, ws + w.q_off, qrows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    if ((s = launch_pad(k, ws + w.k_off, krows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    if ((s = launch_pad(v, ws + w.v_off, krows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    if ((s = launch_pad(o, ws + w.o_off, qrows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    if ((s = launch_pad(dout, ws + w.g_off, qrows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
+    s = bwd_impl(ws + w.q_off, ws + w.k_off, ws + w.v_off, ws + w.o_off, lse, ws + w.g_off, ws + w.dq_off,
+                 ws + w.dk_off, ws + w.dv_off, B, Hq, Hkv, Sq, Skv, w.Dp, scale, causal, dtype, rope_base, q_pos0,
+                 ws + w.inner_off, w.total - w.inner_off, stream, D);
+    if (s != ATTN_OK) return s;
+    if ((s = launch_pad(ws + w.dq_off, dq, qrows, w.Dp * es_g, D * es_g, true, st)) != ATTN_OK) return s;
+    if ((s = launch_pad(ws + w.dk_off, dk, krows, w.Dp * es_g, D * es_g, true, st)) != ATTN_OK) return s;
+    return launch_pad(ws + w.dv_off, dv, krows, w.Dp * es_g, D * es_g, true, st);
+}
+
+namespace {
+
+attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                     int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
+                     size_t workspace_bytes, attn_stream_t stream, int rope_dim) {
     attn_status s = check_common(B, Hq, Hkv, Sq, Skv, D, scale, causal);
     if (s != ATTN_OK) return s;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
@@ -488,7 +630,7 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
         float2* t = reinterpret_cast<float2*>(ws + w.tab_off);   // offset 0 in both layouts
         const long n = static_cast<long>(w.positions) * (D / 2);
         rope_table_kernel<<<static_cast<unsigned>((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096), 256, 0, st>>>(
-            t, w.positions, D, static_cast<double>(rope_base));
+            t, w.positions, D, static_cast<double>(rope_base), rope_dim);
         if ((s = launch_status("rope_table_kernel")) != ATTN_OK) return s;
         tab = t;
     }
@@ -515,6 +657,8 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                 : launch_bwd_mma<128, false>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
                                              causal, tab, q_pos0, ws, wm, st);
 }
+
+}  // namespace
 
 // ------------------------------------------------------------------------------------------
 // Built-in decode scratch for callers that cannot allocate device memory.
@@ -561,20 +705,30 @@ extern "C" {
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int Sq,
                      int Skv, int D, float scale, int causal, attn_dtype dtype, attn_stream_t stream) {
+    if (D > 0 && !native_dim(D)) {
+        // other head dims pad through a workspace: attn_fwd_ex
+        snprintf(g_last_error, sizeof(g_last_error), "head dim %d needs attn_fwd_ex with a workspace", D);
+        return ATTN_ERR_UNSUPPORTED;
+    }
     return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, 0.f, 0, nullptr, 0,
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), D);
 }
 
 attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                         int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
                         void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+    if (D > 0 && !native_dim(D))
+        return fwd_padded(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base, q_pos0, workspace,
+                          workspace_bytes, static_cast<cudaStream_t>(stream));
     return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base, q_pos0, workspace,
-                    workspace_bytes, static_cast<cudaStream_t>(stream));
+                    workspace_bytes, static_cast<cudaStream_t>(stream), D);
 }
 
-size_t attn_fwd_ex_workspace_size(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
+size_t attn_fwd_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,
                                   int q_pos0) {
-    if (!(rope_base > 0.f) || B <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0 || q_pos0 < 0) return 0;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0 || q_pos0 < 0) return 0;
+    if (!native_dim(D)) return paddable_dim(D) ? pad_fwd_workspace(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base, q_pos0).total : 0;
+    if (!(rope_base > 0.f)) return 0;
     return ex_workspace(B, Hkv, Sq, Skv, D, dtype, q_pos0).total;
 }
 

@@ -16,17 +16,48 @@ __device__ __forceinline__ double rope_theta(double pos, int pair, int D, double
     return pos / pow(base, 2.0 * static_cast<double>(pair) / static_cast<double>(D));
 }
 
-// tab[p * (D/2) + i] = (cos, sin) of theta_i at position p, for p in [0, P).
-__global__ void rope_table_kernel(float2* __restrict__ tab, int P, int D, double base) {
+// tab[p * (D/2) + i] = (cos, sin) of theta_i at position p, for p in [0, P).  Dfreq is the head
+// dim whose frequencies are used (the true dim when the vectors are zero-padded to D); pairs at
+// or past Dfreq/2 are padding and get the identity (1, 0).
+__global__ void rope_table_kernel(float2* __restrict__ tab, int P, int D, double base, int Dfreq) {
     const int half = D / 2;
     const long n = static_cast<long>(P) * half;
     for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < n;
          idx += static_cast<long>(gridDim.x) * blockDim.x) {
         const int p = static_cast<int>(idx / half);
         const int i = static_cast<int>(idx % half);
+        if (2 * i >= Dfreq) {
+            tab[idx] = make_float2(1.f, 0.f);
+            continue;
+        }
         double s, c;
-        sincos(rope_theta(static_cast<double>(p), i, D, base), &s, &c);
+        sincos(rope_theta(static_cast<double>(p), i, Dfreq, base), &s, &c);
         tab[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
+    }
+}
+
+// Zero-pad rows: dst rows of dst_words 32-bit words take the src_words of each src row followed
+// by zeros (pads a head dim; src_words < dst_words).
+__global__ void pad_rows_kernel(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst, long rows,
+                                int src_words, int dst_words) {
+    const long n = rows * dst_words;
+    for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<long>(gridDim.x) * blockDim.x) {
+        const long r = idx / dst_words;
+        const int c = static_cast<int>(idx % dst_words);
+        dst[idx] = c < src_words ? src[r * src_words + c] : 0u;
+    }
+}
+
+// Drop the padding: dst rows of dst_words words take the first dst_words of each src row.
+__global__ void unpad_rows_kernel(const uint32_t* __restrict__ src, uint32_t* __restrict__ dst, long rows,
+                                  int src_words, int dst_words) {
+    const long n = rows * dst_words;
+    for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < n;
+         idx += static_cast<long>(gridDim.x) * blockDim.x) {
+        const long r = idx / dst_words;
+        const int c = static_cast<int>(idx % dst_words);
+        dst[idx] = src[r * src_words + c];
     }
 }
 

@@ -37,7 +37,15 @@
  *     unmasked key gets o_i = 0 and lse_i = -inf.
  *   - GQA: q head h reads kv head h / (Hq / Hkv); Hq must be a multiple of Hkv (Hkv == Hq is
  *     multi-head, Hkv == 1 is multi-query attention).
- *   - Supported head dims: D in {64, 128}.  Other values return ATTN_ERR_UNSUPPORTED.
+ *   - Head dims: D in {64, 128} run natively.  attn_fwd_ex and attn_bwd also take any other
+ *     even D < 128: q, k, v (and dout) are zero-padded to 64 or 128 in the
+ *     workspace (zero dims add nothing to q.k; the scale is the caller's, so no correction is
+ *     needed; RoPE keeps the frequencies of D) and the outputs are copied back without the
+ *     padding.  whisper-apr 0.3.1 src/model/lfm2/gqa.rs (GqaConfig::pad_head_dim_to,
+ *     padded_head_dim) pads a head dim up to a multiple for aligned computation (36 -> 40 for
+ *     Moonshine); here the multiple is the kernels' tile width.  attn_fwd,
+ *     which has no workspace, returns ATTN_ERR_UNSUPPORTED for them, as does attn_decode; odd
+ *     head dims are unsupported.
  */
 #ifndef ATTN_B200_H
 #define ATTN_B200_H
@@ -103,8 +111,9 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
                         attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
                         size_t workspace_bytes, attn_stream_t stream);
 
-/* Bytes of workspace attn_fwd_ex needs for these sizes (0 when rope_base <= 0).            */
-size_t attn_fwd_ex_workspace_size(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtype,
+/* Bytes of workspace attn_fwd_ex needs for these sizes: 0 for D in {64, 128} without RoPE; the
+ * rotated-K halves with RoPE; the padded q, k, v, o (and the inner call's needs) otherwise.   */
+size_t attn_fwd_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype,
                                   float rope_base, int q_pos0);
 
 /*

@@ -59,9 +59,9 @@ def test_fwd_validation(lib):
 
 def test_fwd_ex_validation(lib):
     P = FAKE
-    need = lib.attn_fwd_ex_workspace_size(1, 2, 8, 8, 64, 0, 10000.0, 0)
+    need = lib.attn_fwd_ex_workspace_size(1, 2, 2, 8, 8, 64, 0, 10000.0, 0)
     assert need > 0
-    assert lib.attn_fwd_ex_workspace_size(1, 2, 8, 8, 64, 0, 0.0, 0) == 0
+    assert lib.attn_fwd_ex_workspace_size(1, 2, 2, 8, 8, 64, 0, 0.0, 0) == 0
     # workspace missing / too small
     assert lib.attn_fwd_ex(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0.1, 1, 0, 10000.0, 0, None, 0, None) == 5
     assert lib.attn_fwd_ex(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0.1, 1, 0, 10000.0, 0, P, need - 1, None) == 5
