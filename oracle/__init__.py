@@ -46,8 +46,10 @@ def _bind(path: str):
         lib.oracle_decode_f64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, Dd]
         lib.oracle_decode_split_f64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, Dd, I]
         lib.oracle_attn_bwd_f64.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
+        lib.oracle_attn_fwd_mask_f64.argtypes = [P, P, P, P, I64, I64, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
         for f in (lib.oracle_rope_f64, lib.oracle_attn_fwd_f64, lib.oracle_attn_fwd_tiled_f64,
-                  lib.oracle_decode_f64, lib.oracle_decode_split_f64, lib.oracle_attn_bwd_f64):
+                  lib.oracle_decode_f64, lib.oracle_decode_split_f64, lib.oracle_attn_bwd_f64,
+                  lib.oracle_attn_fwd_mask_f64):
             f.restype = I
     return lib
 
@@ -127,6 +129,29 @@ def attn_fwd(q, k, v, scale: float, causal: bool, rope_base: float = 0.0, q_pos0
     _check(_load().oracle_attn_fwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv,
                                        Sq, Skv, D, float(scale), int(bool(causal)), float(rope_base),
                                        int(q_pos0), rp, n))
+    return o, lse
+
+
+def attn_fwd_masked(q, k, v, mask, scale: float, causal: bool, rope_base: float = 0.0, q_pos0: int = 0):
+    """attn_fwd with an additive mask on the scaled scores.  mask: [Sq, Skv], [B, Sq, Skv] (shared
+    by the heads) or [B, Hq, Sq, Skv].  Returns (o [B,Sq,Hq,D], lse [B,Hq,Sq]) in float64."""
+    q, k, v = _f32(q), _f32(k), _f32(v)
+    m = _f32(mask)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    if m.shape[-2:] != (Sq, Skv):
+        raise OracleError("mask shape")
+    if m.ndim == 2:
+        bs, hs = 0, 0
+    elif m.ndim == 3:
+        bs, hs = Sq * Skv, 0
+    else:
+        bs, hs = Hq * Sq * Skv, Sq * Skv
+    o = np.empty((B, Sq, Hq, D), dtype=np.float64)
+    lse = np.empty((B, Hq, Sq), dtype=np.float64)
+    _check(_load().oracle_attn_fwd_mask_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(m), bs, hs, _ptr(o), _ptr(lse), B, Hq,
+                                            Hkv, Sq, Skv, D, float(scale), int(bool(causal)), float(rope_base),
+                                            int(q_pos0)))
     return o, lse
 
 

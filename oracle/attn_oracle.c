@@ -569,3 +569,82 @@ int oracle_attn_bwd_f64(const float* q, const float* k, const float* v, const fl
     }
     return fail ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* Forward with an additive mask                                                               */
+/* ------------------------------------------------------------------------------------------ */
+
+/* As oracle_attn_fwd_f64 (full rows, no row subset), with an additive mask on the scaled scores
+ * ([P3] compute_block_scores: score = dot * scale, then score += mask[q, k]; [P3]
+ * scaled_dot_product_attention adds the mask before the row softmax):
+ *   s_j = scale * q . k_j + mask[b, h, i, j]     (then the causal mask, if any: -inf)
+ * mask element (b, h, i, j) sits at mask[b * mask_bstride + h * mask_hstride + i * Skv + j]
+ * (a stride of 0 broadcasts).  A row whose scores are all -inf gets o = 0, lse = -inf.        */
+int oracle_attn_fwd_mask_f64(const float* q, const float* k, const float* v, const float* mask,
+                             int64_t mask_bstride, int64_t mask_hstride, double* o, double* lse, int B,
+                             int Hq, int Hkv, int Sq, int Skv, int D, double scale, int causal,
+                             double rope_base, int q_pos0) {
+    int st = check_dims(B, Hq, Hkv, Sq, Skv, D);
+    if (st) return st;
+    if (!mask) return ORACLE_ERR_INVALID_ARG;
+    if (rope_base > 0.0 && D % 2) return ORACLE_ERR_INVALID_ARG;
+    const int g = Hq / Hkv;
+    int fail = 0;
+#pragma omp parallel for schedule(dynamic, 1) collapse(2)
+    for (int b = 0; b < B; ++b) {
+        for (int kvh = 0; kvh < Hkv; ++kvh) {
+            double* Kd = (double*)malloc(sizeof(double) * (size_t)Skv * D);
+            double* Vd = (double*)malloc(sizeof(double) * (size_t)Skv * D);
+            double* s = (double*)malloc(sizeof(double) * (size_t)Skv);
+            double* qd = (double*)malloc(sizeof(double) * (size_t)D);
+            if (!Kd || !Vd || !s || !qd) {
+#pragma omp atomic write
+                fail = 1;
+            } else {
+                gather_head(k, b, kvh, Skv, Hkv, D, rope_base, Kd);
+                gather_head(v, b, kvh, Skv, Hkv, D, 0.0, Vd);
+                for (int hg = 0; hg < g; ++hg) {
+                    const int hq = kvh * g + hg;
+                    for (int i = 0; i < Sq; ++i) {
+                        const long qoff = (((long)b * Sq + i) * Hq + hq) * D;
+                        double* orow = o + qoff;
+                        double* lrow = lse + ((long)b * Hq + hq) * Sq + i;
+                        for (int d = 0; d < D; ++d) qd[d] = (double)q[qoff + d];
+                        if (rope_base > 0.0) rope_vec(qd, (double)q_pos0 + (double)i, D, rope_base);
+                        const float* mrow = mask + (long)b * mask_bstride + (long)hq * mask_hstride + (long)i * Skv;
+                        const int nvis = visible_keys(i, Sq, Skv, causal);
+                        double m = -INFINITY;
+                        for (int j = 0; j < Skv; ++j) {
+                            if (j >= nvis) {
+                                s[j] = -INFINITY;
+                                continue;
+                            }
+                            double dot = 0.0;
+                            for (int d = 0; d < D; ++d) dot += qd[d] * Kd[(long)j * D + d];
+                            s[j] = scale * dot + (double)mrow[j];
+                            if (s[j] > m) m = s[j];
+                        }
+                        for (int d = 0; d < D; ++d) orow[d] = 0.0;
+                        if (m == -INFINITY) {
+                            *lrow = -INFINITY;
+                            continue;
+                        }
+                        double l = 0.0;
+                        for (int j = 0; j < Skv; ++j) l += exp(s[j] - m);
+                        for (int j = 0; j < Skv; ++j) {
+                            const double p = exp(s[j] - m) / l;
+                            if (p == 0.0) continue;
+                            for (int d = 0; d < D; ++d) orow[d] += p * Vd[(long)j * D + d];
+                        }
+                        *lrow = m + log(l);
+                    }
+                }
+            }
+            free(Kd);
+            free(Vd);
+            free(s);
+            free(qd);
+        }
+    }
+    return fail ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}

@@ -605,4 +605,57 @@ def pin_backward_invariants():
     _close(dv, mv.reshape(B, Skv, Hkv, G, D).sum(axis=3), 1e-12, "GQA dv = summed MHA dv")
 
 
+def pin_additive_mask():
+    """An additive mask of zeros changes nothing; -inf above the diagonal is the causal mask; a
+    constant mask c leaves o unchanged and adds c to lse; -inf on one key equals attention
+    without that key; a per-head mask [B, Hq, Sq, Skv] acts head by head; a row masked
+    everywhere gives o = 0, lse = -inf; and a tiny case against the pure-Python brute force."""
+    B, Sq, Skv, Hq, Hkv, D = 2, 6, 7, 4, 2, 8
+    q = normal_f32(95, 0, (B, Sq, Hq, D))
+    k = normal_f32(95, 1, (B, Skv, Hkv, D))
+    v = normal_f32(95, 2, (B, Skv, Hkv, D))
+    o0, l0 = oracle.attn_fwd(q, k, v, 0.4, False)
+    o, l = oracle.attn_fwd_masked(q, k, v, np.zeros((Sq, Skv), np.float32), 0.4, False)
+    _close(o, o0, 1e-15, "zero mask")
+    _close(l, l0, 1e-15, "zero mask lse")
+    tri = np.where(np.arange(Skv)[None, :] > np.arange(Sq)[:, None] + (Skv - Sq), -np.inf, 0.0).astype(np.float32)
+    oc, lc = oracle.attn_fwd(q, k, v, 0.4, True)
+    o, l = oracle.attn_fwd_masked(q, k, v, tri, 0.4, False)
+    _close(o, oc, 1e-14, "triangular -inf mask = causal")
+    _close(l, lc, 1e-14, "triangular -inf mask = causal (lse)")
+    o, l = oracle.attn_fwd_masked(q, k, v, np.full((B, Sq, Skv), 1.75, np.float32), 0.4, False)
+    _close(o, o0, 1e-14, "constant mask leaves o")
+    _close(l, l0 + 1.75, 1e-14, "constant mask shifts lse")
+    mk = np.zeros((Sq, Skv), np.float32)
+    mk[:, 3] = -np.inf
+    keep = [j for j in range(Skv) if j != 3]
+    o, l = oracle.attn_fwd_masked(q, k, v, mk, 0.4, False)
+    ok_, lk = oracle.attn_fwd(q, k[:, keep], v[:, keep], 0.4, False)
+    _close(o, ok_, 1e-14, "-inf on a key removes it")
+    _close(l, lk, 1e-14, "-inf on a key removes it (lse)")
+    mh = normal_f32(95, 3, (B, Hq, Sq, Skv))
+    o, l = oracle.attn_fwd_masked(q, k, v, mh, 0.4, True)
+    for h in range(Hq):
+        oh, lh = oracle.attn_fwd_masked(q[:, :, h:h + 1], k[:, :, h // 2:h // 2 + 1], v[:, :, h // 2:h // 2 + 1],
+                                        mh[:, h], 0.4, True)
+        _close(o[:, :, h], oh[:, :, 0], 1e-14, "per-head mask")
+        _close(l[:, h], lh[:, 0], 1e-14, "per-head mask lse")
+    mrow = np.zeros((Sq, Skv), np.float32)
+    mrow[2, :] = -np.inf
+    o, l = oracle.attn_fwd_masked(q, k, v, mrow, 0.4, False)
+    assert np.all(o[:, 2] == 0.0) and np.all(l[:, :, 2] == -np.inf)
+    # brute force: the mask enters as an additive term on the scaled score
+    q1, k1, v1 = q[:1, :3, :1], k[:1, :4, :1], v[:1, :4, :1]
+    m1 = normal_f32(95, 4, (3, 4))
+    o, l = oracle.attn_fwd_masked(q1, k1, v1, m1, 0.7, False)
+    for i in range(3):
+        s = [0.7 * float(np.dot(q1[0, i, 0].astype(np.float64), k1[0, j, 0].astype(np.float64))) + float(m1[i, j])
+             for j in range(4)]
+        mx = max(s)
+        w = [math.exp(x - mx) for x in s]
+        ref = sum(wj * v1[0, j, 0].astype(np.float64) for j, wj in enumerate(w)) / sum(w)
+        _close(o[0, i, 0], ref, 1e-12, "mask brute force")
+        _close(l[0, 0, i], mx + math.log(sum(w)), 1e-12, "mask brute force lse")
+
+
 ALL_PINS = [obj for name, obj in sorted(globals().items()) if name.startswith("pin_")]

@@ -43,6 +43,10 @@ MUTANTS = [
     ("bwd_dk_rope_not_undone", "if (rope_base > 0.0) rope_vec(dkr, -(double)j, D, rope_base);",
      "if (rope_base > 0.0) rope_vec(dkr, (double)j, D, rope_base);"),
     ("bwd_dq_rope_not_undone", "if (rope_base > 0.0) rope_vec(dqr, -((double)q_pos0 + (double)i), D, rope_base);", ""),
+    ("mask_before_scale", "s[j] = scale * dot + (double)mrow[j];", "s[j] = scale * (dot + (double)mrow[j]);"),
+    ("mask_head_stride_ignored", "(long)hq * mask_hstride", "(long)0 * mask_hstride"),
+    ("mask_all_inf_row_nan", "if (m == -INFINITY) {\n                            *lrow = -INFINITY;",
+     "if (0) {\n                            *lrow = -INFINITY;"),
     ("bwd_dp_from_keys", "for (int d = 0; d < D; ++d) dot += go[d] * Vd[(long)j * D + d];",
      "for (int d = 0; d < D; ++d) dot += go[d] * Kd[(long)j * D + d];"),
 ]
