@@ -32,7 +32,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
            "attn_decode_workspace_size", "attn_decode_noalloc", "rope_apply", "attn_status_string",
            "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status", "attn_kv_append",
-           "attn_bwd", "attn_bwd_workspace_size")
+           "attn_bwd", "attn_bwd_workspace_size", "attn_fwd_masked")
 
 _lib = None
 
@@ -68,6 +68,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_status_string.argtypes = [I]
     lib.attn_status_string.restype = ctypes.c_char_p
     lib.attn_read_device_status.argtypes = [P]
+    I64 = ctypes.c_int64
+    lib.attn_fwd_masked.argtypes = [P, P, P, P, I64, I64, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
+    lib.attn_fwd_masked.restype = I
     lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
     lib.attn_bwd.restype = I
     lib.attn_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I, F, I]
@@ -162,6 +165,41 @@ def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: i
         st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Skv, D,
                           float(scale), int(bool(causal)), _dtype_code(q, o), _stream(stream))
         _check(st, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_masked(q, k, v, mask, scale: float, causal: bool, rope_base: float = 0.0, q_pos0: int = 0, o=None,
+                    lse=None, workspace=None, out_dtype=None, stream=None):
+    """Exact attention with an additive fp32 mask on the scaled scores.  mask: [Sq, Skv] (shared),
+    [B, Sq, Skv] (per batch, shared by the heads) or [B, Hq, Sq, Skv]; rows must be contiguous."""
+    lib = load_library()
+    _need_cuda(q, k, v, o, lse, workspace)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    if mask.dtype != torch.float32 or not mask.is_cuda or mask.shape[-2:] != (Sq, Skv) or mask.stride(-1) != 1 \
+            or mask.stride(-2) != Skv:
+        raise ValueError("mask must be a float32 CUDA tensor [..., Sq, Skv] with contiguous rows")
+    if mask.dim() == 2:
+        bs, hs = 0, 0
+    elif mask.dim() == 3:
+        bs, hs = mask.stride(0) if mask.shape[0] > 1 else 0, 0
+    elif mask.dim() == 4:
+        bs = mask.stride(0) if mask.shape[0] > 1 else 0
+        hs = mask.stride(1) if mask.shape[1] > 1 else 0
+    else:
+        raise ValueError("mask must have 2, 3 or 4 dims")
+    if o is None:
+        o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    need = fwd_workspace_bytes(q, k, rope_base, q_pos0, o.dtype)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    st = lib.attn_fwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(mask), bs, hs, _ptr(o), _ptr(lse), B, Hq, Hkv, Sq, Skv,
+                             D, float(scale), int(bool(causal)), _dtype_code(q, o), float(rope_base), int(q_pos0),
+                             _ptr(workspace), ws_bytes, _stream(stream))
+    _check(st, "attn_fwd_masked")
     return o, lse
 
 

@@ -122,6 +122,12 @@ attn_status launch_pad(const void* src, void* dst, long rows, int src_bytes, int
     return launch_status(unpad ? "unpad_rows_kernel" : "pad_rows_kernel");
 }
 
+// Additive mask on the scaled scores: element (b, h, i, j) at ptr[b*bs + h*hs + i*Skv + j].
+struct MaskArg {
+    const float* ptr = nullptr;
+    long bs = 0, hs = 0;
+};
+
 // Layout of the attn_fwd_ex workspace: rope table, then (bf16) rotated K as hi and lo halves.
 struct ExWorkspace {
     size_t tab_off, khi_off, klo_off, total;
@@ -144,7 +150,7 @@ ExWorkspace ex_workspace(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtyp
 template <int D, bool ROPE>
 attn_status launch_tc(const void* q, const void* k, const void* klo, const void* v, void* o, bool o_f32, float* lse,
                       int B, int Hq, int Hkv, int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0,
-                      cudaStream_t st) {
+                      cudaStream_t st, MaskArg mk) {
     CUtensorMap tq, tk, tkl, tv;
     if (!make_tmap_bshd(&tq, q, B, Sq, Hq, D) || !make_tmap_bshd(&tk, k, B, Skv, Hkv, D) ||
         !make_tmap_bshd(&tv, v, B, Skv, Hkv, D) || !make_tmap_bshd(&tkl, ROPE ? klo : k, B, Skv, Hkv, D))
@@ -163,6 +169,10 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     p.heads_per_item = p.pair_heads ? Hq / 2 : Hq;
     p.q_pos0 = q_pos0;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.mask = mk.ptr;
+    p.mask_bs = mk.bs;
+    p.mask_hs = mk.hs;
+    p.inv_scale = 1.f / scale;
     const long grid = static_cast<long>(p.n_row_tiles) * B * p.heads_per_item;
     if (grid > 2147483647L) return ATTN_ERR_UNSUPPORTED;
     auto kern = prefill_tc_kernel<D, ROPE>;
@@ -190,7 +200,8 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
 
 template <int D>
 attn_status launch_f32(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-                       int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0, cudaStream_t st) {
+                       int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0, cudaStream_t st,
+                       MaskArg mk) {
     const size_t smem = 2 * 64 * D * sizeof(float);
     auto kern = prefill_f32_kernel<D>;
     static bool attr_set = false;
@@ -203,13 +214,13 @@ attn_status launch_f32(const void* q, const void* k, const void* v, void* o, flo
     if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
     kern<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
                                   static_cast<const float*>(v), static_cast<float*>(o), lse, Hq, Hkv, Sq, Skv, scale,
-                                  causal, tab, q_pos0);
+                                  causal, tab, q_pos0, mk.ptr, mk.bs, mk.hs);
     return launch_status("prefill_f32_kernel");
 }
 
 attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                      int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
-                     void* workspace, size_t workspace_bytes, cudaStream_t st, int rope_dim) {
+                     void* workspace, size_t workspace_bytes, cudaStream_t st, int rope_dim, MaskArg mk = MaskArg{}) {
     attn_status s = check_common(B, Hq, Hkv, Sq, Skv, D, scale, causal);
     if (s != ATTN_OK) return s;
     if (!q || !k || !v || !o) return ATTN_ERR_INVALID_ARG;
@@ -236,14 +247,14 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
     }
 
     if (dtype == ATTN_FP32) {
-        return D == 64 ? launch_f32<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st)
-                       : launch_f32<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st);
+        return D == 64 ? launch_f32<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st, mk)
+                       : launch_f32<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st, mk);
     }
     if (!rope) {
         return D == 64 ? launch_tc<64, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
-                                              nullptr, 0, st)
+                                              nullptr, 0, st, mk)
                        : launch_tc<128, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
-                                               nullptr, 0, st);
+                                               nullptr, 0, st, mk);
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* khi = reinterpret_cast<uint32_t*>(ws + w.khi_off);
@@ -253,9 +264,9 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
                            0, st>>>(static_cast<const uint32_t*>(k), khi, klo, tab, npairs, Skv, Hkv, D);
     if ((s = launch_status("rope_split_kv_kernel")) != ATTN_OK) return s;
     return D == 64 ? launch_tc<64, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
-                                         q_pos0, st)
+                                         q_pos0, st, mk)
                    : launch_tc<128, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
-                                          q_pos0, st);
+                                          q_pos0, st, mk);
 }
 
 template <int D>
@@ -328,7 +339,7 @@ PadFwd pad_fwd_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dt
 
 attn_status fwd_padded(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
                        int Sq, int Skv, int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
-                       void* workspace, size_t workspace_bytes, cudaStream_t st) {
+                       void* workspace, size_t workspace_bytes, cudaStream_t st, MaskArg mk = MaskArg{}) {
     attn_status s = check_common(B, Hq, Hkv, Sq, Skv, 64, scale, causal);   // everything but D
     if (s != ATTN_OK) return s;
     if (!paddable_dim(D)) return ATTN_ERR_UNSUPPORTED;
@@ -344,7 +355,7 @@ attn_status fwd_padded(const void* q, const void* k, const void* v, void* o, flo
     if ((s = launch_pad(k, ws + w.k_off, krows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
     if ((s = launch_pad(v, ws + w.v_off, krows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
     s = fwd_impl(ws + w.q_off, ws + w.k_off, ws + w.v_off, ws + w.o_off, lse, B, Hq, Hkv, Sq, Skv, w.Dp, scale,
-                 causal, dtype, rope_base, q_pos0, ws + w.inner_off, w.total - w.inner_off, st, D);
+                 causal, dtype, rope_base, q_pos0, ws + w.inner_off, w.total - w.inner_off, st, D, mk);
     if (s != ATTN_OK) return s;
     return launch_pad(ws + w.o_off, o, qrows, w.Dp * es_out, D * es_out, true, st);
 }
@@ -722,6 +733,23 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
                           workspace_bytes, static_cast<cudaStream_t>(stream));
     return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base, q_pos0, workspace,
                     workspace_bytes, static_cast<cudaStream_t>(stream), D);
+}
+
+attn_status attn_fwd_masked(const void* q, const void* k, const void* v, const float* mask, int64_t mask_batch_stride,
+                            int64_t mask_head_stride, void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Skv,
+                            int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
+                            void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+    if (!mask || (reinterpret_cast<uintptr_t>(mask) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (mask_batch_stride < 0 || mask_head_stride < 0) return ATTN_ERR_INVALID_ARG;
+    MaskArg mk;
+    mk.ptr = mask;
+    mk.bs = static_cast<long>(mask_batch_stride);
+    mk.hs = static_cast<long>(mask_head_stride);
+    if (D > 0 && !native_dim(D))
+        return fwd_padded(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base, q_pos0, workspace,
+                          workspace_bytes, static_cast<cudaStream_t>(stream), mk);
+    return fwd_impl(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base, q_pos0, workspace,
+                    workspace_bytes, static_cast<cudaStream_t>(stream), D, mk);
 }
 
 size_t attn_fwd_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, float rope_base,

@@ -17,7 +17,8 @@ template <int D>
 __global__ void __launch_bounds__(256) prefill_f32_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
     float* __restrict__ o, float* __restrict__ lse, int Hq, int Hkv, int Sq, int Skv, float scale,
-    int causal, const float2* __restrict__ rope_tab, int q_pos0) {
+    int causal, const float2* __restrict__ rope_tab, int q_pos0, const float* __restrict__ mask, long mask_bs,
+    long mask_hs) {
     constexpr int BR = 64, BK = 64, DC = D / 4;
     extern __shared__ float smem_f32[];
     float* sK = smem_f32;            // [BK][D]
@@ -54,6 +55,9 @@ __global__ void __launch_bounds__(256) prefill_f32_kernel(
     if (kmax > Skv - 1) kmax = Skv - 1;
     const int ntiles = kmax < 0 ? 0 : static_cast<int>(kmax / BK) + 1;
     const long my_last = causal ? static_cast<long>(i) + off : static_cast<long>(Skv) - 1;
+    // additive mask row of this query (scirs2 / whisper-apr: score = dot * scale + mask[q, k])
+    const float* mrow = (mask != nullptr && row_ok)
+                            ? mask + b * mask_bs + h * mask_hs + static_cast<long>(i) * Skv : nullptr;
 
     for (int jt = 0; jt < ntiles; ++jt) {
         const int k0 = jt * BK;
@@ -92,7 +96,8 @@ __global__ void __launch_bounds__(256) prefill_f32_kernel(
             part += __shfl_xor_sync(0xffffffffu, part, 1);
             part += __shfl_xor_sync(0xffffffffu, part, 2);
             if (j >= Skv || static_cast<long>(j) > my_last) continue;   // masked key
-            const float s = part * scale;
+            const float s = part * scale + (mrow != nullptr ? mrow[j] : 0.f);
+            if (s == -INFINITY) continue;                               // masked by the additive mask
             const float mn = fmaxf(m, s);
             const float corr = (m == -INFINITY) ? 0.f : expf(m - mn);
             const float p = expf(s - mn);

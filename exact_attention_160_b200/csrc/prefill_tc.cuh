@@ -92,6 +92,9 @@ struct TcParams {
     int n_row_tiles;          // row tiles per head in the work decomposition
     int heads_per_item;       // Hq / 2 when pairing heads, Hq otherwise
     float scale_log2;         // scale * log2(e)
+    const float* mask;        // additive mask on the scaled scores, or null
+    long mask_bs, mask_hs;    // its batch and head strides (elements; 0 broadcasts); rows of Skv
+    float inv_scale;          // 1 / scale: the mask enters the raw scores as mask / scale
 };
 
 struct TcTile {
@@ -428,8 +431,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 tc_fence_before();
                 mbar_arrive(bar_s_free + wg);
             }
-            // mask: keys past Skv, and (causal) keys beyond this row's diagonal
             const int k0 = j * 128;
+            if (p.mask != nullptr && qrow < p.Sq) {
+                // additive mask: S holds q.k unscaled, so add mask / scale; the exponent
+                // (s * scale + mask) * log2(e) - m then keeps its form
+                const float* mrow = p.mask + b * p.mask_bs + T.h * p.mask_hs + static_cast<long>(qrow) * p.Skv + k0;
+                const int ncol = p.Skv - k0;
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+                    for (int e = 0; e < 32; ++e)
+                        if (cb * 32 + e < ncol)
+                            sr[cb][e] = __float_as_uint(__uint_as_float(sr[cb][e]) + __ldg(mrow + cb * 32 + e) * p.inv_scale);
+            }
+            // mask: keys past Skv, and (causal) keys beyond this row's diagonal
             const long lim_causal = p.causal ? static_cast<long>(qrow) + off_c : static_cast<long>(p.Skv) - 1;
             const long lim = lim_causal < p.Skv - 1 ? lim_causal : static_cast<long>(p.Skv) - 1;
             float mx = -INFINITY;

@@ -10,6 +10,8 @@
  *                cache offset).
  *   attn_fwd_ex  attn_fwd with rotary position embedding applied to Q and K first.
  *                scirs2-neural 0.4.4 grouped_query_attention.rs (RotaryPositionEmbedding::apply).
+ *   attn_fwd_masked  attn_fwd_ex with an additive score mask.  whisper-apr 0.3.1
+ *                attention_generated.rs (compute_block_scores, scaled_dot_product_attention).
  *   attn_decode  one query token per (sequence, q head) against a KV cache, split along the keys
  *                and merged by logsumexp.  oxibonsai-model 0.1.4 src/layers/flash_decode.rs
  *                (flash_decode_tile, combine_tile_outputs, flash_decode_single_head);
@@ -110,6 +112,23 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
                         int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal,
                         attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
                         size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_fwd_masked -- attn_fwd_ex with an additive mask on the scaled scores:
+ *   s_ij = scale * q_i . k_j + mask[b, h, i, j]   (then the causal mask, if causal)
+ *   whisper-apr 0.3.1 src/model/attention_generated.rs (compute_block_scores: score = dot *
+ *   scale, then score += mask[q, k]; scaled_dot_product_attention adds the mask before the row
+ *   softmax).  mask: float32, element (b, h, i, j) at mask[b * mask_batch_stride +
+ *   h * mask_head_stride + i * Skv + j] (strides in elements, >= 0; 0 broadcasts, e.g. both 0
+ *   for one [Sq, Skv] mask shared by every batch and head), 4-byte aligned, read on the device.
+ *   -inf entries remove keys; a row whose scores are all -inf gets o = 0, lse = -inf.  Other
+ *   arguments, workspace and errors as attn_fwd_ex (attn_fwd_ex_workspace_size gives the bytes).
+ *   The mask is read with plain loads per row (it is a generality path: no TMA staging).
+ */
+attn_status attn_fwd_masked(const void* q, const void* k, const void* v, const float* mask, int64_t mask_batch_stride,
+                            int64_t mask_head_stride, void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Skv,
+                            int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
+                            void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
 /* Bytes of workspace attn_fwd_ex needs for these sizes: 0 for D in {64, 128} without RoPE; the
  * rotated-K halves with RoPE; the padded q, k, v, o (and the inner call's needs) otherwise.   */
