@@ -175,9 +175,10 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     p.inv_scale = 1.f / scale;
     const long grid = static_cast<long>(p.n_row_tiles) * B * p.heads_per_item;
     if (grid > 2147483647L) return ATTN_ERR_UNSUPPORTED;
-    auto kern = prefill_tc_kernel<D, ROPE>;
-    static bool attr_set = false;
-    if (!attr_set) {
+    // the masked kernel is a separate instantiation, so the unmasked one carries no mask code
+    auto kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true> : prefill_tc_kernel<D, ROPE, false>;
+    static bool attr_set[2] = {false, false};
+    if (!attr_set[mk.ptr != nullptr]) {
         // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds
         // fewer than the split asks for would stall in setmaxnreg.inc, so refuse it.
         cudaFuncAttributes fa;
@@ -192,7 +193,7 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
         }
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(prefill_tc_kernel)", cudaGetErrorString(e));
-        attr_set = true;
+        attr_set[mk.ptr != nullptr] = true;
     }
     kern<<<static_cast<unsigned>(grid), kTcThreads, C::SMEM_BYTES, st>>>(tq, tk, tkl, tv, p);
     return launch_status("prefill_tc_kernel");

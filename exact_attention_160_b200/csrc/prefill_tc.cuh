@@ -113,7 +113,7 @@ __device__ __forceinline__ int tc_kv_tiles(const TcParams& p, int r0) {
     return n < nkv_all ? static_cast<int>(n) : nkv_all;
 }
 
-template <int D, bool ROPE>
+template <int D, bool ROPE, bool MASK>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
@@ -432,7 +432,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 mbar_arrive(bar_s_free + wg);
             }
             const int k0 = j * 128;
-            if (p.mask != nullptr && qrow < p.Sq) {
+            if (MASK && qrow < p.Sq) {
                 // additive mask: S holds q.k unscaled, so add mask / scale; the exponent
                 // (s * scale + mask) * log2(e) - m then keeps its form
                 const float* mrow = p.mask + b * p.mask_bs + T.h * p.mask_hs + static_cast<long>(qrow) * p.Skv + k0;
