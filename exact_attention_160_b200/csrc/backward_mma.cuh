@@ -100,21 +100,24 @@ __device__ __forceinline__ void lda(uint32_t tile, int r0, int kk, int lane, uin
     ldsm_x4(tile + bsw<D>(r0 + (m & 1) * 8 + (lane & 7), 2 * kk + (m >> 1)), a[0], a[1], a[2], a[3]);
 }
 
-// acc[nt] (16 x 8 for 8 rows nt of `tile`) += A(16 x D) * tile^T, over all k steps.
+// acc[nt] (16 x 8 for 8 rows nt of `tile`) += A(16 x D) * tile^T, over all k steps.  The two
+// k steps that one ldmatrix brings in are issued in two passes over the eight accumulators, so
+// consecutive MMAs never wait on each other's result.
 template <int D>
 __device__ __forceinline__ void mma_rows_t(float (&acc)[8][4], uint32_t atile, int ar0, uint32_t btile, int lane) {
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk += 2) {
-        uint32_t a0[4], a1[4];
+        uint32_t a0[4], a1[4], bh[8][2];
         lda<D>(atile, ar0, kk, lane, a0);
         lda<D>(atile, ar0, kk + 1, lane, a1);
 #pragma unroll
         for (int nt = 0; nt < 8; ++nt) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(btile + bsw<D>(nt * 8 + (lane & 7), 2 * kk + (lane >> 3)), b0, b1, b2, b3);
+            uint32_t b0, b1;
+            ldsm_x4(btile + bsw<D>(nt * 8 + (lane & 7), 2 * kk + (lane >> 3)), b0, b1, bh[nt][0], bh[nt][1]);
             mma_bf16_16816(acc[nt], a0[0], a0[1], a0[2], a0[3], b0, b1);
-            mma_bf16_16816(acc[nt], a1[0], a1[1], a1[2], a1[3], b2, b3);
         }
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) mma_bf16_16816(acc[nt], a1[0], a1[1], a1[2], a1[3], bh[nt][0], bh[nt][1]);
     }
 }
 
