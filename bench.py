@@ -467,7 +467,8 @@ def run_gpu(args):
                                   "peak_source": how + " bf16_tflops (burst, cuBLAS bf16 GEMM); the backward "
                                                  "issues m16n8k16 mma.sync, not tcgen05"}}
         extra = {"backward": extra_bwd,
-                 "decode": {"workload": dec_w.name, "l2": "not flushed: the cache is larger than L2",
+                 "decode": {"workload": dec_w.name, "num_splits": dec_w.num_splits,
+                            "l2": "not flushed: the cache is larger than L2",
                             "value": round(whole_job_rate(dec["kv_bytes"], dec_ms, world) / 1e9, 1),
                             "unit": "GB/s", "ms_per_call": round(dec_ms, 4),
                             "roofline": roofline_decode(dec, peaks, how), "append": dec["append"]}}

@@ -145,8 +145,10 @@ C2 = Prefill("c2_bf16_mha_causal_B4_H8_S2048_D64", "bf16", 4, 8, 8, 2048, 2048, 
              seed=1002)
 C3 = Prefill("c3_bf16_gqa32x8_causal_rope_B2_S4096_D64", "bf16", 2, 32, 8, 4096, 4096, 64, True,
              1.0 / 8.0, rope_base=10000.0, seed=1003)
+# num_splits = 16: with the split policy (each split covers >= 512 keys) a sequence of L keys
+# uses min(L / 512, 16) splits of >= 1024 keys for every L >= 8192.
 C4 = Decode("c4_bf16_decode_B16_Hq32_Hkv8_D64_Smax32768", 16, 32, 8, 64, 32768, 1024, 32768,
-            1.0 / 8.0, 64, seed=1004)
+            1.0 / 8.0, 16, seed=1004)
 C5 = Prefill("c5_bf16_mha_causal_B1_H16_S16384_D128_peaked", "bf16", 1, 16, 16, 16384, 16384, 128,
              True, 1.0 / np.sqrt(128.0), qk_std=3.0, seed=1005)
 
