@@ -47,9 +47,10 @@ def _bind(path: str):
         lib.oracle_decode_split_f64.argtypes = [P, P, P, P, P, P, I, I, I, I, I, Dd, I]
         lib.oracle_attn_bwd_f64.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
         lib.oracle_attn_fwd_mask_f64.argtypes = [P, P, P, P, I64, I64, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
+        lib.oracle_attn_bwd_mask_f64.argtypes = [P, P, P, P, P, I64, I64, P, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
         for f in (lib.oracle_rope_f64, lib.oracle_attn_fwd_f64, lib.oracle_attn_fwd_tiled_f64,
                   lib.oracle_decode_f64, lib.oracle_decode_split_f64, lib.oracle_attn_bwd_f64,
-                  lib.oracle_attn_fwd_mask_f64):
+                  lib.oracle_attn_fwd_mask_f64, lib.oracle_attn_bwd_mask_f64):
             f.restype = I
     return lib
 
@@ -153,6 +154,31 @@ def attn_fwd_masked(q, k, v, mask, scale: float, causal: bool, rope_base: float 
                                             Hkv, Sq, Skv, D, float(scale), int(bool(causal)), float(rope_base),
                                             int(q_pos0)))
     return o, lse
+
+
+def _mask_strides(m, B, Hq, Sq, Skv):
+    if m.shape[-2:] != (Sq, Skv):
+        raise OracleError("mask shape")
+    if m.ndim == 2:
+        return 0, 0
+    if m.ndim == 3:
+        return Sq * Skv, 0
+    return Hq * Sq * Skv, Sq * Skv
+
+
+def attn_bwd_masked(q, k, v, dout, mask, scale: float, causal: bool, rope_base: float = 0.0, q_pos0: int = 0):
+    """attn_bwd for the forward with an additive mask (see attn_fwd_masked)."""
+    q, k, v, dout, m = _f32(q), _f32(k), _f32(v), _f32(dout), _f32(mask)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    bs, hs = _mask_strides(m, B, Hq, Sq, Skv)
+    dq = np.empty((B, Sq, Hq, D), dtype=np.float64)
+    dk = np.empty((B, Skv, Hkv, D), dtype=np.float64)
+    dv = np.empty((B, Skv, Hkv, D), dtype=np.float64)
+    _check(_load().oracle_attn_bwd_mask_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(m), bs, hs, _ptr(dq),
+                                            _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Skv, D, float(scale),
+                                            int(bool(causal)), float(rope_base), int(q_pos0)))
+    return dq, dk, dv
 
 
 def attn_fwd_tiled(q, k, v, scale: float, causal: bool, bq: int, bkv: int):

@@ -474,9 +474,10 @@ int oracle_decode_split_f64(const float* q, const float* kc, const float* vc,
  * rotation by the negated angle.  A row with no visible key contributes nothing.
  * q, dout [B,Sq,Hq,D]; k, v [B,Skv,Hkv,D] (float32 values); dq [B,Sq,Hq,D], dk, dv [B,Skv,Hkv,D]
  * (double).                                                                                  */
-int oracle_attn_bwd_f64(const float* q, const float* k, const float* v, const float* dout,
-                        double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Sq, int Skv,
-                        int D, double scale, int causal, double rope_base, int q_pos0) {
+static int attn_bwd_core(const float* q, const float* k, const float* v, const float* dout,
+                         const float* mask, int64_t mask_bstride, int64_t mask_hstride, double* dq, double* dk,
+                         double* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, double scale, int causal,
+                         double rope_base, int q_pos0) {
     int st = check_dims(B, Hq, Hkv, Sq, Skv, D);
     if (st) return st;
     if (rope_base > 0.0 && D % 2) return ORACLE_ERR_INVALID_ARG;
@@ -514,13 +515,19 @@ int oracle_attn_bwd_f64(const float* q, const float* k, const float* v, const fl
                         for (int d = 0; d < D; ++d) qd[d] = (double)q[qoff + d];
                         if (rope_base > 0.0) rope_vec(qd, (double)q_pos0 + (double)i, D, rope_base);
                         for (int d = 0; d < D; ++d) go[d] = (double)dout[qoff + d];
-                        /* scores and the three-pass softmax over the visible keys */
+                        /* scores (with the additive mask, if any) and the three-pass softmax */
+                        const float* mrow =
+                            mask ? mask + (long)b * mask_bstride + (long)hq * mask_hstride + (long)i * Skv : NULL;
                         double m = -INFINITY;
                         for (int j = 0; j < nvis; ++j) {
                             double dot = 0.0;
                             for (int d = 0; d < D; ++d) dot += qd[d] * Kd[(long)j * D + d];
-                            s[j] = scale * dot;
+                            s[j] = scale * dot + (mrow ? (double)mrow[j] : 0.0);
                             if (s[j] > m) m = s[j];
+                        }
+                        if (m == -INFINITY) { /* every key masked: no gradient through this row */
+                            for (int d = 0; d < D; ++d) dqo[d] = 0.0;
+                            continue;
                         }
                         double l = 0.0;
                         for (int j = 0; j < nvis; ++j) l += exp(s[j] - m);
@@ -568,6 +575,23 @@ int oracle_attn_bwd_f64(const float* q, const float* k, const float* v, const fl
         }
     }
     return fail ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+int oracle_attn_bwd_f64(const float* q, const float* k, const float* v, const float* dout,
+                        double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Sq, int Skv,
+                        int D, double scale, int causal, double rope_base, int q_pos0) {
+    return attn_bwd_core(q, k, v, dout, NULL, 0, 0, dq, dk, dv, B, Hq, Hkv, Sq, Skv, D, scale, causal,
+                         rope_base, q_pos0);
+}
+
+/* The backward of oracle_attn_fwd_mask_f64: the same definition with s_j including the mask.   */
+int oracle_attn_bwd_mask_f64(const float* q, const float* k, const float* v, const float* dout,
+                             const float* mask, int64_t mask_bstride, int64_t mask_hstride, double* dq,
+                             double* dk, double* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D,
+                             double scale, int causal, double rope_base, int q_pos0) {
+    if (!mask) return ORACLE_ERR_INVALID_ARG;
+    return attn_bwd_core(q, k, v, dout, mask, mask_bstride, mask_hstride, dq, dk, dv, B, Hq, Hkv, Sq, Skv, D,
+                         scale, causal, rope_base, q_pos0);
 }
 
 /* ------------------------------------------------------------------------------------------ */

@@ -583,6 +583,41 @@ def pin_backward_matches_finite_differences():
             _close(a, b, 2e-6 * max(1.0, float(np.max(np.abs(b)))), f"case {n} {name} vs finite differences")
 
 
+def pin_masked_backward_matches_finite_differences():
+    """The masked backward equals central differences of the masked *forward* oracle (per-head
+    mask with -inf entries, causal, GQA), and a zero mask gives the unmasked backward."""
+    B, Sq, Skv, Hq, Hkv, D = 1, 4, 5, 2, 1, 4
+    q = _grid(normal_f32(97, 0, (B, Sq, Hq, D)))
+    k = _grid(normal_f32(97, 1, (B, Skv, Hkv, D)))
+    v = _grid(normal_f32(97, 2, (B, Skv, Hkv, D)))
+    g = _grid(normal_f32(97, 3, (B, Sq, Hq, D)))
+    m = _grid(normal_f32(97, 4, (B, Hq, Sq, Skv)))
+    m[0, 1, 2, 0] = -np.inf
+    m[0, 0, 3, :] = -np.inf                               # a row masked everywhere
+    dq, dk, dv = oracle.attn_bwd_masked(q, k, v, g, m, 0.6, True)
+
+    def loss(qq, kk, vv):
+        o, _ = oracle.attn_fwd_masked(qq, kk, vv, m, 0.6, True)
+        return float(np.sum(o * g.astype(np.float64)))
+    eps = 2.0 ** -10
+    for which, ref in enumerate((dq, dk, dv)):
+        xs = [q.copy(), k.copy(), v.copy()]
+        flat = xs[which].reshape(-1)
+        fd = np.zeros(flat.size)
+        for idx in range(flat.size):
+            x0 = flat[idx]
+            flat[idx] = x0 + np.float32(eps)
+            lp = loss(*xs)
+            flat[idx] = x0 - np.float32(eps)
+            lm = loss(*xs)
+            flat[idx] = x0
+            fd[idx] = (lp - lm) / (2 * eps)
+        _close(ref.reshape(-1), fd, 2e-6 * max(1.0, float(np.max(np.abs(fd)))), f"masked backward {which}")
+    z = oracle.attn_bwd_masked(q, k, v, g, np.zeros((Sq, Skv), np.float32), 0.6, True)
+    for a, b in zip(z, oracle.attn_bwd(q, k, v, g, 0.6, True)):
+        _close(a, b, 1e-15, "zero mask backward")
+
+
 def pin_backward_invariants():
     """Without RoPE each row's dS sums to zero, so the key gradients of a (b, kv head) sum to
     zero; each row's probabilities sum to one, so the value gradients sum to the sum of dout over

@@ -47,6 +47,7 @@ MUTANTS = [
     ("mask_head_stride_ignored", "(long)hq * mask_hstride", "(long)0 * mask_hstride"),
     ("mask_all_inf_row_nan", "if (m == -INFINITY) {\n                            *lrow = -INFINITY;",
      "if (0) {\n                            *lrow = -INFINITY;"),
+    ("bwd_mask_dropped", "s[j] = scale * dot + (mrow ? (double)mrow[j] : 0.0);", "s[j] = scale * dot;"),
     ("bwd_dp_from_keys", "for (int d = 0; d < D; ++d) dot += go[d] * Vd[(long)j * D + d];",
      "for (int d = 0; d < D; ++d) dot += go[d] * Kd[(long)j * D + d];"),
 ]
