@@ -32,7 +32,7 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
            "attn_decode_workspace_size", "attn_decode_noalloc", "rope_apply", "attn_status_string",
            "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status", "attn_kv_append",
-           "attn_bwd", "attn_bwd_workspace_size", "attn_fwd_masked")
+           "attn_bwd", "attn_bwd_workspace_size", "attn_fwd_masked", "attn_bwd_masked")
 
 _lib = None
 
@@ -71,6 +71,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     I64 = ctypes.c_int64
     lib.attn_fwd_masked.argtypes = [P, P, P, P, I64, I64, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
     lib.attn_fwd_masked.restype = I
+    lib.attn_bwd_masked.argtypes = [P, P, P, P, I64, I64, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
+    lib.attn_bwd_masked.restype = I
     lib.attn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
     lib.attn_bwd.restype = I
     lib.attn_bwd_workspace_size.argtypes = [I, I, I, I, I, I, I, F, I]
@@ -168,6 +170,21 @@ def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: i
     return o, lse
 
 
+def _mask_strides(mask, Sq: int, Skv: int):
+    """(batch, head) element strides of a float32 mask [Sq, Skv], [B, Sq, Skv] or [B, Hq, Sq, Skv]
+    (size-1 or expanded dims broadcast); rows must be contiguous."""
+    if mask.dtype != torch.float32 or not mask.is_cuda or mask.shape[-2:] != (Sq, Skv) or mask.stride(-1) != 1 \
+            or mask.stride(-2) != Skv:
+        raise ValueError("mask must be a float32 CUDA tensor [..., Sq, Skv] with contiguous rows")
+    if mask.dim() == 2:
+        return 0, 0
+    if mask.dim() == 3:
+        return (mask.stride(0) if mask.shape[0] > 1 else 0), 0
+    if mask.dim() == 4:
+        return (mask.stride(0) if mask.shape[0] > 1 else 0), (mask.stride(1) if mask.shape[1] > 1 else 0)
+    raise ValueError("mask must have 2, 3 or 4 dims")
+
+
 def attn_fwd_masked(q, k, v, mask, scale: float, causal: bool, rope_base: float = 0.0, q_pos0: int = 0, o=None,
                     lse=None, workspace=None, out_dtype=None, stream=None):
     """Exact attention with an additive fp32 mask on the scaled scores.  mask: [Sq, Skv] (shared),
@@ -176,18 +193,7 @@ def attn_fwd_masked(q, k, v, mask, scale: float, causal: bool, rope_base: float 
     _need_cuda(q, k, v, o, lse, workspace)
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
-    if mask.dtype != torch.float32 or not mask.is_cuda or mask.shape[-2:] != (Sq, Skv) or mask.stride(-1) != 1 \
-            or mask.stride(-2) != Skv:
-        raise ValueError("mask must be a float32 CUDA tensor [..., Sq, Skv] with contiguous rows")
-    if mask.dim() == 2:
-        bs, hs = 0, 0
-    elif mask.dim() == 3:
-        bs, hs = mask.stride(0) if mask.shape[0] > 1 else 0, 0
-    elif mask.dim() == 4:
-        bs = mask.stride(0) if mask.shape[0] > 1 else 0
-        hs = mask.stride(1) if mask.shape[1] > 1 else 0
-    else:
-        raise ValueError("mask must have 2, 3 or 4 dims")
+    bs, hs = _mask_strides(mask, Sq, Skv)
     if o is None:
         o = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     if lse is None:
@@ -269,6 +275,30 @@ def attn_bwd(q, k, v, o, lse, dout, scale: float, causal: bool, rope_base: float
                       Hkv, Sq, Skv, D, float(scale), int(bool(causal)), code, float(rope_base), int(q_pos0),
                       _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_bwd_masked(q, k, v, mask, o, lse, dout, scale: float, causal: bool, rope_base: float = 0.0,
+                    q_pos0: int = 0, grad_dtype=None, workspace=None, stream=None):
+    """attn_bwd for attn_fwd_masked (same mask)."""
+    lib = load_library()
+    _need_cuda(q, k, v, o, lse, dout, workspace)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    bs, hs = _mask_strides(mask, Sq, Skv)
+    gd = q.dtype if grad_dtype is None else grad_dtype
+    code = ATTN_FP32 if q.dtype == torch.float32 else (ATTN_BF16_OUT_F32 if gd == torch.float32 else ATTN_BF16)
+    dq = torch.empty(q.shape, dtype=gd, device=q.device)
+    dk = torch.empty(k.shape, dtype=gd, device=q.device)
+    dv = torch.empty(v.shape, dtype=gd, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(bwd_workspace_bytes(q, k, rope_base, q_pos0, gd), 1), dtype=torch.uint8,
+                                device=q.device)
+    st = lib.attn_bwd_masked(_ptr(q), _ptr(k), _ptr(v), _ptr(mask), bs, hs, _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                             _ptr(dk), _ptr(dv), B, Hq, Hkv, Sq, Skv, D, float(scale), int(bool(causal)), code,
+                             float(rope_base), int(q_pos0), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "attn_bwd_masked")
     return dq, dk, dv
 
 

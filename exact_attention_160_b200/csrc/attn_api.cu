@@ -389,7 +389,7 @@ template <int D, typename T>
 attn_status launch_bwd(const T* q, const T* k, const T* v, const T* o, const float* lse, const T* dout, void* dq,
                        void* dk, void* dv, bool g_f32, int B, int Hq, int Hkv, int Sq, int Skv, float scale,
                        int causal, const float2* tab, int q_pos0, uint8_t* ws, const BwdWorkspace& w,
-                       cudaStream_t st) {
+                       cudaStream_t st, MaskArg mk) {
     float* Qf = reinterpret_cast<float*>(ws + w.q_off);
     float* dOf = reinterpret_cast<float*>(ws + w.do_off);
     float* Kf = reinterpret_cast<float*>(ws + w.k_off);
@@ -419,6 +419,9 @@ attn_status launch_bwd(const T* q, const T* k, const T* v, const T* o, const flo
     p.q_pos0 = q_pos0;
     p.causal = causal;
     p.scale = scale;
+    p.mask = mk.ptr;
+    p.mask_bs = mk.bs;
+    p.mask_hs = mk.hs;
     const size_t smem_dq = 2 * kBwdTile * D * sizeof(float);
     const size_t smem_dkdv = (2 * kBwdTile * D + 2 * kBwdTile) * sizeof(float);
     static bool attr_set = false;
@@ -470,7 +473,8 @@ template <int D, bool ROPE>
 attn_status launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
                            const __nv_bfloat16* o, const float* lse, const __nv_bfloat16* dout, void* dq, void* dk,
                            void* dv, bool g_f32, int B, int Hq, int Hkv, int Sq, int Skv, float scale, int causal,
-                           const float2* tab, int q_pos0, uint8_t* ws, const BmWorkspace& w, cudaStream_t st) {
+                           const float2* tab, int q_pos0, uint8_t* ws, const BmWorkspace& w, cudaStream_t st,
+                           MaskArg mk) {
     float* Dvec = reinterpret_cast<float*>(ws + w.d_off);
     const long nq = static_cast<long>(B) * Sq * Hq;
     bwd_rowdot_kernel<D><<<static_cast<unsigned>((nq * (D / 8) + 255) / 256), 256, 0, st>>>(o, dout, Dvec, nq, Sq, Hq);
@@ -508,26 +512,29 @@ attn_status launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const
     p.q_pos0 = q_pos0;
     p.causal = causal;
     p.scale = scale;
+    p.mask = mk.ptr;
+    p.mask_bs = mk.bs;
+    p.mask_hs = mk.hs;
     using C = BmCfg<D, ROPE>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(bwd_dq_mma_kernel<D, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::SMEM);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(bwd_dkdv_mma_kernel<D, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     C::SMEM);
+    const bool masked = mk.ptr != nullptr;   // separate instantiations: the unmasked ones carry no mask code
+    auto kdq = masked ? bwd_dq_mma_kernel<D, ROPE, true> : bwd_dq_mma_kernel<D, ROPE, false>;
+    auto kkv = masked ? bwd_dkdv_mma_kernel<D, ROPE, true> : bwd_dkdv_mma_kernel<D, ROPE, false>;
+    static bool attr_set[2] = {false, false};
+    if (!attr_set[masked]) {
+        cudaError_t e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        if (e == cudaSuccess) e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(bwd mma kernels)", cudaGetErrorString(e));
-        attr_set = true;
+        attr_set[masked] = true;
     }
     p.g_f32 = g_f32 ? static_cast<float*>(dq) : nullptr;
     p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq);
-    bwd_dq_mma_kernel<D, ROPE><<<dim3((Sq + kBmRows - 1) / kBmRows, Hq, B), kBmThreads, C::SMEM, st>>>(p);
+    kdq<<<dim3((Sq + kBmRows - 1) / kBmRows, Hq, B), kBmThreads, C::SMEM, st>>>(p);
     if ((s = launch_status("bwd_dq_mma_kernel")) != ATTN_OK) return s;
     p.g_f32 = g_f32 ? static_cast<float*>(dk) : nullptr;
     p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
     p.g2_f32 = g_f32 ? static_cast<float*>(dv) : nullptr;
     p.g2_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
-    bwd_dkdv_mma_kernel<D, ROPE><<<dim3((Skv + kBmRows - 1) / kBmRows, Hkv, B), kBmThreads, C::SMEM, st>>>(p);
+    kkv<<<dim3((Skv + kBmRows - 1) / kBmRows, Hkv, B), kBmThreads, C::SMEM, st>>>(p);
     return launch_status("bwd_dkdv_mma_kernel");
 }
 
@@ -568,7 +575,7 @@ PadBwd pad_bwd_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dt
 attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
                      int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
-                     size_t workspace_bytes, attn_stream_t stream, int rope_dim);
+                     size_t workspace_bytes, attn_stream_t stream, int rope_dim, MaskArg mk);
 
 }  // namespace
 
@@ -579,13 +586,16 @@ size_t attn_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, a
     return bwd_inner_bytes(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base, q_pos0);
 }
 
-attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
-                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
-                     int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
-                     size_t workspace_bytes, attn_stream_t stream) {
+namespace {
+
+// attn_bwd and attn_bwd_masked: native head dims go straight to bwd_impl, others through padding.
+attn_status bwd_entry(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                      int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
+                      size_t workspace_bytes, attn_stream_t stream, MaskArg mk) {
     if (D <= 0 || native_dim(D))
         return bwd_impl(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base,
-                        q_pos0, workspace, workspace_bytes, stream, D);
+                        q_pos0, workspace, workspace_bytes, stream, D, mk);
     attn_status s = check_common(B, Hq, Hkv, Sq, Skv, 64, scale, causal);   // everything but D
     if (s != ATTN_OK) return s;
     if (!paddable_dim(D)) return ATTN_ERR_UNSUPPORTED;
@@ -607,11 +617,36 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
     if ((s = launch_pad(dout, ws + w.g_off, qrows, D * es_in, w.Dp * es_in, false, st)) != ATTN_OK) return s;
     s = bwd_impl(ws + w.q_off, ws + w.k_off, ws + w.v_off, ws + w.o_off, lse, ws + w.g_off, ws + w.dq_off,
                  ws + w.dk_off, ws + w.dv_off, B, Hq, Hkv, Sq, Skv, w.Dp, scale, causal, dtype, rope_base, q_pos0,
-                 ws + w.inner_off, w.total - w.inner_off, stream, D);
+                 ws + w.inner_off, w.total - w.inner_off, stream, D, mk);
     if (s != ATTN_OK) return s;
     if ((s = launch_pad(ws + w.dq_off, dq, qrows, w.Dp * es_g, D * es_g, true, st)) != ATTN_OK) return s;
     if ((s = launch_pad(ws + w.dk_off, dk, krows, w.Dp * es_g, D * es_g, true, st)) != ATTN_OK) return s;
     return launch_pad(ws + w.dv_off, dv, krows, w.Dp * es_g, D * es_g, true, st);
+}
+
+}  // namespace
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
+                     int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
+                     size_t workspace_bytes, attn_stream_t stream) {
+    return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base,
+                     q_pos0, workspace, workspace_bytes, stream, MaskArg{});
+}
+
+attn_status attn_bwd_masked(const void* q, const void* k, const void* v, const float* mask, int64_t mask_batch_stride,
+                            int64_t mask_head_stride, const void* o, const float* lse, const void* dout, void* dq,
+                            void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal,
+                            attn_dtype dtype, float rope_base, int q_pos0, void* workspace, size_t workspace_bytes,
+                            attn_stream_t stream) {
+    if (!mask || (reinterpret_cast<uintptr_t>(mask) & 3u) != 0) return ATTN_ERR_INVALID_ARG;
+    if (mask_batch_stride < 0 || mask_head_stride < 0) return ATTN_ERR_INVALID_ARG;
+    MaskArg mk;
+    mk.ptr = mask;
+    mk.bs = static_cast<long>(mask_batch_stride);
+    mk.hs = static_cast<long>(mask_head_stride);
+    return bwd_entry(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, Sq, Skv, D, scale, causal, dtype, rope_base,
+                     q_pos0, workspace, workspace_bytes, stream, mk);
 }
 
 namespace {
@@ -619,7 +654,7 @@ namespace {
 attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                      void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale,
                      int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
-                     size_t workspace_bytes, attn_stream_t stream, int rope_dim) {
+                     size_t workspace_bytes, attn_stream_t stream, int rope_dim, MaskArg mk) {
     attn_status s = check_common(B, Hq, Hkv, Sq, Skv, D, scale, causal);
     if (s != ATTN_OK) return s;
     if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID_ARG;
@@ -652,22 +687,22 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
                     *vf = static_cast<const float*>(v), *of = static_cast<const float*>(o),
                     *gf = static_cast<const float*>(dout);
         return D == 64 ? launch_bwd<64>(qf, kf, vf, of, lse, gf, dq, dk, dv, true, B, Hq, Hkv, Sq, Skv, scale, causal,
-                                        tab, q_pos0, ws, w, st)
+                                        tab, q_pos0, ws, w, st, mk)
                        : launch_bwd<128>(qf, kf, vf, of, lse, gf, dq, dk, dv, true, B, Hq, Hkv, Sq, Skv, scale,
-                                         causal, tab, q_pos0, ws, w, st);
+                                         causal, tab, q_pos0, ws, w, st, mk);
     }
     using bf = __nv_bfloat16;
     const bf *qb = static_cast<const bf*>(q), *kb = static_cast<const bf*>(k), *vb = static_cast<const bf*>(v),
              *ob = static_cast<const bf*>(o), *gb = static_cast<const bf*>(dout);
     if (D == 64)
         return rope ? launch_bwd_mma<64, true>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
-                                               causal, tab, q_pos0, ws, wm, st)
+                                               causal, tab, q_pos0, ws, wm, st, mk)
                     : launch_bwd_mma<64, false>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
-                                                causal, tab, q_pos0, ws, wm, st);
+                                                causal, tab, q_pos0, ws, wm, st, mk);
     return rope ? launch_bwd_mma<128, true>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
-                                            causal, tab, q_pos0, ws, wm, st)
+                                            causal, tab, q_pos0, ws, wm, st, mk)
                 : launch_bwd_mma<128, false>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
-                                             causal, tab, q_pos0, ws, wm, st);
+                                             causal, tab, q_pos0, ws, wm, st, mk);
 }
 
 }  // namespace

@@ -3,7 +3,7 @@
 // The method (scirs2-neural 0.4.3, src/layers/flash_attention.rs, flash_backward_head: FA-2's
 // backward, Algorithm 4 of Dao 2023): with the row logsumexp saved by the forward, the
 // probabilities are recomputed tile by tile instead of stored,
-//   P_ij = exp(scale * q_i . k_j - lse_i)            (0 for masked keys and rows without keys)
+//   P_ij = exp(scale * q_i . k_j [+ mask_ij] - lse_i) (0 for masked keys and rows without keys)
 //   D_i  = sum_d dO_id O_id
 //   dS_ij = P_ij (dO_i . v_j - D_i)
 //   dV_j += P_ij dO_i,   dK_j += scale dS_ij q_i,   dQ_i += scale dS_ij k_j
@@ -12,7 +12,8 @@
 // and k, and the gradients are rotated back (the transpose of a rotation is the rotation by the
 // negated angle).
 //
-// B200 layout of the work (fp32 on the CUDA cores; the tensor-core version is future work):
+// This file is the fp32 path (ATTN_FP32 inputs, CUDA cores); bf16 inputs take the tensor-core
+// kernels of backward_mma.cuh.  Layout of the work:
 //   bwd_prep_q_kernel    one warp per (b, i, h): D_i, dO and q (rotated) as fp32 copies
 //   bwd_prep_kv_kernel   one warp per (b, j, kvh): k (rotated) and v as fp32 copies
 //   bwd_dq_kernel<D>     one CTA per (b, h, 64 query rows), 4 threads per row, each owning D/4
@@ -109,6 +110,8 @@ struct BwdParams {
     int B, Hq, Hkv, Sq, Skv, q_pos0;
     int causal;
     float scale;
+    const float* mask;       // additive mask of the forward or null; element strides below, rows of Skv
+    long mask_bs, mask_hs;
 };
 
 // Sum over the 4 threads of a row (lanes 4r .. 4r+3 of the warp).
@@ -193,7 +196,10 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dq_kernel(const BwdParams p) 
             s = quad_sum(s);
             dp = quad_sum(dp);
             const bool vis = k0 + jj < nvis;
-            const float pr = vis ? __expf(s * p.scale - lse) : 0.f;
+            const float mval = (vis && p.mask != nullptr)
+                                   ? p.mask[b * p.mask_bs + h * p.mask_hs + static_cast<long>(i) * p.Skv + k0 + jj]
+                                   : 0.f;
+            const float pr = vis ? __expf(s * p.scale + mval - lse) : 0.f;
             const float ds = pr * (dp - Dv) * p.scale;
 #pragma unroll
             for (int e = 0; e < DQ; ++e) acc[e] = fmaf(ds, kr[e], acc[e]);
@@ -277,7 +283,10 @@ __global__ void __launch_bounds__(kBwdThreads) bwd_dkdv_kernel(const BwdParams p
                 const long i = i0 + ii;
                 const float lse = sL[ii];
                 const bool vis = live && lse != -INFINITY && (!p.causal || static_cast<long>(j) <= i + off_c);
-                const float pr = vis ? __expf(s * p.scale - lse) : 0.f;
+                const float mval = (vis && p.mask != nullptr)
+                                       ? p.mask[b * p.mask_bs + h * p.mask_hs + i * p.Skv + j]
+                                       : 0.f;
+                const float pr = vis ? __expf(s * p.scale + mval - lse) : 0.f;
                 const float ds = pr * (dp - sD[ii]) * p.scale;
 #pragma unroll
                 for (int e = 0; e < DQ; ++e) {

@@ -69,6 +69,8 @@ struct BmParams {
     __nv_bfloat16* g2_bf16;
     int Hq, Hkv, Sq, Skv, q_pos0, causal;
     float scale;
+    const float* mask;          // additive mask of the forward (MASK kernels), element strides:
+    long mask_bs, mask_hs;      // batch, head; rows of Skv
 };
 
 // Store a 16-row x D accumulator fragment set (rows g, g+8 of the warp) with optional RoPE undo.
@@ -157,7 +159,7 @@ struct BmCfg {
 };
 
 // dQ: CTA (64 query rows, q head h, batch b).
-template <int D, bool ROPE>
+template <int D, bool ROPE, bool MASK>
 __global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p) {
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
@@ -242,7 +244,11 @@ __global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p
                 const long key = k0 + nt * 8 + 2 * t4 + (e & 1);
                 const bool top = e < 2;
                 const bool vis = key < (top ? nv_a : nv_b);
-                const float pr = vis ? fast_exp2(s[nt][e] * sl2 - (top ? lse_a : lse_b)) : 0.f;
+                float mb = 0.f;   // the forward's additive mask, in log2 units
+                if (MASK && vis)
+                    mb = __ldg(p.mask + b * p.mask_bs + h * p.mask_hs + static_cast<long>(top ? ra : rb) * p.Skv + key) *
+                         kLog2e;
+                const float pr = vis ? fast_exp2(s[nt][e] * sl2 + mb - (top ? lse_a : lse_b)) : 0.f;
                 s[nt][e] = pr * (dp[nt][e] - (top ? d_a : d_b)) * p.scale;
             }
         }
@@ -261,7 +267,7 @@ __global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p
 }
 
 // dK, dV: CTA (64 keys, kv head, batch b); loops over the group's q heads and the query tiles.
-template <int D, bool ROPE>
+template <int D, bool ROPE, bool MASK>
 __global__ void __launch_bounds__(kBmThreads) bwd_dkdv_mma_kernel(const BmParams p) {
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
@@ -347,7 +353,11 @@ __global__ void __launch_bounds__(kBmThreads) bwd_dkdv_mma_kernel(const BmParams
                 const float lse = sL[qi];
                 const bool vis = qi < qvalid && key < p.Skv && lse != -INFINITY &&
                                  (!p.causal || key <= i0 + qi + off_c);
-                const float pr = vis ? fast_exp2(s[nt][e] * sl2 - lse * kLog2e) : 0.f;
+                float mb = 0.f;   // the forward's additive mask, in log2 units
+                if (MASK && vis)
+                    mb = __ldg(p.mask + b * p.mask_bs + static_cast<long>(kvh * G + (t / t_per_head)) * p.mask_hs +
+                               (i0 + qi) * p.Skv + key) * kLog2e;
+                const float pr = vis ? fast_exp2(s[nt][e] * sl2 + mb - lse * kLog2e) : 0.f;
                 dp[nt][e] = pr * (dp[nt][e] - sD[qi]) * p.scale;
                 s[nt][e] = pr;
             }

@@ -215,6 +215,18 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
                      int causal, attn_dtype dtype, float rope_base, int q_pos0, void* workspace,
                      size_t workspace_bytes, attn_stream_t stream);
 
+/*
+ * attn_bwd_masked -- attn_bwd for attn_fwd_masked: the probabilities are recomputed with the
+ * same additive mask (same pointer and strides as the forward); mask entries are constants, so
+ * no gradient flows to them.  Arguments, workspace (attn_bwd_workspace_size) and errors as
+ * attn_bwd.
+ */
+attn_status attn_bwd_masked(const void* q, const void* k, const void* v, const float* mask, int64_t mask_batch_stride,
+                            int64_t mask_head_stride, const void* o, const float* lse, const void* dout, void* dq,
+                            void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal,
+                            attn_dtype dtype, float rope_base, int q_pos0, void* workspace, size_t workspace_bytes,
+                            attn_stream_t stream);
+
 /* Bytes of workspace attn_bwd needs for these sizes and dtype (fp32: fp32 copies of rotated q
  * and k, dout, v; bf16: the rotated q and k as hi/lo bf16 pairs with RoPE; both: the row sums
  * D_i and, with RoPE, the angle table); 0 for invalid sizes.                               */

@@ -70,3 +70,35 @@ def test_expanded_head_broadcast_mask():
     torch.cuda.synchronize()
     ro, rl = oracle.attn_fwd_masked(x["q"], x["k"], x["v"], m[:, 0], w.scale, w.causal)
     compare(to_host_f64(o), ro, to_host_f64(lse), rl, TOL_BF16_O, TOL_BF16_LSE, "expanded mask")
+
+
+BWD_CASES = [CASES[0], CASES[1], CASES[2], CASES[4], CASES[5], CASES[6]]
+
+
+@pytest.mark.parametrize("w,kind", BWD_CASES, ids=lambda c: c.name if hasattr(c, "name") else c)
+def test_masked_backward_matches_oracle(w, kind):
+    """attn_bwd_masked with o and lse of the oracle's masked forward (bf16: 1e-2, fp32: 2e-5 of the
+    largest reference gradient, as in tests/test_gpu_backward.py)."""
+    x, dev = make_prefill(w)
+    m = _mask(kind, w)
+    if w.dtype == "fp32":
+        g = si.normal_f32(w.seed, 7, (w.B, w.Sq, w.Hq, w.D))
+        dout = torch.from_numpy(g).cuda()
+        tol = 2e-5
+    else:
+        gb, g = si.bf16_normal(w.seed, 7, (w.B, w.Sq, w.Hq, w.D))
+        dout = torch.from_numpy(np.ascontiguousarray(gb).view(np.int16)).view(torch.bfloat16).cuda()
+        tol = 1e-2
+    ro, rl = oracle.attn_fwd_masked(x["q"], x["k"], x["v"], m, w.scale, w.causal, w.rope_base, w.q_pos0)
+    o = torch.from_numpy(ro.astype(np.float32)).cuda().to(dev["q"].dtype)
+    lse = torch.from_numpy(rl.astype(np.float32)).cuda()
+    dq, dk, dv = ea.attn_bwd_masked(dev["q"], dev["k"], dev["v"], torch.from_numpy(m).cuda(), o, lse, dout, w.scale,
+                                    w.causal, w.rope_base, w.q_pos0, grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ea.read_device_status() == 0
+    rq, rk, rv = oracle.attn_bwd_masked(x["q"], x["k"], x["v"], g, m, w.scale, w.causal, w.rope_base, w.q_pos0)
+    for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
+        gh = got.cpu().numpy().astype(np.float64)
+        assert np.isfinite(gh).all(), name
+        err = float(np.max(np.abs(gh - ref)) / max(1.0, float(np.max(np.abs(ref)))))
+        assert err <= tol, (w.name, name, err)
