@@ -167,6 +167,14 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     p.pair_heads = (G % 2 == 0) ? 1 : 0;
     p.n_row_tiles = p.pair_heads ? (Sq + 127) / 128 : (Sq + 255) / 256;
     p.heads_per_item = p.pair_heads ? Hq / 2 : Hq;
+    // A problem whose tile pairs fill less than one wave of the 148 SMs runs one query tile per
+    // CTA instead: twice the CTAs, and each SM's exponentials are shared by one tile, not two.
+    if (static_cast<long>(p.n_row_tiles) * B * p.heads_per_item < 148) {
+        p.single_tile = 1;
+        p.pair_heads = 0;
+        p.n_row_tiles = (Sq + 127) / 128;
+        p.heads_per_item = Hq;
+    }
     p.q_pos0 = q_pos0;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.mask = mk.ptr;

@@ -88,6 +88,7 @@ struct TcParams {
     int B, Hq, Hkv, Sq, Skv;
     int causal;
     int pair_heads;           // 1: tile pair = two heads of a group; 0: two row tiles of one head
+    int single_tile;          // 1: one query tile per CTA (small problems: twice the CTAs)
     int q_pos0;
     int n_row_tiles;          // row tiles per head in the work decomposition
     int heads_per_item;       // Hq / 2 when pairing heads, Hq otherwise
@@ -147,7 +148,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const int b = rem / p.heads_per_item;
     const int hi = rem % p.heads_per_item;
     TcTile tile[2];
-    if (p.pair_heads) {
+    if (p.single_tile) {
+        tile[0].h = tile[1].h = hi;
+        tile[0].r0 = rt * 128;
+        tile[1].r0 = p.Sq;    // inactive
+    } else if (p.pair_heads) {
         tile[0].h = 2 * hi;
         tile[1].h = 2 * hi + 1;
         tile[0].r0 = tile[1].r0 = rt * 128;

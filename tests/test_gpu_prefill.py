@@ -127,3 +127,29 @@ def test_repeated_calls_are_deterministic():
     o2, l2 = ea.attn_fwd(dev["q"], dev["k"], dev["v"], w.scale, True)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+# Problems with at least 148 tile pairs run two query tiles per CTA; smaller ones one tile per
+# CTA.  The cases below are sized to stay in the paired decomposition (row pairs of one head for
+# odd groups, head pairs for even groups) while keeping ragged tails, offsets and RoPE.
+PAIRED_CASES = [
+    P("paired_rows_odd_group_ragged", "bf16", 4, 40, 8, 300, 300, 64, True, seed=91),       # 2 x 4 x 40 = 320 pairs
+    P("paired_heads_gqa8_rope_offset", "bf16", 5, 32, 4, 200, 330, 64, True, rope_base=10000.0, q_pos0=130,
+      seed=92),                                                                              # 2 x 5 x 16 = 160
+    P("paired_heads_d128_noncausal", "bf16", 3, 64, 32, 130, 150, 128, False, seed=93),   # 2 x 3 x 32 = 192
+]
+
+
+@pytest.mark.parametrize("w", PAIRED_CASES, ids=[c.name for c in PAIRED_CASES])
+def test_paired_decomposition_matches_oracle(w):
+    """Sampled rows of every (batch, head) plus tile edges, against the oracle."""
+    from attn_cases import gather_rows, sample_rows
+    x, dev = make_prefill(w)
+    o, lse = ea.attn_fwd_ex(dev["q"], dev["k"], dev["v"], w.scale, w.causal, w.rope_base, w.q_pos0,
+                            out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ea.read_device_status() == 0
+    rows = sample_rows(w, 1500, seed=5)
+    ro, rl = oracle.attn_fwd(x["q"], x["k"], x["v"], w.scale, w.causal, w.rope_base, w.q_pos0, rows=rows)
+    go, gl = gather_rows(to_host_f64(o), to_host_f64(lse), rows, w)
+    compare(go, ro, gl, rl, TOL_BF16_O, TOL_BF16_LSE, w.name)
