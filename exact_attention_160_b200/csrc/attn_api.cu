@@ -167,9 +167,10 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     p.pair_heads = (G % 2 == 0) ? 1 : 0;
     p.n_row_tiles = p.pair_heads ? (Sq + 127) / 128 : (Sq + 255) / 256;
     p.heads_per_item = p.pair_heads ? Hq / 2 : Hq;
-    // A problem whose tile pairs fill less than one wave of the 148 SMs runs one query tile per
-    // CTA instead: twice the CTAs, and each SM's exponentials are shared by one tile, not two.
-    if (static_cast<long>(p.n_row_tiles) * B * p.heads_per_item < 148) {
+    // A problem so small that even one query tile per CTA fits in one wave of the 148 SMs runs
+    // that way: twice the CTAs of the paired decomposition, each SM's exponentials spent on one
+    // tile.  (When the single tiles would need a second wave, the pairs' shared K/V loads win.)
+    if (static_cast<long>((Sq + 127) / 128) * B * Hq <= 148) {
         p.single_tile = 1;
         p.pair_heads = 0;
         p.n_row_tiles = (Sq + 127) / 128;

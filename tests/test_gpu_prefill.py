@@ -129,8 +129,8 @@ def test_repeated_calls_are_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
-# Problems with at least 148 tile pairs run two query tiles per CTA; smaller ones one tile per
-# CTA.  The cases below are sized to stay in the paired decomposition (row pairs of one head for
+# Problems whose single query tiles would exceed 148 CTAs run two query tiles per CTA; smaller
+# ones one tile per CTA.  The cases below are sized to stay in the paired decomposition (row pairs of one head for
 # odd groups, head pairs for even groups) while keeping ragged tails, offsets and RoPE.
 PAIRED_CASES = [
     P("paired_rows_odd_group_ragged", "bf16", 4, 40, 8, 300, 300, 64, True, seed=91),       # 2 x 4 x 40 = 320 pairs
