@@ -160,7 +160,7 @@ struct BmCfg {
 
 // dQ: CTA (64 query rows, q head h, batch b).
 template <int D, bool ROPE, bool MASK>
-__global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p) {
+__global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dq_mma_kernel(const BmParams p) {
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
     const uint32_t base = smem_u32(bm_smem);
@@ -268,7 +268,7 @@ __global__ void __launch_bounds__(kBmThreads) bwd_dq_mma_kernel(const BmParams p
 
 // dK, dV: CTA (64 keys, kv head, batch b); loops over the group's q heads and the query tiles.
 template <int D, bool ROPE, bool MASK>
-__global__ void __launch_bounds__(kBmThreads) bwd_dkdv_mma_kernel(const BmParams p) {
+__global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dkdv_mma_kernel(const BmParams p) {
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
     const uint32_t base = smem_u32(bm_smem);
