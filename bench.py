@@ -531,8 +531,10 @@ def run_reference(args):
     if not isinstance(w, si.Prefill):
         raise SystemExit("the reference arm times prefill workloads")
     x = si.prefill_inputs(w)
-    # each step: every 64th query row of every (batch, head) -- a bounded slice of the workload
-    rows = np.arange(0, w.B * w.Hq * w.Sq, 64, dtype=np.int64)
+    # each step: every r-th query row of every (batch, head), r chosen so that a step is at most
+    # about 20 GFLOP of fp64 work (the whole workload when it is smaller) -- a bounded slice
+    stride = max(1, int(np.ceil(w.flops / 20e9)))
+    rows = np.arange(0, w.B * w.Hq * w.Sq, stride, dtype=np.int64)
     i = rows % w.Sq
     vis = np.clip(i + (w.Skv - w.Sq) + 1, 0, w.Skv) if w.causal else np.full_like(i, w.Skv)
     flops = float(np.sum(4.0 * w.D * vis))
@@ -544,7 +546,8 @@ def run_reference(args):
     dt = (time.perf_counter() - t0) / args.steps
     value = flops / dt / 1e12
     threads = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    sample = f"{len(rows)} query rows per step (every 64th row of every (batch, head)), {flops / 1e9:.3f} GFLOP fp64"
+    sample = (f"{len(rows)} query rows per step (every {stride}th row of every (batch, head)), "
+              f"{flops / 1e9:.3f} GFLOP fp64")
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
