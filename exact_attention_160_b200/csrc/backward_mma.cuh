@@ -20,7 +20,7 @@ namespace attn {
 
 constexpr int kBmThreads = 128;   // 4 warps x 16 rows = 64 rows per CTA
 constexpr int kBmRows = 64;
-constexpr int kBmTile = 64;       // keys (dq) / query rows (dkdv) per step
+constexpr int kBmTile = 64;       // keys (dq) / query rows (dkdv) per step at D=64 (32 at D=128)
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Byte offset of 16-byte chunk ch (8 bf16) of row r in a tile of rows of D bf16, with the low
@@ -43,10 +43,10 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// stage_rows with cp.async: rows >= nvalid are zero-filled (their source address is row 0).
-template <int D>
+// Stage ROWS rows with cp.async: rows >= nvalid are zero-filled (their source address is row 0).
+template <int D, int ROWS>
 __device__ __forceinline__ void stage_rows_async(uint32_t tile, const __nv_bfloat16* src, long stride, int nvalid) {
-    for (int idx = threadIdx.x; idx < kBmTile * (D / 8); idx += kBmThreads) {
+    for (int idx = threadIdx.x; idx < ROWS * (D / 8); idx += kBmThreads) {
         const int r = idx / (D / 8), ch = idx % (D / 8);
         const bool ok = r < nvalid;
         cp_async16(tile + bsw<D>(r, ch), src + (ok ? r * stride : 0) + ch * 8, ok);
@@ -105,29 +105,29 @@ __device__ __forceinline__ void lda(uint32_t tile, int r0, int kk, int lane, uin
 // acc[nt] (16 x 8 for 8 rows nt of `tile`) += A(16 x D) * tile^T, over all k steps.  The two
 // k steps that one ldmatrix brings in are issued in two passes over the eight accumulators, so
 // consecutive MMAs never wait on each other's result.
-template <int D>
-__device__ __forceinline__ void mma_rows_t(float (&acc)[8][4], uint32_t atile, int ar0, uint32_t btile, int lane) {
+template <int D, int NTB>
+__device__ __forceinline__ void mma_rows_t(float (&acc)[NTB][4], uint32_t atile, int ar0, uint32_t btile, int lane) {
 #pragma unroll
     for (int kk = 0; kk < D / 16; kk += 2) {
-        uint32_t a0[4], a1[4], bh[8][2];
+        uint32_t a0[4], a1[4], bh[NTB][2];
         lda<D>(atile, ar0, kk, lane, a0);
         lda<D>(atile, ar0, kk + 1, lane, a1);
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < NTB; ++nt) {
             uint32_t b0, b1;
             ldsm_x4(btile + bsw<D>(nt * 8 + (lane & 7), 2 * kk + (lane >> 3)), b0, b1, bh[nt][0], bh[nt][1]);
             mma_bf16_16816(acc[nt], a0[0], a0[1], a0[2], a0[3], b0, b1);
         }
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) mma_bf16_16816(acc[nt], a1[0], a1[1], a1[2], a1[3], bh[nt][0], bh[nt][1]);
+        for (int nt = 0; nt < NTB; ++nt) mma_bf16_16816(acc[nt], a1[0], a1[1], a1[2], a1[3], bh[nt][0], bh[nt][1]);
     }
 }
 
-// acc (16 x D) += A(16 x 64, given as bf16 fragments per 16-column step) * tile (64 x D).
-template <int D>
-__device__ __forceinline__ void mma_p_tile(float (&acc)[D / 8][4], const uint32_t (&pa)[4][4], uint32_t btile, int lane) {
+// acc (16 x D) += A(16 x 16KS, given as bf16 fragments per 16-column step) * tile (16KS x D).
+template <int D, int KS>
+__device__ __forceinline__ void mma_p_tile(float (&acc)[D / 8][4], const uint32_t (&pa)[KS][4], uint32_t btile, int lane) {
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
+    for (int ks = 0; ks < KS; ++ks) {
 #pragma unroll
         for (int nd = 0; nd < D / 8; nd += 2) {
             uint32_t b0, b1, b2, b3;
@@ -138,10 +138,12 @@ __device__ __forceinline__ void mma_p_tile(float (&acc)[D / 8][4], const uint32_
     }
 }
 
-// Round 16 x 64 fp32 accumulators (8 column blocks of 8) to the bf16 A fragments of 4 k steps.
-__device__ __forceinline__ void to_afrag(const float (&x)[8][4], uint32_t (&pa)[4][4]) {
+// Round 16 x 8NTB fp32 accumulators (NTB column blocks of 8) to the bf16 A fragments of NTB/2
+// k steps.
+template <int NTB>
+__device__ __forceinline__ void to_afrag(const float (&x)[NTB][4], uint32_t (&pa)[NTB / 2][4]) {
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
+    for (int ks = 0; ks < NTB / 2; ++ks) {
         pa[ks][0] = pack_bf16x2(x[2 * ks][0], x[2 * ks][1]);
         pa[ks][1] = pack_bf16x2(x[2 * ks][2], x[2 * ks][3]);
         pa[ks][2] = pack_bf16x2(x[2 * ks + 1][0], x[2 * ks + 1][1]);
@@ -151,11 +153,17 @@ __device__ __forceinline__ void to_afrag(const float (&x)[8][4], uint32_t (&pa)[
 
 template <int D, bool ROPE>
 struct BmCfg {
-    static constexpr int TILE = kBmTile * D * 2;                 // bytes of one 64-row bf16 tile
-    static constexpr int NT = ROPE ? 3 : 2;                       // streamed tiles per step (K,Kl,V / Q,Ql,dO)
-    static constexpr int STEP = NT * TILE + 2 * kBmTile * 4;      // + lse and D rows (dkdv)
+    // streamed rows per step: 32 at D=128 keeps the 16 x TT score fragments and the two 16 x D
+    // gradient accumulators of the dk/dv kernel inside the register file
+    static constexpr int TT = (D == 128) ? 32 : kBmTile;
+    static constexpr int NTB = TT / 8;                            // 8-column blocks of a score tile
+    static constexpr int KS = TT / 16;                            // 16-row k steps of a P/dS product
+    static constexpr int FIX = kBmRows * D * 2;                   // bytes of a 64-row bf16 tile
+    static constexpr int STR = TT * D * 2;                        // bytes of a streamed tile
+    static constexpr int NT = ROPE ? 3 : 2;                       // tiles per kind (K,Kl,V / Q,Ql,dO)
+    static constexpr int STEP = NT * STR + 2 * TT * 4;            // + lse and D rows (dkdv)
     // fixed: Q, Ql, dO (dq) or K, Kl, V (dkdv); two buffers of the streamed step
-    static constexpr int SMEM = NT * TILE + 2 * STEP + 128;
+    static constexpr int SMEM = NT * FIX + 2 * STEP + 128;
 };
 
 // dQ: CTA (64 query rows, q head h, batch b).
@@ -164,10 +172,10 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dq
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
     const uint32_t base = smem_u32(bm_smem);
-    const uint32_t uQ = base, uQl = base + C::TILE, uG = base + (C::NT - 1) * C::TILE;
-    auto uK = [&](int buf) { return base + C::NT * C::TILE + buf * C::STEP; };
-    auto uKl = [&](int buf) { return uK(buf) + C::TILE; };
-    auto uV = [&](int buf) { return uK(buf) + (C::NT - 1) * C::TILE; };
+    const uint32_t uQ = base, uQl = base + C::FIX, uG = base + (C::NT - 1) * C::FIX;
+    auto uK = [&](int buf) { return base + C::NT * C::FIX + buf * C::STEP; };
+    auto uKl = [&](int buf) { return uK(buf) + C::STR; };
+    auto uV = [&](int buf) { return uK(buf) + (C::NT - 1) * C::STR; };
     const int h = blockIdx.y, b = blockIdx.z;
     const int kvh = h / (p.Hq / p.Hkv);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -181,18 +189,18 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dq
     const long last_row = static_cast<long>(i0) + kBmRows - 1;
     long kmax = p.causal ? last_row + off_c + 1 : p.Skv;
     kmax = kmax < 0 ? 0 : (kmax > p.Skv ? p.Skv : kmax);
-    const int nsteps = static_cast<int>((kmax + kBmTile - 1) / kBmTile);
+    const int nsteps = static_cast<int>((kmax + C::TT - 1) / C::TT);
     auto issue_step = [&](int t) {
-        const long k0 = static_cast<long>(t) * kBmTile;
+        const long k0 = static_cast<long>(t) * C::TT;
         const long kbase = ((static_cast<long>(b) * p.Skv + k0) * p.Hkv + kvh) * D;
-        const int kvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Skv - k0));
-        stage_rows_async<D>(uK(t & 1), p.k + kbase, kstride, kvalid);
-        if (ROPE) stage_rows_async<D>(uKl(t & 1), p.kl + kbase, kstride, kvalid);
-        stage_rows_async<D>(uV(t & 1), p.v + kbase, kstride, kvalid);
+        const int kvalid = static_cast<int>(min(static_cast<long>(C::TT), p.Skv - k0));
+        stage_rows_async<D, C::TT>(uK(t & 1), p.k + kbase, kstride, kvalid);
+        if (ROPE) stage_rows_async<D, C::TT>(uKl(t & 1), p.kl + kbase, kstride, kvalid);
+        stage_rows_async<D, C::TT>(uV(t & 1), p.v + kbase, kstride, kvalid);
     };
-    stage_rows_async<D>(uQ, p.q + qbase, qstride, qvalid);
-    if (ROPE) stage_rows_async<D>(uQl, p.ql + qbase, qstride, qvalid);
-    stage_rows_async<D>(uG, p.dout + qbase, qstride, qvalid);
+    stage_rows_async<D, kBmRows>(uQ, p.q + qbase, qstride, qvalid);
+    if (ROPE) stage_rows_async<D, kBmRows>(uQl, p.ql + qbase, qstride, qvalid);
+    stage_rows_async<D, kBmRows>(uG, p.dout + qbase, qstride, qvalid);
     if (nsteps > 0) issue_step(0);
     cp_async_commit();
     // this thread's two rows: r_a = warp*16 + g, r_b = r_a + 8
@@ -223,22 +231,22 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dq
         cp_async_commit();
         cp_async_wait<1>();
         __syncthreads();
-        const long k0 = static_cast<long>(t) * kBmTile;
+        const long k0 = static_cast<long>(t) * C::TT;
         const int buf = t & 1;
-        float s[8][4], dp[8][4];
+        float s[C::NTB][4], dp[C::NTB][4];
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < C::NTB; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
-        mma_rows_t<D>(s, uQ, warp * 16, uK(buf), lane);
+        mma_rows_t<D, C::NTB>(s, uQ, warp * 16, uK(buf), lane);
         if (ROPE) {
-            mma_rows_t<D>(s, uQ, warp * 16, uKl(buf), lane);
-            mma_rows_t<D>(s, uQl, warp * 16, uK(buf), lane);
+            mma_rows_t<D, C::NTB>(s, uQ, warp * 16, uKl(buf), lane);
+            mma_rows_t<D, C::NTB>(s, uQl, warp * 16, uK(buf), lane);
         }
-        mma_rows_t<D>(dp, uG, warp * 16, uV(buf), lane);
+        mma_rows_t<D, C::NTB>(dp, uG, warp * 16, uV(buf), lane);
         // dS * scale in place of s
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < C::NTB; ++nt) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const long key = k0 + nt * 8 + 2 * t4 + (e & 1);
@@ -252,9 +260,9 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dq
                 s[nt][e] = pr * (dp[nt][e] - (top ? d_a : d_b)) * p.scale;
             }
         }
-        uint32_t pa[4][4];
-        to_afrag(s, pa);
-        mma_p_tile<D>(dq, pa, uK(buf), lane);
+        uint32_t pa[C::KS][4];
+        to_afrag<C::NTB>(s, pa);
+        mma_p_tile<D, C::KS>(dq, pa, uK(buf), lane);
         __syncthreads();   // buffer buf is refilled by the step after next
     }
     cp_async_wait<0>();
@@ -272,11 +280,11 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dk
     using C = BmCfg<D, ROPE>;
     extern __shared__ __align__(128) uint8_t bm_smem[];
     const uint32_t base = smem_u32(bm_smem);
-    const uint32_t uK = base, uKl = base + C::TILE, uV = base + (C::NT - 1) * C::TILE;
-    auto uQ = [&](int buf) { return base + C::NT * C::TILE + buf * C::STEP; };
-    auto uQl = [&](int buf) { return uQ(buf) + C::TILE; };
-    auto uG = [&](int buf) { return uQ(buf) + (C::NT - 1) * C::TILE; };
-    auto sLrow = [&](int buf) { return reinterpret_cast<float*>(bm_smem + C::NT * C::TILE + buf * C::STEP + C::NT * C::TILE); };
+    const uint32_t uK = base, uKl = base + C::FIX, uV = base + (C::NT - 1) * C::FIX;
+    auto uQ = [&](int buf) { return base + C::NT * C::FIX + buf * C::STEP; };
+    auto uQl = [&](int buf) { return uQ(buf) + C::STR; };
+    auto uG = [&](int buf) { return uQ(buf) + (C::NT - 1) * C::STR; };
+    auto sLrow = [&](int buf) { return reinterpret_cast<float*>(bm_smem + C::NT * C::FIX + buf * C::STEP + C::NT * C::STR); };
     const int kvh = blockIdx.y, b = blockIdx.z;
     const int G = p.Hq / p.Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -288,31 +296,31 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dk
     const long off_c = static_cast<long>(p.Skv) - p.Sq;
     long i_lo = p.causal ? static_cast<long>(j0) - off_c : 0;
     i_lo = i_lo < 0 ? 0 : i_lo;
-    const int t_start = static_cast<int>(i_lo / kBmTile);
-    const int t_per_head = (p.Sq + kBmTile - 1) / kBmTile - t_start;   // query tiles per q head
+    const int t_start = static_cast<int>(i_lo / C::TT);
+    const int t_per_head = (p.Sq + C::TT - 1) / C::TT - t_start;   // query tiles per q head
     const int nsteps = t_per_head > 0 ? t_per_head * G : 0;
     // step -> (group head, query tile); lse and D rows land after the step's tiles
     auto issue_step = [&](int t) {
         const int hg = t / t_per_head;
-        const long i0 = static_cast<long>(t_start + t % t_per_head) * kBmTile;
+        const long i0 = static_cast<long>(t_start + t % t_per_head) * C::TT;
         const int h = kvh * G + hg;
         const long qbase = ((static_cast<long>(b) * p.Sq + i0) * p.Hq + h) * D;
-        const int qvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Sq - i0));
-        stage_rows_async<D>(uQ(t & 1), p.q + qbase, qstride, qvalid);
-        if (ROPE) stage_rows_async<D>(uQl(t & 1), p.ql + qbase, qstride, qvalid);
-        stage_rows_async<D>(uG(t & 1), p.dout + qbase, qstride, qvalid);
+        const int qvalid = static_cast<int>(min(static_cast<long>(C::TT), p.Sq - i0));
+        stage_rows_async<D, C::TT>(uQ(t & 1), p.q + qbase, qstride, qvalid);
+        if (ROPE) stage_rows_async<D, C::TT>(uQl(t & 1), p.ql + qbase, qstride, qvalid);
+        stage_rows_async<D, C::TT>(uG(t & 1), p.dout + qbase, qstride, qvalid);
         const uint32_t dl = smem_u32(sLrow(t & 1));
         const long srow0 = (static_cast<long>(b) * p.Hq + h) * p.Sq + i0;
-        for (int w = threadIdx.x; w < 2 * kBmTile; w += kBmThreads) {
-            const int r = w % kBmTile;
+        for (int w = threadIdx.x; w < 2 * C::TT; w += kBmThreads) {
+            const int r = w % C::TT;
             const bool ok = r < qvalid;
-            const float* src = (w < kBmTile ? p.lse : p.Dvec) + srow0 + (ok ? r : 0);
+            const float* src = (w < C::TT ? p.lse : p.Dvec) + srow0 + (ok ? r : 0);
             cp_async4(dl + w * 4, src, ok);
         }
     };
-    stage_rows_async<D>(uK, p.k + kbase, kstride, kvalid);
-    if (ROPE) stage_rows_async<D>(uKl, p.kl + kbase, kstride, kvalid);
-    stage_rows_async<D>(uV, p.v + kbase, kstride, kvalid);
+    stage_rows_async<D, kBmRows>(uK, p.k + kbase, kstride, kvalid);
+    if (ROPE) stage_rows_async<D, kBmRows>(uKl, p.kl + kbase, kstride, kvalid);
+    stage_rows_async<D, kBmRows>(uV, p.v + kbase, kstride, kvalid);
     if (nsteps > 0) issue_step(0);
     cp_async_commit();
     const int ja = j0 + warp * 16 + g, jb = ja + 8;    // this thread's two keys
@@ -328,24 +336,24 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dk
         cp_async_wait<1>();
         __syncthreads();
         const int buf = t & 1;
-        const long i0 = static_cast<long>(t_start + t % t_per_head) * kBmTile;
-        const int qvalid = static_cast<int>(min(static_cast<long>(kBmTile), p.Sq - i0));
+        const long i0 = static_cast<long>(t_start + t % t_per_head) * C::TT;
+        const int qvalid = static_cast<int>(min(static_cast<long>(C::TT), p.Sq - i0));
         const float* sL = sLrow(buf);
-        const float* sD = sL + kBmTile;
-        float s[8][4], dp[8][4];
+        const float* sD = sL + C::TT;
+        float s[C::NTB][4], dp[C::NTB][4];
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
+        for (int nt = 0; nt < C::NTB; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) s[nt][e] = dp[nt][e] = 0.f;
-        mma_rows_t<D>(s, uK, warp * 16, uQ(buf), lane);        // S^T = K Q^T
+        mma_rows_t<D, C::NTB>(s, uK, warp * 16, uQ(buf), lane);        // S^T = K Q^T
         if (ROPE) {
-            mma_rows_t<D>(s, uK, warp * 16, uQl(buf), lane);
-            mma_rows_t<D>(s, uKl, warp * 16, uQ(buf), lane);
+            mma_rows_t<D, C::NTB>(s, uK, warp * 16, uQl(buf), lane);
+            mma_rows_t<D, C::NTB>(s, uKl, warp * 16, uQ(buf), lane);
         }
-        mma_rows_t<D>(dp, uV, warp * 16, uG(buf), lane);       // dP^T = V dO^T
+        mma_rows_t<D, C::NTB>(dp, uV, warp * 16, uG(buf), lane);       // dP^T = V dO^T
         // s <- P^T, dp <- dS^T * scale
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int nt = 0; nt < C::NTB; ++nt) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int qi = nt * 8 + 2 * t4 + (e & 1);   // query row within the tile
@@ -362,11 +370,11 @@ __global__ void __launch_bounds__(kBmThreads, (D == 64 && !ROPE) ? 3 : 1) bwd_dk
                 s[nt][e] = pr;
             }
         }
-        uint32_t pa[4][4];
-        to_afrag(s, pa);
-        mma_p_tile<D>(dv, pa, uG(buf), lane);                   // dV += P^T dO
-        to_afrag(dp, pa);
-        mma_p_tile<D>(dk, pa, uQ(buf), lane);                   // dK += dS^T Q
+        uint32_t pa[C::KS][4];
+        to_afrag<C::NTB>(s, pa);
+        mma_p_tile<D, C::KS>(dv, pa, uG(buf), lane);                   // dV += P^T dO
+        to_afrag<C::NTB>(dp, pa);
+        mma_p_tile<D, C::KS>(dk, pa, uQ(buf), lane);                   // dK += dS^T Q
         __syncthreads();   // buffer buf is refilled by the step after next
     }
     cp_async_wait<0>();
