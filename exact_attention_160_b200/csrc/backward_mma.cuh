@@ -20,7 +20,7 @@ namespace attn {
 
 constexpr int kBmThreads = 128;   // 4 warps x 16 rows = 64 rows per CTA
 constexpr int kBmRows = 64;
-constexpr int kBmTile = 64;       // keys (dq) / query rows (dkdv) per step at D=64 (32 at D=128)
+constexpr int kBmTile = 64;       // keys (dq) / query rows (dkdv) per step
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Byte offset of 16-byte chunk ch (8 bf16) of row r in a tile of rows of D bf16, with the low
@@ -153,9 +153,9 @@ __device__ __forceinline__ void to_afrag(const float (&x)[NTB][4], uint32_t (&pa
 
 template <int D, bool ROPE>
 struct BmCfg {
-    // streamed rows per step: 32 at D=128 keeps the 16 x TT score fragments and the two 16 x D
-    // gradient accumulators of the dk/dv kernel inside the register file
-    static constexpr int TT = (D == 128) ? 32 : kBmTile;
+    // streamed rows per step (32 at D=128 removes the dk/dv kernel's register spills but costs
+    // more in extra steps than it saves: 14.3 ms against 12.9 ms on a D=128, S=16384 backward)
+    static constexpr int TT = kBmTile;
     static constexpr int NTB = TT / 8;                            // 8-column blocks of a score tile
     static constexpr int KS = TT / 16;                            // 16-row k steps of a P/dS product
     static constexpr int FIX = kBmRows * D * 2;                   // bytes of a 64-row bf16 tile
