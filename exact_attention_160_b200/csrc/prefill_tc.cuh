@@ -11,9 +11,11 @@
 // B200 design (not the pages' CPU loop structure):
 //   * One CTA holds two 128-row query tiles that read the same K/V: two q heads of one GQA group
 //     at the same rows when the group size is even, else two consecutive row tiles of one head.
-//     Each K/V tile is therefore loaded once for 256 query rows.
+//     Each K/V tile is therefore loaded once for 256 query rows.  A problem small enough that its
+//     single tiles fit in one wave of the SMs runs one tile per CTA (the second tile inactive).
 //   * Warp roles (3 warpgroups): warp 0 issues TMA loads (Q once, then a ring of K/V stages);
-//     warp 1 owns tensor memory and issues every tcgen05.mma from one thread; warps 4-7 and
+//     warp 1 owns tensor memory; warps 1 and 2 issue the tcgen05.mma of query tile 0 and 1, one
+//     thread each, from precomputed shared-memory descriptors; warps 4-7 and
 //     8-11 are the softmax warpgroups of query tile 0 and 1, one thread per query row (a warp
 //     may only touch TMEM lanes 32*(warp%4) .. +31, so the row of a softmax thread is
 //     32*(warp%4) + lane).
@@ -30,6 +32,9 @@
 //     makes rows with no visible key yet contribute nothing.
 //   * With RoPE, Q is rotated in shared memory right after its TMA load and K arrives
 //     pre-rotated; both carry hi + lo bf16 halves and S = Qh Kh^T + Qh Kl^T + Ql Kh^T.
+//   * MASK instantiations add an additive score mask (whisper-apr attention_generated.rs,
+//     compute_block_scores: score = dot * scale + mask) to the row of S in registers, as
+//     mask / scale on the unscaled dot products, before the row max.
 //
 // TMEM columns (512 allocated): S0 [0,128) S1 [128,256) O0, O1 (D each) after them; with D=64
 // P0 and P1 get their own 64 columns, with D=128 P_i overwrites the first 64 columns of S_i
