@@ -8,6 +8,8 @@
 #include <string.h>
 
 #include <mutex>
+#include <set>
+#include <utility>
 
 #include "../../include/attn_b200.h"
 #include "common.cuh"
@@ -87,6 +89,36 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 attn_status launch_status(const char* what) {
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? ATTN_OK : cuda_failure(what, cudaGetErrorString(e));
+}
+
+// Kernel attributes belong to the kernel's image on one device, so each (device, kernel) pair
+// is configured once, on its first launch from that device.  With min_regs > 0 the kernel is
+// first checked to be compiled with at least that many registers per thread.
+std::mutex g_attr_mu;
+std::set<std::pair<int, const void*>> g_attr_done;
+
+attn_status prepare_kernel(const void* fn, int smem_bytes, const char* name, int min_regs = 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_failure("cudaGetDevice", cudaGetErrorString(e));
+    const std::pair<int, const void*> key(dev, fn);
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (g_attr_done.count(key) != 0) return ATTN_OK;
+    if (min_regs > 0) {
+        cudaFuncAttributes fa;
+        e = cudaFuncGetAttributes(&fa, fn);
+        if (e != cudaSuccess) return cuda_failure(name, cudaGetErrorString(e));
+        if (fa.numRegs < min_regs) {
+            char buf[96];
+            snprintf(buf, sizeof(buf), "compiled with %d registers per thread, needs %d", fa.numRegs, min_regs);
+            cuda_failure(name, buf);
+            return ATTN_ERR_UNSUPPORTED;
+        }
+    }
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e != cudaSuccess) return cuda_failure(name, cudaGetErrorString(e));
+    g_attr_done.insert(key);
+    return ATTN_OK;
 }
 
 attn_status check_common(int B, int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal) {
@@ -186,24 +218,11 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     if (grid > 2147483647L) return ATTN_ERR_UNSUPPORTED;
     // the masked kernel is a separate instantiation, so the unmasked one carries no mask code
     auto kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true> : prefill_tc_kernel<D, ROPE, false>;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[mk.ptr != nullptr]) {
-        // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds
-        // fewer than the split asks for would stall in setmaxnreg.inc, so refuse it.
-        cudaFuncAttributes fa;
-        cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-        if (e != cudaSuccess) return cuda_failure("cudaFuncGetAttributes(prefill_tc_kernel)", cudaGetErrorString(e));
-        if (fa.numRegs < kTcLaunchRegsMin) {
-            char buf[96];
-            snprintf(buf, sizeof(buf), "compiled with %d registers per thread, the warpgroup split needs %d",
-                     fa.numRegs, kTcLaunchRegsMin);
-            cuda_failure("prefill_tc_kernel register budget", buf);
-            return ATTN_ERR_UNSUPPORTED;
-        }
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(prefill_tc_kernel)", cudaGetErrorString(e));
-        attr_set[mk.ptr != nullptr] = true;
-    }
+    // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds fewer
+    // than the split asks for would stall in setmaxnreg.inc, so such a build is refused.
+    attn_status ps = prepare_kernel(reinterpret_cast<const void*>(kern), C::SMEM_BYTES, "prefill_tc_kernel set-up",
+                                    kTcLaunchRegsMin);
+    if (ps != ATTN_OK) return ps;
     kern<<<static_cast<unsigned>(grid), kTcThreads, C::SMEM_BYTES, st>>>(tq, tk, tkl, tv, p);
     return launch_status("prefill_tc_kernel");
 }
@@ -214,12 +233,9 @@ attn_status launch_f32(const void* q, const void* k, const void* v, void* o, flo
                        MaskArg mk) {
     const size_t smem = 2 * 64 * D * sizeof(float);
     auto kern = prefill_f32_kernel<D>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(prefill_f32_kernel)", cudaGetErrorString(e));
-        attr_set = true;
-    }
+    const attn_status ps = prepare_kernel(reinterpret_cast<const void*>(kern), static_cast<int>(smem),
+                                          "cudaFuncSetAttribute(prefill_f32_kernel)");
+    if (ps != ATTN_OK) return ps;
     dim3 grid((Sq + 63) / 64, Hq, B);
     if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
     kern<<<grid, 256, smem, st>>>(static_cast<const float*>(q), static_cast<const float*>(k),
@@ -294,12 +310,9 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
     dim3 grid(num_splits, Hkv * (G / GC), B);
     if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
     auto kern = decode_split_kernel<D>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(decode_split_kernel)", cudaGetErrorString(e));
-        attr_set = true;
-    }
+    const attn_status ps = prepare_kernel(reinterpret_cast<const void*>(kern), C::SMEM_BYTES,
+                                          "cudaFuncSetAttribute(decode_split_kernel)");
+    if (ps != ATTN_OK) return ps;
     kern<<<grid, kDecodeThreads, C::SMEM_BYTES, st>>>(tk, tv, static_cast<const __nv_bfloat16*>(q), seqlens, o_part,
                                                       lse_part, Hkv, G, GC, Smax, num_splits,
                                                       scale * 1.4426950408889634f);
@@ -433,16 +446,12 @@ attn_status launch_bwd(const T* q, const T* k, const T* v, const T* o, const flo
     p.mask_hs = mk.hs;
     const size_t smem_dq = 2 * kBwdTile * D * sizeof(float);
     const size_t smem_dkdv = (2 * kBwdTile * D + 2 * kBwdTile) * sizeof(float);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem_dq));
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(smem_dkdv));
-        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(bwd kernels)", cudaGetErrorString(e));
-        attr_set = true;
-    }
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(bwd_dq_kernel<D>), static_cast<int>(smem_dq),
+                            "cudaFuncSetAttribute(bwd_dq_kernel)")) != ATTN_OK)
+        return s;
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(bwd_dkdv_kernel<D>), static_cast<int>(smem_dkdv),
+                            "cudaFuncSetAttribute(bwd_dkdv_kernel)")) != ATTN_OK)
+        return s;
     p.g_f32 = g_f32 ? static_cast<float*>(dq) : nullptr;
     p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq);
     bwd_dq_kernel<D><<<dim3((Sq + kBwdRows - 1) / kBwdRows, Hq, B), kBwdThreads, smem_dq, st>>>(p);
@@ -528,13 +537,12 @@ attn_status launch_bwd_mma(const __nv_bfloat16* q, const __nv_bfloat16* k, const
     const bool masked = mk.ptr != nullptr;   // separate instantiations: the unmasked ones carry no mask code
     auto kdq = masked ? bwd_dq_mma_kernel<D, ROPE, true> : bwd_dq_mma_kernel<D, ROPE, false>;
     auto kkv = masked ? bwd_dkdv_mma_kernel<D, ROPE, true> : bwd_dkdv_mma_kernel<D, ROPE, false>;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[masked]) {
-        cudaError_t e = cudaFuncSetAttribute(kdq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e == cudaSuccess) e = cudaFuncSetAttribute(kkv, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-        if (e != cudaSuccess) return cuda_failure("cudaFuncSetAttribute(bwd mma kernels)", cudaGetErrorString(e));
-        attr_set[masked] = true;
-    }
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(kdq), C::SMEM, "cudaFuncSetAttribute(bwd_dq_mma_kernel)")) !=
+        ATTN_OK)
+        return s;
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(kkv), C::SMEM,
+                            "cudaFuncSetAttribute(bwd_dkdv_mma_kernel)")) != ATTN_OK)
+        return s;
     p.g_f32 = g_f32 ? static_cast<float*>(dq) : nullptr;
     p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq);
     kdq<<<dim3((Sq + kBmRows - 1) / kBmRows, Hq, B), kBmThreads, C::SMEM, st>>>(p);
