@@ -290,15 +290,18 @@ def bench_prefill_gpu(w: si.Prefill, args, torch, ea, dist, device):
     # bf16 inputs, fp32 accumulation, O taken in fp32: the configuration the parity tests check
     o = torch.empty(q.shape, dtype=torch.float32, device=device)
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=device)
-    ws = None
-    if w.rope_base > 0:
-        ws = torch.empty(ea.fwd_workspace_bytes(q, k, w.rope_base, w.q_pos0), dtype=torch.uint8, device=device)
+    # the workspace (RoPE table and rotated K, key-split partials) is allocated once, outside the
+    # timed region
+    ws_bytes = ea.fwd_workspace_bytes(q, k, w.rope_base, w.q_pos0, o.dtype)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device) if ws_bytes > 0 else None
+    splits = ea.fwd_kv_splits(q, k, o.dtype)
     flush = make_l2_flush(torch, device)
 
     def step():
         ea.attn_fwd_ex(q, k, v, w.scale, w.causal, w.rope_base, w.q_pos0, o=o, lse=lse, workspace=ws)
 
-    launches_per_step = 1 if w.rope_base <= 0 else 3
+    # rope: table + rotated K + prefill; key splits add the combine
+    launches_per_step = (1 if w.rope_base <= 0 else 3) + (1 if splits > 1 else 0)
     with ClockSampler(device.index) as clk:
         ms = time_steps(step, args.steps, args.warmup, flush, torch, dist, device)
     status = ea.read_device_status()
@@ -317,7 +320,7 @@ def bench_prefill_gpu(w: si.Prefill, args, torch, ea, dist, device):
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
     d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
     return {"ms": mean_ms, "ms_list": ms, "clocks": clk.summary(), "ms_e2e": ms_e2e,
-            "h2d": h2d, "d2h": d2h, "launches_per_step": launches_per_step}
+            "h2d": h2d, "d2h": d2h, "launches_per_step": launches_per_step, "kv_splits": splits}
 
 
 def bench_decode_gpu(w: si.Decode, args, torch, ea, dist, device, steps=None):
@@ -487,6 +490,7 @@ def run_gpu(args):
         launches = r["launches_per_step"] * args.steps
         config = {"workload": w.name, "global_batch": w.B * world, "seq_len": w.Sq, "heads_q": w.Hq,
                   "heads_kv": w.Hkv, "head_dim": w.D, "causal": w.causal, "rope_base": w.rope_base,
+                  "kv_splits": r["kv_splits"],
                   "parallelism": f"replicas{world}", "l2": L2_NOTE,
                   "inputs": "seeded synthetic N(0,1) rounded to bf16 (seeded_inputs)"}
     else:

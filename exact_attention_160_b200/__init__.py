@@ -32,7 +32,8 @@ STATUS = {0: "ok", 1: "invalid argument", 2: "dimension mismatch", 3: "empty KV"
 EXPORTS = ("attn_fwd", "attn_fwd_ex", "attn_fwd_ex_workspace_size", "attn_decode",
            "attn_decode_workspace_size", "attn_decode_noalloc", "rope_apply", "attn_status_string",
            "attn_last_error", "attn_selftest_wait_timeout", "attn_read_device_status", "attn_kv_append",
-           "attn_bwd", "attn_bwd_workspace_size", "attn_fwd_masked", "attn_bwd_masked")
+           "attn_bwd", "attn_bwd_workspace_size", "attn_fwd_masked", "attn_bwd_masked",
+           "attn_fwd_kv_splits")
 
 _lib = None
 
@@ -59,6 +60,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_fwd_ex.argtypes = [P, P, P, P, P, I, I, I, I, I, I, F, I, I, F, I, P, Z, P]
     lib.attn_fwd_ex_workspace_size.argtypes = [I, I, I, I, I, I, I, F, I]
     lib.attn_fwd_ex_workspace_size.restype = Z
+    lib.attn_fwd_kv_splits.argtypes = [I, I, I, I, I]
+    lib.attn_fwd_kv_splits.restype = I
     lib.attn_decode.argtypes = [P, P, P, P, P, P, I, I, I, I, I, F, I, P, Z, I, P]
     lib.attn_decode_workspace_size.argtypes = [I, I, I, I]
     lib.attn_decode_workspace_size.restype = Z
@@ -125,25 +128,38 @@ def _need_cuda(*ts):
 
 
 def attn_fwd(q, k, v, scale: float, causal: bool, o=None, lse=None, want_lse: bool = True, out_dtype=None,
-             stream=None):
+             stream=None, kv_split: bool = True):
     """Exact attention forward.  Returns (o, lse); lse is None when want_lse is False.
-    out_dtype: torch.float32 to take a bf16 problem's output in fp32 (default: q's dtype)."""
+    out_dtype: torch.float32 to take a bf16 problem's output in fp32 (default: q's dtype).
+    kv_split=False runs a small problem unsplit (the C attn_fwd, no workspace)."""
     return attn_fwd_ex(q, k, v, scale, causal, 0.0, 0, o=o, lse=lse, want_lse=want_lse, out_dtype=out_dtype,
-                       stream=stream)
+                       stream=stream, kv_split=kv_split)
+
+
+def fwd_kv_splits(q, k, out_dtype=None) -> int:
+    """Key splits attn_fwd_ex uses for these shapes when it has its workspace (1: unsplit)."""
+    lib = load_library()
+    B, Sq, Hq, _ = q.shape
+    return int(lib.attn_fwd_kv_splits(B, Hq, Sq, k.shape[1], _out_code(q, out_dtype)))
+
+
+def _out_code(q, out_dtype):
+    return _dtype_code(q) if out_dtype is None or q.dtype != torch.bfloat16 else (
+        ATTN_BF16_OUT_F32 if out_dtype == torch.float32 else ATTN_BF16)
 
 
 def fwd_workspace_bytes(q, k, rope_base: float, q_pos0: int, out_dtype=None) -> int:
     lib = load_library()
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
-    code = _dtype_code(q) if out_dtype is None or q.dtype != torch.bfloat16 else (
-        ATTN_BF16_OUT_F32 if out_dtype == torch.float32 else ATTN_BF16)
-    return int(lib.attn_fwd_ex_workspace_size(B, Hq, Hkv, Sq, Skv, D, code, float(rope_base), int(q_pos0)))
+    return int(lib.attn_fwd_ex_workspace_size(B, Hq, Hkv, Sq, Skv, D, _out_code(q, out_dtype), float(rope_base),
+                                              int(q_pos0)))
 
 
 def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: int = 0, o=None, lse=None,
-                want_lse: bool = True, workspace=None, out_dtype=None, stream=None):
-    """Exact attention forward with RoPE on Q (positions q_pos0 + i) and K (positions j)."""
+                want_lse: bool = True, workspace=None, out_dtype=None, stream=None, kv_split: bool = True):
+    """Exact attention forward with RoPE on Q (positions q_pos0 + i) and K (positions j).
+    kv_split=False (without RoPE, D 64 or 128) calls the C attn_fwd: no workspace, no key splits."""
     lib = load_library()
     _need_cuda(q, k, v, o, lse, workspace)
     B, Sq, Hq, D = q.shape
@@ -153,7 +169,10 @@ def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: i
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
     ws_bytes = 0
-    need = fwd_workspace_bytes(q, k, rope_base, q_pos0, o.dtype)
+    if not kv_split and rope_base <= 0 and D in (64, 128):
+        need, workspace = 0, None
+    else:
+        need = fwd_workspace_bytes(q, k, rope_base, q_pos0, o.dtype)
     if need > 0 or workspace is not None:
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

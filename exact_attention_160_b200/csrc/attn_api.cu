@@ -161,28 +161,59 @@ struct MaskArg {
 };
 
 // Layout of the attn_fwd_ex workspace: rope table, then (bf16) rotated K as hi and lo halves.
+constexpr int kNumSms = 148;   // B200
+
+// Key splits of the tensor-core forward.  A bf16 problem whose query tiles fill at most half of
+// the SMs divides each tile's key tiles among up to kMaxKvSplits CTAs (at least two key tiles
+// each), so that the whole GPU works on it; the partials are merged by prefill_combine_kernel.
+// Depends on the sizes only, so the workspace query and the launch agree.
+int fwd_kv_splits(int B, int Hq, int Sq, int Skv, attn_dtype dtype) {
+    if (dtype == ATTN_FP32) return 1;
+    const long tiles = static_cast<long>((Sq + 127) / 128) * B * Hq;
+    if (tiles > kNumSms / 2) return 1;
+    long n = kNumSms / tiles;
+    const long nkv = (static_cast<long>(Skv) + 127) / 128;
+    if (n > nkv / 2) n = nkv / 2;
+    if (n > kMaxKvSplits) n = kMaxKvSplits;
+    return n >= 2 ? static_cast<int>(n) : 1;
+}
+
+// Workspace of attn_fwd_ex: with RoPE the cos/sin table and the rotated K as hi/lo bf16 halves;
+// with key splits the fp32 partial O and logsumexp of every split.
 struct ExWorkspace {
-    size_t tab_off, khi_off, klo_off, total;
+    size_t tab_off, khi_off, klo_off, opart_off, lpart_off, total;
     int positions;
+    int splits;
 };
 
-ExWorkspace ex_workspace(int B, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, int q_pos0) {
+ExWorkspace ex_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype, bool rope, int q_pos0) {
     ExWorkspace w{};
-    long pq = static_cast<long>(q_pos0) + Sq;
-    w.positions = static_cast<int>(pq > Skv ? pq : Skv);
-    w.tab_off = 0;
-    size_t tab = static_cast<size_t>(w.positions) * (D / 2) * sizeof(float2);
-    w.khi_off = round_up(tab, 256);
-    size_t kbytes = dtype != ATTN_FP32 ? static_cast<size_t>(B) * Skv * Hkv * D * 2 : 0;
-    w.klo_off = round_up(w.khi_off + kbytes, 256);
-    w.total = round_up(w.klo_off + kbytes, 256);
+    size_t end = 0;
+    if (rope) {
+        long pq = static_cast<long>(q_pos0) + Sq;
+        w.positions = static_cast<int>(pq > Skv ? pq : Skv);
+        w.tab_off = 0;
+        size_t tab = static_cast<size_t>(w.positions) * (D / 2) * sizeof(float2);
+        w.khi_off = round_up(tab, 256);
+        size_t kbytes = dtype != ATTN_FP32 ? static_cast<size_t>(B) * Skv * Hkv * D * 2 : 0;
+        w.klo_off = round_up(w.khi_off + kbytes, 256);
+        end = round_up(w.klo_off + kbytes, 256);
+    }
+    w.splits = fwd_kv_splits(B, Hq, Sq, Skv, dtype);
+    if (w.splits > 1) {
+        const size_t rows = static_cast<size_t>(B) * Sq * Hq;
+        w.opart_off = end;
+        w.lpart_off = round_up(w.opart_off + w.splits * rows * D * sizeof(float), 256);
+        end = round_up(w.lpart_off + w.splits * rows * sizeof(float), 256);
+    }
+    w.total = end;
     return w;
 }
 
 template <int D, bool ROPE>
 attn_status launch_tc(const void* q, const void* k, const void* klo, const void* v, void* o, bool o_f32, float* lse,
                       int B, int Hq, int Hkv, int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0,
-                      cudaStream_t st, MaskArg mk) {
+                      cudaStream_t st, MaskArg mk, int splits, float* o_part, float* lse_part) {
     CUtensorMap tq, tk, tkl, tv;
     if (!make_tmap_bshd(&tq, q, B, Sq, Hq, D) || !make_tmap_bshd(&tk, k, B, Skv, Hkv, D) ||
         !make_tmap_bshd(&tv, v, B, Skv, Hkv, D) || !make_tmap_bshd(&tkl, ROPE ? klo : k, B, Skv, Hkv, D))
@@ -214,7 +245,14 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     p.mask_bs = mk.bs;
     p.mask_hs = mk.hs;
     p.inv_scale = 1.f / scale;
-    const long grid = static_cast<long>(p.n_row_tiles) * B * p.heads_per_item;
+    p.kv_splits = 1;
+    if (splits > 1) {
+        if (!p.single_tile || splits > kMaxKvSplits || !o_part || !lse_part) return ATTN_ERR_UNSUPPORTED;
+        p.kv_splits = splits;
+        p.o_part = o_part;
+        p.lse_part = lse_part;
+    }
+    const long grid = static_cast<long>(p.n_row_tiles) * B * p.heads_per_item * p.kv_splits;
     if (grid > 2147483647L) return ATTN_ERR_UNSUPPORTED;
     // the masked kernel is a separate instantiation, so the unmasked one carries no mask code
     auto kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true> : prefill_tc_kernel<D, ROPE, false>;
@@ -224,7 +262,26 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
                                     kTcLaunchRegsMin);
     if (ps != ATTN_OK) return ps;
     kern<<<static_cast<unsigned>(grid), kTcThreads, C::SMEM_BYTES, st>>>(tq, tk, tkl, tv, p);
-    return launch_status("prefill_tc_kernel");
+    attn_status s = launch_status("prefill_tc_kernel");
+    if (s != ATTN_OK || p.kv_splits == 1) return s;
+    // merge of the key splits, a programmatic dependent launch (it waits for the split grid)
+    const long rows = static_cast<long>(B) * Sq * Hq;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((rows + kPcThreads / 32 - 1) / (kPcThreads / 32)));
+    cfg.blockDim = dim3(kPcThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, prefill_combine_kernel<D>, static_cast<const float*>(o_part),
+                                             static_cast<const float*>(lse_part),
+                                             o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
+                                             o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Sq, Hq, splits);
+    if (e != cudaSuccess) return cuda_failure("prefill_combine_kernel launch", cudaGetErrorString(e));
+    return launch_status("prefill_combine_kernel");
 }
 
 template <int D>
@@ -259,10 +316,15 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
     if (rope && (D % 2) != 0) return ATTN_ERR_DIM_MISMATCH;
 
     const float2* tab = nullptr;
-    ExWorkspace w{};
+    // The workspace is required with RoPE; without it, a caller's workspace (attn_fwd_ex) turns on
+    // the key splits of a small problem, and attn_fwd (none) runs it unsplit.
+    const ExWorkspace w = ex_workspace(B, Hq, Hkv, Sq, Skv, D, dtype, rope, q_pos0);
+    const int splits = (rope || workspace != nullptr) ? w.splits : 1;
+    if ((rope || splits > 1) && (!workspace || workspace_bytes < w.total || !aligned16(workspace)))
+        return ATTN_ERR_WORKSPACE;
+    float* o_part = splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.opart_off) : nullptr;
+    float* lse_part = splits > 1 ? reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.lpart_off) : nullptr;
     if (rope) {
-        w = ex_workspace(B, Hkv, Sq, Skv, D, dtype, q_pos0);
-        if (!workspace || workspace_bytes < w.total || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
         uint8_t* ws = static_cast<uint8_t*>(workspace);
         float2* t = reinterpret_cast<float2*>(ws + w.tab_off);
         const long n = static_cast<long>(w.positions) * (D / 2);
@@ -278,9 +340,9 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
     }
     if (!rope) {
         return D == 64 ? launch_tc<64, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
-                                              nullptr, 0, st, mk)
+                                              nullptr, 0, st, mk, splits, o_part, lse_part)
                        : launch_tc<128, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
-                                               nullptr, 0, st, mk);
+                                               nullptr, 0, st, mk, splits, o_part, lse_part);
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* khi = reinterpret_cast<uint32_t*>(ws + w.khi_off);
@@ -290,9 +352,9 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
                            0, st>>>(static_cast<const uint32_t*>(k), khi, klo, tab, npairs, Skv, Hkv, D);
     if ((s = launch_status("rope_split_kv_kernel")) != ATTN_OK) return s;
     return D == 64 ? launch_tc<64, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
-                                         q_pos0, st, mk)
+                                         q_pos0, st, mk, splits, o_part, lse_part)
                    : launch_tc<128, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
-                                          q_pos0, st, mk);
+                                          q_pos0, st, mk, splits, o_part, lse_part);
 }
 
 template <int D>
@@ -356,7 +418,7 @@ PadFwd pad_fwd_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dt
     w.v_off = round_up(w.k_off + ke * es_in, 256);
     w.o_off = round_up(w.v_off + ke * es_in, 256);
     w.inner_off = round_up(w.o_off + qe * es_out, 256);
-    w.total = w.inner_off + (rope_base > 0.f ? ex_workspace(B, Hkv, Sq, Skv, w.Dp, dtype, q_pos0).total : 0);
+    w.total = w.inner_off + ex_workspace(B, Hq, Hkv, Sq, Skv, w.Dp, dtype, rope_base > 0.f, q_pos0).total;
     return w;
 }
 
@@ -809,8 +871,12 @@ size_t attn_fwd_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D
                                   int q_pos0) {
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0 || q_pos0 < 0) return 0;
     if (!native_dim(D)) return paddable_dim(D) ? pad_fwd_workspace(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base, q_pos0).total : 0;
-    if (!(rope_base > 0.f)) return 0;
-    return ex_workspace(B, Hkv, Sq, Skv, D, dtype, q_pos0).total;
+    return ex_workspace(B, Hq, Hkv, Sq, Skv, D, dtype, rope_base > 0.f, q_pos0).total;
+}
+
+int attn_fwd_kv_splits(int B, int Hq, int Sq, int Skv, attn_dtype dtype) {
+    if (B <= 0 || Hq <= 0 || Sq <= 0 || Skv <= 0) return 1;
+    return fwd_kv_splits(B, Hq, Sq, Skv, dtype);
 }
 
 size_t attn_decode_workspace_size(int B, int Hq, int D, int num_splits) {

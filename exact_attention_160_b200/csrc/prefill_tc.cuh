@@ -101,6 +101,10 @@ struct TcParams {
     const float* mask;        // additive mask on the scaled scores, or null
     long mask_bs, mask_hs;    // its batch and head strides (elements; 0 broadcasts); rows of Skv
     float inv_scale;          // 1 / scale: the mask enters the raw scores as mask / scale
+    int kv_splits;            // >= 1; > 1 (single-tile mode only): each query tile's key tiles are
+                              // divided among this many CTAs, which write partials
+    float* o_part;            // [kv_splits][B][Sq][Hq][D] fp32 partial O, normalised per split
+    float* lse_part;          // [kv_splits][B][Hq][Sq] partial logsumexp (natural log)
 };
 
 struct TcTile {
@@ -147,9 +151,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const int warp = tid >> 5, lane = tid & 31;
 
     // ---- work item -> (batch, two query tiles) -------------------------------------------
+    // consecutive CTAs are the key splits of one work item (kv_splits == 1: one CTA per item)
+    const int split = static_cast<int>(blockIdx.x) % p.kv_splits;
+    const int item = static_cast<int>(blockIdx.x) / p.kv_splits;
     const int items_per_rowtile = p.B * p.heads_per_item;
-    const int rt = (p.n_row_tiles - 1) - static_cast<int>(blockIdx.x) / items_per_rowtile;   // heavy first
-    const int rem = static_cast<int>(blockIdx.x) % items_per_rowtile;
+    const int rt = (p.n_row_tiles - 1) - item / items_per_rowtile;   // heavy first
+    const int rem = item % items_per_rowtile;
     const int b = rem / p.heads_per_item;
     const int hi = rem % p.heads_per_item;
     TcTile tile[2];
@@ -170,6 +177,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     for (int i = 0; i < 2; ++i) {
         tile[i].active = tile[i].r0 < p.Sq;
         tile[i].nkv = tile[i].active ? tc_kv_tiles(p, tile[i].r0) : 0;
+    }
+    // Key split (single-tile mode): this CTA takes a contiguous chunk of the tile's key tiles,
+    // near-equal chunks with the remainder going to the first ones, and numbers them from 0 so
+    // that every pipeline phase below runs as for a whole tile; only the key coordinates move.
+    int kv0 = 0;
+    if (p.kv_splits > 1) {
+        const int n = tile[0].nkv, base = n / p.kv_splits, extra = n % p.kv_splits;
+        kv0 = split * base + min(split, extra);
+        tile[0].nkv = base + (split < extra ? 1 : 0);
     }
     const int kvh = tile[0].h / (p.Hq / p.Hkv);
     const int nkv = max(tile[0].nkv, tile[1].nkv);
@@ -239,16 +255,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 mbar_arrive_expect_tx(bar_k_full + s, C::K_TILES * C::TILE_BYTES);
                 for (int bx = 0; bx < C::NBOX; ++bx) {
                     tma_load_4d(&tm_k, bar_k_full + s, st + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
-                                j * 128, b, pol_kv);
+                                (kv0 + j) * 128, b, pol_kv);
                     if (ROPE)
                         tma_load_4d(&tm_klo, bar_k_full + s, st + C::TILE_BYTES + bx * (C::TILE_BYTES / C::NBOX),
-                                    bx * 64, kvh, j * 128, b, pol_kv);
+                                    bx * 64, kvh, (kv0 + j) * 128, b, pol_kv);
                 }
                 uint8_t* sv = st + C::K_TILES * C::TILE_BYTES;
                 mbar_arrive_expect_tx(bar_v_full + s, C::TILE_BYTES);
                 for (int bx = 0; bx < C::NBOX; ++bx)
                     tma_load_4d(&tm_v, bar_v_full + s, sv + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
-                                j * 128, b, pol_kv);
+                                (kv0 + j) * 128, b, pol_kv);
             }
             // no copy may still be landing in shared memory when the CTA exits
             mbar_wait(bar_q_full, 0);
@@ -441,7 +457,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 tc_fence_before();
                 mbar_arrive(bar_s_free + wg);
             }
-            const int k0 = j * 128;
+            const int k0 = (kv0 + j) * 128;
             if (MASK && qrow < p.Sq) {
                 // additive mask: S holds q.k unscaled, so add mask / scale; the exponent
                 // (s * scale + mask) * log2(e) - m then keeps its form
@@ -563,6 +579,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             }
             const bool store = qrow < p.Sq;
             const float inv = (have && l_mma > 0.f) ? 1.f / l_mma : 0.f;
+            // a key split writes its normalised partial O (fp32) and its logsumexp to its slabs
+            float* out_f32 = p.o_f32;
+            __nv_bfloat16* out_bf16 = p.o;
+            float* out_lse = p.lse;
+            if (p.kv_splits > 1) {
+                const long rows = static_cast<long>(p.B) * p.Sq * p.Hq;
+                out_f32 = p.o_part + split * rows * D;
+                out_bf16 = nullptr;
+                out_lse = p.lse_part + split * rows;
+            }
             const long orow_off = ((static_cast<long>(b) * p.Sq + qrow) * p.Hq + T.h) * D;
 #pragma unroll
             for (int cb = 0; cb < D / 32; ++cb) {
@@ -575,8 +601,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     for (int e = 0; e < 32; ++e) orr[e] = 0u;
                 }
                 if (!store) continue;
-                if (p.o_f32) {
-                    float4* dst = reinterpret_cast<float4*>(p.o_f32 + orow_off + cb * 32);
+                if (out_f32) {
+                    float4* dst = reinterpret_cast<float4*>(out_f32 + orow_off + cb * 32);
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
                         dst[e] = make_float4(__uint_as_float(orr[4 * e]) * inv, __uint_as_float(orr[4 * e + 1]) * inv,
@@ -586,14 +612,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
                         pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
-                    uint4* dst = reinterpret_cast<uint4*>(p.o + orow_off + cb * 32);
+                    uint4* dst = reinterpret_cast<uint4*>(out_bf16 + orow_off + cb * 32);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                 }
             }
-            if (store && p.lse != nullptr)
-                p.lse[(static_cast<long>(b) * p.Hq + T.h) * p.Sq + qrow] =
+            if (store && out_lse != nullptr)
+                out_lse[(static_cast<long>(b) * p.Hq + T.h) * p.Sq + qrow] =
                     (have && l_run > 0.f) ? (m_run + fast_log2(l_run)) * kLn2 : -INFINITY;
         }
     }
@@ -604,6 +630,74 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// Merge of a key-split forward: one warp per (b, query row, q head) combines the row's
+// kv_splits partials by their logsumexp, as the split-KV decode does (oxibonsai-model 0.1.4
+// src/layers/flash_decode.rs, combine_tile_outputs):  L = log sum_s e^(lse_s);
+// O = sum_s e^(lse_s - L) o_s.
+// Partials with lse_s = -inf (no visible key in that chunk) weigh nothing; a row with none at all
+// gets O = 0 and LSE = -inf.  Launched as a programmatic dependent of the split forward.
+constexpr int kPcThreads = 256;
+constexpr int kMaxKvSplits = 16;   // <= 32: one split per lane for the logsumexp reduction
+
+template <int D>
+__global__ void __launch_bounds__(kPcThreads) prefill_combine_kernel(
+    const float* __restrict__ o_part, const float* __restrict__ lse_part, __nv_bfloat16* __restrict__ o,
+    float* __restrict__ o_f32, float* __restrict__ lse, int B, int Sq, int Hq, int nsplit) {
+    constexpr int E = D / 32;   // output elements per lane
+    griddep_wait();
+    const long rows = static_cast<long>(B) * Sq * Hq;
+    const long r = static_cast<long>(blockIdx.x) * (kPcThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (r >= rows) return;   // whole warps leave together
+    const int h = static_cast<int>(r % Hq);
+    const long bq = r / Hq;
+    const int qi = static_cast<int>(bq % Sq);
+    const int b = static_cast<int>(bq / Sq);
+    const long lrow = (static_cast<long>(b) * Hq + h) * Sq + qi;
+    const float ls = lane < nsplit ? lse_part[lane * rows + lrow] : -INFINITY;
+    float M = ls;
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, w));
+    const float wt = (M == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - M);
+    float total = wt;
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) total += __shfl_xor_sync(0xffffffffu, total, w);
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) {
+        const float ws = __shfl_sync(0xffffffffu, wt, sp);
+        if (ws == 0.f) continue;   // the same for every lane
+        const float* src = o_part + (sp * rows + r) * D + lane * E;
+        float x[E];
+        if constexpr (E == 2) {
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            x[0] = v.x, x[1] = v.y;
+        } else {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            x[0] = v.x, x[1] = v.y, x[2] = v.z, x[3] = v.w;
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(ws, x[e], acc[e]);
+    }
+    const float inv = total > 0.f ? 1.f / total : 0.f;
+    const long dst = r * D + lane * E;
+    if constexpr (E == 2) {
+        if (o_f32 != nullptr)
+            *reinterpret_cast<float2*>(o_f32 + dst) = make_float2(acc[0] * inv, acc[1] * inv);
+        else
+            *reinterpret_cast<uint32_t*>(o + dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    } else {
+        if (o_f32 != nullptr)
+            *reinterpret_cast<float4*>(o_f32 + dst) =
+                make_float4(acc[0] * inv, acc[1] * inv, acc[2] * inv, acc[3] * inv);
+        else
+            *reinterpret_cast<uint2*>(o + dst) =
+                make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+    }
+    if (lane == 0 && lse != nullptr) lse[lrow] = total > 0.f ? M + logf(total) : -INFINITY;
 }
 
 }  // namespace attn

@@ -104,7 +104,15 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
  *   x_2p sin + x_2p+1 cos).  Angles are formed in double precision.  q_pos0 >= 0; D even.
  *   workspace / workspace_bytes: device scratch of at least attn_fwd_ex_workspace_size(...)
  *   bytes, owned by the caller; its contents are overwritten.  With rope_base <= 0 the
- *   workspace may be NULL.
+ *   workspace may be NULL: the call then runs as attn_fwd.  A non-NULL workspace smaller
+ *   than the size query returns ATTN_ERR_WORKSPACE.
+ * Key splits: a bf16 problem whose 128-row query tiles (ceil(Sq/128) * B * Hq of them) fill at
+ * most half of the 148 SMs divides each tile's key tiles among attn_fwd_kv_splits(...) CTAs
+ * (contiguous near-equal chunks) and merges their normalised partial outputs by logsumexp,
+ * L = log sum_s e^(lse_s), O = sum_s e^(lse_s - L) o_s (the split-KV combine of the decode
+ * path: oxibonsai-model 0.1.4 src/layers/flash_decode.rs, combine_tile_outputs).  This needs the workspace (the partials live
+ * there); attn_fwd and a NULL workspace run unsplit.  The result is the same attention up to
+ * rounding.
  * bf16 path: rotated Q and K are carried as a pair of bf16 values (hi + lo) each, so the
  * rotated operands keep about 16 mantissa bits; QK^T runs as three bf16 MMA chains.
  */
@@ -130,10 +138,17 @@ attn_status attn_fwd_masked(const void* q, const void* k, const void* v, const f
                             int D, float scale, int causal, attn_dtype dtype, float rope_base, int q_pos0,
                             void* workspace, size_t workspace_bytes, attn_stream_t stream);
 
-/* Bytes of workspace attn_fwd_ex needs for these sizes: 0 for D in {64, 128} without RoPE; the
- * rotated-K halves with RoPE; the padded q, k, v, o (and the inner call's needs) otherwise.   */
+/* Bytes of workspace attn_fwd_ex needs for these sizes: with RoPE the cos/sin table and the
+ * rotated-K halves; with key splits the fp32 partial outputs and logsumexps,
+ * splits * B * Sq * Hq * (D + 1) * 4 bytes (each part rounded up to 256 bytes); for D outside
+ * {64, 128} the padded q, k, v, o and the inner call's needs.  0 when none applies.          */
 size_t attn_fwd_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dtype dtype,
                                   float rope_base, int q_pos0);
+
+/* Key splits attn_fwd_ex uses for these sizes when given its workspace (1: unsplit):
+ * min(148 / tiles, ceil(Skv/128) / 2, 16) for bf16 problems with tiles = ceil(Sq/128) * B * Hq
+ * <= 74, when that is >= 2; 1 otherwise (and for ATTN_FP32).  Sizes <= 0 give 1.              */
+int attn_fwd_kv_splits(int B, int Hq, int Sq, int Skv, attn_dtype dtype);
 
 /*
  * attn_decode -- one query token per (sequence b, q head) against a KV cache, split-KV.

@@ -68,6 +68,28 @@ def test_fwd_ex_validation(lib):
     assert lib.attn_fwd_ex(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0.1, 1, 0, 10000.0, -1, P, need, None) == 1
 
 
+def test_fwd_key_split_sizing(lib):
+    """Key splits: min(148 // tiles, ceil(Skv/128) // 2, 16) for bf16 problems of <= 74 query tiles;
+    their partials (splits x rows x (D + 1) floats) follow the RoPE part of the workspace."""
+    assert lib.attn_fwd_kv_splits(1, 6, 1500, 1500, 0) == 2      # 72 tiles, 12 key tiles
+    assert lib.attn_fwd_kv_splits(1, 8, 128, 4096, 0) == 16      # 8 tiles, 32 key tiles
+    assert lib.attn_fwd_kv_splits(1, 2, 300, 1000, 2) == 4       # bf16 in, fp32 out
+    assert lib.attn_fwd_kv_splits(4, 8, 2048, 2048, 0) == 1      # 512 tiles
+    assert lib.attn_fwd_kv_splits(1, 2, 300, 300, 0) == 1        # 3 key tiles
+    assert lib.attn_fwd_kv_splits(1, 6, 1500, 1500, 1) == 1      # fp32 path
+    assert lib.attn_fwd_kv_splits(0, 6, 1500, 1500, 0) == 1
+    rows = 1500 * 6
+    part = -(-2 * rows * 64 * 4 // 256) * 256 + -(-2 * rows * 4 // 256) * 256
+    assert lib.attn_fwd_ex_workspace_size(1, 6, 6, 1500, 1500, 64, 0, 0.0, 0) == part
+    # RoPE part: cos/sin table (1500 positions x 32 pairs x 8 B), then K hi and lo (bf16)
+    rope = 1500 * 32 * 8 + 2 * (1500 * 6 * 64 * 2)
+    assert lib.attn_fwd_ex_workspace_size(1, 6, 6, 1500, 1500, 64, 0, 10000.0, 0) == rope + part
+    # a non-NULL workspace below the size is refused before any launch
+    P = FAKE
+    assert lib.attn_fwd_ex(P, P, P, P, None, 1, 6, 6, 1500, 1500, 64, 0.125, 0, 0, 0.0, 0, P, part - 1,
+                           None) == 5
+
+
 def test_decode_validation(lib):
     P = FAKE
     need = lib.attn_decode_workspace_size(2, 8, 64, 4)
