@@ -12,8 +12,12 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libattn_b200.so")
 SOURCES = ["attn_api.cu"]
-HEADERS = ["common.cuh", "decode.cuh", "prefill_f32.cuh", "prefill_tc.cuh", "rope.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include", "attn_b200.h")
+
+
+def _headers() -> list:
+    """Every header the translation unit may include (all of csrc/*.cuh)."""
+    return sorted(f for f in os.listdir(CSRC) if f.endswith(".cuh"))
 
 
 def nvcc() -> str:
@@ -25,7 +29,7 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [INCLUDE, os.path.abspath(__file__)]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + _headers()] + [INCLUDE, os.path.abspath(__file__)]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
