@@ -109,10 +109,11 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
  * Key splits: a bf16 problem whose 128-row query tiles (ceil(Sq/128) * B * Hq of them) fill at
  * most half of the 148 SMs divides each tile's key tiles among attn_fwd_kv_splits(...) CTAs
  * (contiguous near-equal chunks) and merges their normalised partial outputs by logsumexp,
- * L = log sum_s e^(lse_s), O = sum_s e^(lse_s - L) o_s (the split-KV combine of the decode
- * path: oxibonsai-model 0.1.4 src/layers/flash_decode.rs, combine_tile_outputs).  This needs the workspace (the partials live
- * there); attn_fwd and a NULL workspace run unsplit.  The result is the same attention up to
- * rounding.
+ * L = log sum_s e^(lse_s), O = sum_s e^(lse_s - L) o_s, in a second kernel launched as a
+ * programmatic dependent (the split-KV combine of the decode path: oxibonsai-model 0.1.4
+ * src/layers/flash_decode.rs, combine_tile_outputs).  This needs the workspace (the partials
+ * live there); attn_fwd and a NULL workspace run unsplit.  The result is the same attention
+ * up to rounding.
  * bf16 path: rotated Q and K are carried as a pair of bf16 values (hi + lo) each, so the
  * rotated operands keep about 16 mantissa bits; QK^T runs as three bf16 MMA chains.
  */
