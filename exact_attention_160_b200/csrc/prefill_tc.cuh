@@ -656,7 +656,27 @@ __global__ void __launch_bounds__(kPcThreads) prefill_combine_kernel(
     const int qi = static_cast<int>(bq % Sq);
     const int b = static_cast<int>(bq / Sq);
     const long lrow = (static_cast<long>(b) * Hq + h) * Sq + qi;
+    // Every load of the row is issued before any result is used (one round trip): the lse of
+    // split `lane`, and this lane's slice of every split's partial (the partials of rows below
+    // Sq are always written, zeros where a split saw no key, so all of them are finite).
     const float ls = lane < nsplit ? lse_part[lane * rows + lrow] : -INFINITY;
+    float x[kMaxKvSplits][E];
+#pragma unroll
+    for (int sp = 0; sp < kMaxKvSplits; ++sp) {
+        if (sp < nsplit) {
+            const float* src = o_part + (sp * rows + r) * D + lane * E;
+            if constexpr (E == 2) {
+                const float2 v = *reinterpret_cast<const float2*>(src);
+                x[sp][0] = v.x, x[sp][1] = v.y;
+            } else {
+                const float4 v = *reinterpret_cast<const float4*>(src);
+                x[sp][0] = v.x, x[sp][1] = v.y, x[sp][2] = v.z, x[sp][3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) x[sp][e] = 0.f;
+        }
+    }
     float M = ls;
 #pragma unroll
     for (int w = 16; w >= 1; w >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, w));
@@ -667,20 +687,11 @@ __global__ void __launch_bounds__(kPcThreads) prefill_combine_kernel(
     float acc[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int sp = 0; sp < nsplit; ++sp) {
-        const float ws = __shfl_sync(0xffffffffu, wt, sp);
-        if (ws == 0.f) continue;   // the same for every lane
-        const float* src = o_part + (sp * rows + r) * D + lane * E;
-        float x[E];
-        if constexpr (E == 2) {
-            const float2 v = *reinterpret_cast<const float2*>(src);
-            x[0] = v.x, x[1] = v.y;
-        } else {
-            const float4 v = *reinterpret_cast<const float4*>(src);
-            x[0] = v.x, x[1] = v.y, x[2] = v.z, x[3] = v.w;
-        }
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = fmaf(ws, x[e], acc[e]);
+    for (int sp = 0; sp < kMaxKvSplits; ++sp) {
+        const float ws = __shfl_sync(0xffffffffu, wt, sp);   // 0 for sp >= nsplit
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(ws, x[sp][e], acc[e]);
     }
     const float inv = total > 0.f ? 1.f / total : 0.f;
     const long dst = r * D + lane * E;
