@@ -3,6 +3,8 @@ the host before any launch (CPU only: these paths make no CUDA call)."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -88,6 +90,30 @@ def test_fwd_key_split_sizing(lib):
     P = FAKE
     assert lib.attn_fwd_ex(P, P, P, P, None, 1, 6, 6, 1500, 1500, 64, 0.125, 0, 0, 0.0, 0, P, part - 1,
                            None) == 5
+
+
+def test_key_split_count_follows_its_documented_rule(lib):
+    """attn_fwd_kv_splits against the header's formula over a grid of sizes."""
+    def rule(B, Hq, Sq, Skv, dtype):
+        tiles = -(-Sq // 128) * B * Hq
+        if dtype == 1 or tiles > 74:
+            return 1
+        n = min(148 // tiles, -(-Skv // 128) // 2, 16)
+        return n if n >= 2 else 1
+    for B in (1, 2, 3):
+        for Hq in (1, 2, 6, 8, 32):
+            for Sq in (1, 127, 128, 129, 700, 1500, 4096):
+                for Skv in (1, 255, 256, 511, 512, 1500, 4096, 65536):
+                    for dtype in (0, 1, 2):
+                        assert lib.attn_fwd_kv_splits(B, Hq, Sq, Skv, dtype) == rule(B, Hq, Sq, Skv, dtype), \
+                            (B, Hq, Sq, Skv, dtype)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    """No fallback: a binding whose library is absent raises instead of computing anything."""
+    code = f"import exact_attention_160_b200 as ea; ea.load_library({str(tmp_path / 'absent.so')!r})"
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, cwd=ROOT, timeout=300)
+    assert r.returncode != 0 and "not found" in r.stderr
 
 
 def test_decode_validation(lib):
