@@ -121,6 +121,32 @@ def _check(st: int, what: str):
         raise AttnError(st, what)
 
 
+def _shape(t):
+    return tuple(t.shape)
+
+
+def _check_qkv(q, k, v, o=None, lse=None, same_dtype_o=False):
+    """Shapes and dtypes the C ABI cannot see (it takes pointers and sizes): q [B, Sq, Hq, D],
+    k and v [B, Skv, Hkv, D] of q's dtype, o like q, lse [B, Hq, Sq] fp32."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [B, S, H, D], got {_shape(t)}")
+    if _shape(k) != _shape(v):
+        raise ValueError(f"k {_shape(k)} and v {_shape(v)} differ")
+    if q.shape[0] != k.shape[0] or q.shape[3] != k.shape[3]:
+        raise ValueError(f"q {_shape(q)} and k {_shape(k)} disagree on the batch or the head dim")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError(f"q, k and v must share one dtype ({q.dtype}, {k.dtype}, {v.dtype})")
+    B, Sq, Hq, _ = q.shape
+    if o is not None:
+        if _shape(o) != _shape(q):
+            raise ValueError(f"o {_shape(o)} must have q's shape {_shape(q)}")
+        if same_dtype_o and o.dtype != q.dtype:
+            raise TypeError(f"o must have q's dtype {q.dtype}")
+    if lse is not None and (lse.dtype != torch.float32 or _shape(lse) != (B, Hq, Sq)):
+        raise ValueError(f"lse must be float32 [B, Hq, Sq] = {(B, Hq, Sq)}, got {lse.dtype} {_shape(lse)}")
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -161,6 +187,7 @@ def attn_fwd_ex(q, k, v, scale: float, causal: bool, rope_base: float, q_pos0: i
     """Exact attention forward with RoPE on Q (positions q_pos0 + i) and K (positions j).
     kv_split=False (without RoPE, D 64 or 128) calls the C attn_fwd: no workspace, no key splits."""
     lib = load_library()
+    _check_qkv(q, k, v, o, lse)
     _need_cuda(q, k, v, o, lse, workspace)
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
@@ -209,6 +236,7 @@ def attn_fwd_masked(q, k, v, mask, scale: float, causal: bool, rope_base: float 
     """Exact attention with an additive fp32 mask on the scaled scores.  mask: [Sq, Skv] (shared),
     [B, Sq, Skv] (per batch, shared by the heads) or [B, Hq, Sq, Skv]; rows must be contiguous."""
     lib = load_library()
+    _check_qkv(q, k, v, o, lse)
     _need_cuda(q, k, v, o, lse, workspace)
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
@@ -236,6 +264,19 @@ def attn_decode(q, kcache, vcache, seqlens, scale: float, num_splits: int, o=Non
                 want_lse: bool = True, workspace=None, out_dtype=None, stream=None):
     """Split-KV decode of one token per (sequence, q head).  Returns (o, lse)."""
     lib = load_library()
+    if q.dim() != 3 or kcache.dim() != 4 or _shape(kcache) != _shape(vcache):
+        raise ValueError(f"q must be [B, Hq, D] and the caches one [B, Smax, Hkv, D] shape, got {_shape(q)}, "
+                         f"{_shape(kcache)}, {_shape(vcache)}")
+    if kcache.shape[0] != q.shape[0] or kcache.shape[3] != q.shape[2]:
+        raise ValueError(f"q {_shape(q)} and the caches {_shape(kcache)} disagree on the batch or the head dim")
+    if q.dtype != torch.bfloat16 or kcache.dtype != torch.bfloat16 or vcache.dtype != torch.bfloat16:
+        raise TypeError("attn_decode takes bf16 q and caches")
+    if seqlens.dtype != torch.int32 or _shape(seqlens) != (q.shape[0],):
+        raise ValueError(f"seqlens must be int32 [B], got {seqlens.dtype} {_shape(seqlens)}")
+    if o is not None and _shape(o) != _shape(q):
+        raise ValueError(f"o {_shape(o)} must have q's shape {_shape(q)}")
+    if lse is not None and (lse.dtype != torch.float32 or _shape(lse) != _shape(q)[:2]):
+        raise ValueError(f"lse must be float32 [B, Hq], got {lse.dtype} {_shape(lse)}")
     _need_cuda(q, kcache, vcache, seqlens, o, lse, workspace)
     B, Hq, D = q.shape
     Smax, Hkv = kcache.shape[1], kcache.shape[2]
@@ -256,6 +297,8 @@ def attn_decode(q, kcache, vcache, seqlens, scale: float, num_splits: int, o=Non
 def rope_apply(x, pos, base: float, stream=None):
     """Rotate x [T, H, D] in place at positions pos [T] (int32)."""
     lib = load_library()
+    if x.dim() != 3 or pos.dtype != torch.int32 or _shape(pos) != (x.shape[0],):
+        raise ValueError(f"x must be [T, H, D] and pos int32 [T], got {_shape(x)}, {pos.dtype} {_shape(pos)}")
     _need_cuda(x, pos)
     T, H, D = x.shape
     st = lib.rope_apply(_ptr(x), _ptr(pos), T, H, D, float(base), _dtype_code(x), _stream(stream))
@@ -277,12 +320,14 @@ def attn_bwd(q, k, v, o, lse, dout, scale: float, causal: bool, rope_base: float
     forward's outputs.  grad_dtype: torch.float32 to take a bf16 problem's gradients in fp32
     (default: q's dtype)."""
     lib = load_library()
-    _need_cuda(q, k, v, o, lse, dout, workspace)
-    B, Sq, Hq, D = q.shape
-    Skv, Hkv = k.shape[1], k.shape[2]
+    _check_qkv(q, k, v, o, lse, same_dtype_o=True)
+    _check_qkv(q, k, v, dout, None, same_dtype_o=True)
     gd = q.dtype if grad_dtype is None else grad_dtype
     if q.dtype == torch.float32 and gd != torch.float32:
         raise TypeError("fp32 inputs take fp32 gradients")
+    _need_cuda(q, k, v, o, lse, dout, workspace)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
     code = ATTN_FP32 if q.dtype == torch.float32 else (ATTN_BF16_OUT_F32 if gd == torch.float32 else ATTN_BF16)
     dq = torch.empty(q.shape, dtype=gd, device=q.device)
     dk = torch.empty(k.shape, dtype=gd, device=q.device)
@@ -301,6 +346,11 @@ def attn_bwd_masked(q, k, v, mask, o, lse, dout, scale: float, causal: bool, rop
                     q_pos0: int = 0, grad_dtype=None, workspace=None, stream=None):
     """attn_bwd for attn_fwd_masked (same mask)."""
     lib = load_library()
+    _check_qkv(q, k, v, o, lse, same_dtype_o=True)
+    _check_qkv(q, k, v, dout, None, same_dtype_o=True)
+    gd0 = q.dtype if grad_dtype is None else grad_dtype
+    if q.dtype == torch.float32 and gd0 != torch.float32:
+        raise TypeError("fp32 inputs take fp32 gradients")
     _need_cuda(q, k, v, o, lse, dout, workspace)
     B, Sq, Hq, D = q.shape
     Skv, Hkv = k.shape[1], k.shape[2]
@@ -327,6 +377,16 @@ def kv_append(kcache, vcache, seqlens, k_new, v_new, q=None, rope_base: float = 
     rope_base > 0; advances seqlens [B] (int32, device).  Overflowing sequences are skipped and
     flagged in the device status word."""
     lib = load_library()
+    if kcache.dim() != 4 or _shape(kcache) != _shape(vcache) or k_new.dim() != 4 or _shape(k_new) != _shape(v_new):
+        raise ValueError(f"caches [B, Smax, Hkv, D] and new rows [B, T, Hkv, D] of one shape each, got "
+                         f"{_shape(kcache)}, {_shape(vcache)}, {_shape(k_new)}, {_shape(v_new)}")
+    if (k_new.shape[0], k_new.shape[2], k_new.shape[3]) != (kcache.shape[0], kcache.shape[2], kcache.shape[3]):
+        raise ValueError(f"new rows {_shape(k_new)} do not fit the caches {_shape(kcache)}")
+    if q is not None and (q.dim() != 4 or q.shape[0] != k_new.shape[0] or q.shape[1] != k_new.shape[1]
+                          or q.shape[3] != k_new.shape[3]):
+        raise ValueError(f"q must be [B, T, Hq, D] for new rows {_shape(k_new)}, got {_shape(q)}")
+    if _shape(seqlens) != (kcache.shape[0],):
+        raise ValueError(f"seqlens must be [B], got {_shape(seqlens)}")
     _need_cuda(kcache, vcache, seqlens, k_new, v_new, q)
     for t in (kcache, vcache, k_new, v_new, q):
         if t is not None and t.dtype != torch.bfloat16:
