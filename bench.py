@@ -555,7 +555,9 @@ def run_reference(args):
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.Sq, "parallelism": "cpu"},
+           "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.Sq, "heads_q": w.Hq,
+                      "heads_kv": w.Hkv, "head_dim": w.D, "causal": w.causal, "rope_base": w.rope_base,
+                      "parallelism": "cpu", "inputs": "seeded synthetic N(0,1) rounded to bf16 (seeded_inputs)"},
            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": sample},
            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
