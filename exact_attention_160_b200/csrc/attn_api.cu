@@ -784,6 +784,41 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
                                              causal, tab, q_pos0, ws, wm, st, mk);
 }
 
+// Argument rules of the split-KV decode, shared by attn_decode and attn_decode_noalloc so that the
+// two entry points accept exactly the same calls (they differ only in where the partials live).
+attn_status decode_check(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens, const void* o,
+                         int B, int Hq, int Hkv, int Smax, int D, float scale, int num_splits, attn_dtype dtype) {
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_splits <= 0) return ATTN_ERR_INVALID_ARG;
+    if (Smax == 0) return ATTN_ERR_EMPTY_KV;
+    if (Smax < 0) return ATTN_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0) return ATTN_ERR_DIM_MISMATCH;
+    if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+    if (!q || !kcache || !vcache || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+    if (dtype != ATTN_BF16 && dtype != ATTN_BF16_OUT_F32)
+        return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
+    if (num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
+    if (static_cast<long>(B) * Hq > 2147483647L) return ATTN_ERR_UNSUPPORTED;
+    return ATTN_OK;
+}
+
+// Launch of a checked decode with its partials at `part` (attn_decode_workspace_size bytes, 16-byte
+// aligned): o_part [B*Hq*num_splits][D] fp32, then lse_part [B*Hq*num_splits] fp32.
+attn_status decode_launch(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens, void* o,
+                          float* lse, int B, int Hq, int Hkv, int Smax, int D, float scale, int num_splits, void* part,
+                          attn_dtype dtype, cudaStream_t st) {
+    const size_t slots = static_cast<size_t>(B) * Hq * num_splits;
+    float* o_part = static_cast<float*>(part);
+    float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(part) + round_up(slots * D * sizeof(float), 256));
+    const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
+    if (D == 64)
+        return launch_decode<64>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, o_part,
+                                 lse_part, st);
+    return launch_decode<128>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, o_part,
+                              lse_part, st);
+}
+
 }  // namespace
 
 // ------------------------------------------------------------------------------------------
@@ -888,49 +923,21 @@ size_t attn_decode_workspace_size(int B, int Hq, int D, int num_splits) {
 attn_status attn_decode(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens, void* o,
                         float* lse, int B, int Hq, int Hkv, int Smax, int D, float scale, int num_splits,
                         void* workspace, size_t workspace_bytes, attn_dtype dtype, attn_stream_t stream) {
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_splits <= 0) return ATTN_ERR_INVALID_ARG;
-    if (Smax == 0) return ATTN_ERR_EMPTY_KV;
-    if (Smax < 0) return ATTN_ERR_INVALID_ARG;
-    if (Hq % Hkv != 0) return ATTN_ERR_DIM_MISMATCH;
-    if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-    if (!q || !kcache || !vcache || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
-    if (dtype != ATTN_BF16 && dtype != ATTN_BF16_OUT_F32)
-        return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
-    const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
-    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
-    if (static_cast<long>(B) * Hq > 2147483647L) return ATTN_ERR_UNSUPPORTED;
+    const attn_status s = decode_check(q, kcache, vcache, seqlens, o, B, Hq, Hkv, Smax, D, scale, num_splits, dtype);
+    if (s != ATTN_OK) return s;
     const size_t need = attn_decode_workspace_size(B, Hq, D, num_splits);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return ATTN_ERR_WORKSPACE;
-    const size_t slots = static_cast<size_t>(B) * Hq * num_splits;
-    float* o_part = static_cast<float*>(workspace);
-    float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(slots * D * sizeof(float), 256));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    if (D == 64)
-        return launch_decode<64>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, o_part,
-                                 lse_part, st);
-    if (D == 128)
-        return launch_decode<128>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits,
-                                  o_part, lse_part, st);
-    return ATTN_ERR_UNSUPPORTED;
+    return decode_launch(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Smax, D, scale, num_splits, workspace, dtype,
+                         static_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_decode_noalloc(const void* q, const void* kcache, const void* vcache, const int32_t* seqlens,
                                 void* o, float* lse, int B, int Hq, int Hkv, int Smax, int D, float scale,
                                 int num_splits, attn_dtype dtype, attn_stream_t stream) {
-    // Same checks as attn_decode, then the size check against the built-in scratch.
-    if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_splits <= 0) return ATTN_ERR_INVALID_ARG;
-    if (Smax == 0) return ATTN_ERR_EMPTY_KV;
-    if (Smax < 0) return ATTN_ERR_INVALID_ARG;
-    if (Hq % Hkv != 0) return ATTN_ERR_DIM_MISMATCH;
-    if (!(scale > 0.f) || !isfinite(scale)) return ATTN_ERR_INVALID_ARG;
-    if (!q || !kcache || !vcache || !seqlens || !o) return ATTN_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
-    if (dtype != ATTN_BF16 && dtype != ATTN_BF16_OUT_F32)
-        return dtype == ATTN_FP32 ? ATTN_ERR_UNSUPPORTED : ATTN_ERR_INVALID_ARG;
-    if (D != 64 && D != 128) return ATTN_ERR_UNSUPPORTED;
-    if (num_splits > 65535) return ATTN_ERR_UNSUPPORTED;
+    // The same argument rules as attn_decode (one shared check), then the size check against the
+    // built-in scratch in place of the caller's workspace.
+    attn_status s = decode_check(q, kcache, vcache, seqlens, o, B, Hq, Hkv, Smax, D, scale, num_splits, dtype);
+    if (s != ATTN_OK) return s;
     const size_t need = attn_decode_workspace_size(B, Hq, D, num_splits);
     if (need > ATTN_NOALLOC_SCRATCH_BYTES) {
         char buf[160];
@@ -940,22 +947,11 @@ attn_status attn_decode_noalloc(const void* q, const void* kcache, const void* v
         return ATTN_ERR_WORKSPACE;
     }
     void* scratch = nullptr;
-    attn_status s = noalloc_scratch(&scratch);
-    if (s != ATTN_OK) return s;
+    if ((s = noalloc_scratch(&scratch)) != ATTN_OK) return s;
     // Nothing in the scratch has to start at zero: every partial the combine reads is written
     // earlier in the same call by the split kernel.
-    const size_t slots = static_cast<size_t>(B) * Hq * num_splits;
-    float* o_part = static_cast<float*>(scratch);
-    float* lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + round_up(slots * D * sizeof(float), 256));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const bool o_f32 = dtype == ATTN_BF16_OUT_F32;
-    if (D == 64)
-        return launch_decode<64>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits, o_part,
-                                 lse_part, st);
-    if (D == 128)
-        return launch_decode<128>(q, kcache, vcache, seqlens, o, o_f32, lse, B, Hq, Hkv, Smax, scale, num_splits,
-                                  o_part, lse_part, st);
-    return ATTN_ERR_UNSUPPORTED;
+    return decode_launch(q, kcache, vcache, seqlens, o, lse, B, Hq, Hkv, Smax, D, scale, num_splits, scratch, dtype,
+                         static_cast<cudaStream_t>(stream));
 }
 
 attn_status rope_apply(void* x, const int32_t* pos, int T, int H, int D, float base, attn_dtype dtype,
