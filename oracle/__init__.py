@@ -91,8 +91,21 @@ def _ptr(a: np.ndarray):
 
 
 def set_threads(n: int) -> None:
-    """Bound the OpenMP threads the oracle uses."""
+    """Bound the OpenMP threads the oracle uses in later calls from this thread (the
+    environment variable for a runtime not started yet, omp_set_num_threads for a running one)."""
     os.environ["OMP_NUM_THREADS"] = str(int(n))
+    try:
+        ctypes.CDLL("libgomp.so.1").omp_set_num_threads(int(n))
+    except OSError:
+        pass
+
+
+def threads() -> int:
+    """OpenMP threads the next oracle call from this thread will use."""
+    try:
+        return int(ctypes.CDLL("libgomp.so.1").omp_get_max_threads())
+    except OSError:
+        return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
 def rope(x, pos, base: float) -> np.ndarray:
