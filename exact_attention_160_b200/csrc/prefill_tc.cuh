@@ -14,18 +14,17 @@
 //     Each K/V tile is therefore loaded once for 256 query rows.  A problem small enough that its
 //     single tiles fit in one wave of the SMs runs one tile per CTA (the second tile inactive).
 //   * Warp roles (3 warpgroups): warp 0 issues TMA loads (Q once, then a ring of K/V stages);
-//     warp 1 owns tensor memory; warps 1 and 2 issue the tcgen05.mma of query tile 0 and 1, one
-//     thread each, from precomputed shared-memory descriptors; warps 4-7 and
-//     8-11 are the softmax warpgroups of query tile 0 and 1, one thread per query row (a warp
-//     may only touch TMEM lanes 32*(warp%4) .. +31, so the row of a softmax thread is
-//     32*(warp%4) + lane).
+//     warp 1 owns tensor memory and one of its threads issues every tcgen05.mma of the CTA from
+//     precomputed shared-memory descriptors; warps 4-7 and 8-11 are the softmax warpgroups of
+//     query tile 0 and 1, one thread per query row (a warp may only touch TMEM lanes
+//     32*(warp%4) .. +31, so the row of a softmax thread is 32*(warp%4) + lane).
 //   * S = Q K^T is a bf16 MMA (A and B from shared memory, M=128, N=128) into TMEM; the softmax
 //     threads read their row of S with tcgen05.ld, compute P = exp2(S*scale*log2e - m) in fp32,
-//     round P to bf16 and write it back to TMEM; O += P V is an MMA with A = P from TMEM and
-//     B = V from shared memory (N = D), accumulating in TMEM.
-//   * At D=128 the two softmax warpgroups take turns for their exponentiation phase (ping-pong
-//     through two mbarriers): the MUFU unit of each sub-partition is shared by one warp of each
-//     group, so while one group exponentiates the other loads S, takes its row max, corrects O.
+//     round P to bf16 and write it back to TMEM over S; O += P V is an MMA with A = P from TMEM
+//     and B = V from shared memory (N = D), accumulating in TMEM.
+//   * The MMA thread interleaves the tiles per KV tile j as PV_0(j), S_0(j+1), PV_1(j), S_1(j+1):
+//     while one softmax warpgroup exponentiates its tile, the tensor core runs the other tile's
+//     two products, so the groups fall into alternating phases without any turn-taking barrier.
 //   * Lazy rescale: the running max used for the exponent only moves when the block max exceeds
 //     it by more than kRescaleThreshold (log2 units, i.e. a factor 256), which keeps P <= 256
 //     while skipping the O correction on almost every block.  The "running max is -inf" guard
@@ -36,9 +35,9 @@
 //     compute_block_scores: score = dot * scale + mask) to the row of S in registers, as
 //     mask / scale on the unscaled dot products, before the row max.
 //
-// TMEM columns (512 allocated): S0 [0,128) S1 [128,256) O0, O1 (D each) after them; with D=64
-// P0 and P1 get their own 64 columns, with D=128 P_i overwrites the first 64 columns of S_i
-// (S_i is fully in registers by then; the next S_i MMA is issued only after PV_i completed).
+// TMEM columns (512 allocated): S0 [0,128) S1 [128,256) O0, O1 (D each) after them; P_t overwrites
+// the first 64 columns of S_t (S_t is fully in registers by then, and the next S_t MMA is issued
+// after PV_t, which reads P_t first).
 #pragma once
 
 #include "common.cuh"
@@ -72,16 +71,11 @@ struct TcCfg {
     static constexpr int Q_BYTES = 2 * Q_TILES * TILE_BYTES;
     static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES;
     static constexpr int SMEM_BYTES = SMEM_DATA + 1024 /* alignment slack */ + 256 /* barriers */;
-    static_assert(8 * (14 + 3 * STAGES) + 4 <= 256, "barrier area");
+    static_assert(8 * (10 + 3 * STAGES) + 4 <= 256, "barrier area");
+    // TMEM columns: S_t of query tile t at [128 t, 128 t + 128); P_t (bf16, 64 columns) is written
+    // over the first half of S_t once the softmax holds S_t in registers; O_t after both S tiles.
     static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
     static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
-    static constexpr uint32_t COL_P0 = (D == 64) ? 384 : 0;
-    static constexpr uint32_t COL_P1 = (D == 64) ? 448 : 128;
-    static constexpr bool P_ALIASES_S = (D != 64);
-    // Exponentiation turns between the two softmax warpgroups: at D=128 the softmax otherwise
-    // idles while P_i -> PV_i -> S_i(j+1) runs, so alternating keeps MUFU busy; at D=64 one warp
-    // alone cannot keep MUFU busy and the groups do better exponentiating concurrently.
-    static constexpr bool PINGPONG = (D != 64);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -136,16 +130,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_DATA);
     uint64_t* bar_q_full = bars + 0;
     uint64_t* bar_q_ready = bars + 1;
-    uint64_t* bar_s_full = bars + 2;       // [2]
-    uint64_t* bar_p_ready = bars + 4;      // [2]
-    uint64_t* bar_pv_done = bars + 6;      // [2]
-    uint64_t* bar_s_free = bars + 8;       // [2] softmax has read S_i into registers
-    uint64_t* bar_turn = bars + 10;        // [2] exponentiation turn of softmax warpgroup i
-    uint64_t* bar_k_full = bars + 12;      // [STAGES]
+    uint64_t* bar_s_full = bars + 2;       // [2] S_t(j) computed (commit after its MMAs)
+    uint64_t* bar_p_ready = bars + 4;      // [2] softmax t wrote P_t(j) (and corrected O_t)
+    uint64_t* bar_o_done = bars + 6;       // [2] the last PV_t completed
+    uint64_t* bar_mma_final = bars + 8;    // every MMA of the CTA completed
+    uint64_t* bar_k_full = bars + 10;      // [STAGES]
     uint64_t* bar_v_full = bar_k_full + C::STAGES;
     uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
-    uint64_t* bar_mma_final = bar_kv_empty + C::STAGES;   // [2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_mma_final + 2);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_kv_empty + C::STAGES);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -197,17 +189,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_s_full + i, 1);
             mbar_init(bar_p_ready + i, 128);
-            mbar_init(bar_pv_done + i, 1);
-            mbar_init(bar_s_free + i, 128);
-            mbar_init(bar_turn + i, 128);      // the other warpgroup's 128 threads hand over
+            mbar_init(bar_o_done + i, 1);
         }
+        mbar_init(bar_mma_final, 1);
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(bar_k_full + s, 1);
             mbar_init(bar_v_full + s, 1);
-            mbar_init(bar_kv_empty + s, 2);   // one commit from each MMA warp
+            mbar_init(bar_kv_empty + s, 1);   // one commit from the MMA thread
         }
-        mbar_init(bar_mma_final, 1);
-        mbar_init(bar_mma_final + 1, 1);
         mbar_fence_init();
     }
     if (warp == 0 && lane == 0) {
@@ -273,37 +262,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 mbar_wait(bar_v_full + j % C::STAGES, (j / C::STAGES) & 1);
             }
         }
-      } else if (warp == 1 || warp == 2) {
-        // =============================== MMA issuers =====================================
-        // Warp 1 issues every MMA of query tile 0, warp 2 those of tile 1 (one thread each), so
-        // the two tiles' pipelines do not wait on each other.  Per KV tile j:
-        //   S_i(j) = Q_i K_j^T  -> s_full_i ;  softmax_i reads S_i, writes P_i -> p_ready_i
-        //   O_i += P_i V_j      -> pv_done_i ;  both warps commit kv_empty once per stage
-        // D=64 (P_i has its own TMEM columns): S_i(j+1) is issued as soon as softmax_i has read
-        // S_i(j) (s_free_i), so the next scores are computed while the current ones are
-        // exponentiated.  D=128 (P_i overwrites S_i): S_i(j+1) waits until PV_i(j) consumed P_i(j).
-        const int i = warp - 1;
+      } else if (warp == 1) {
+        // =============================== MMA issuer ======================================
+        // One thread issues every MMA of both query tiles, interleaved per KV tile j as
+        //   PV_0(j)  S_0(j+1)  PV_1(j)  S_1(j+1)
+        // where S_t(j) = Q_t K_j^T (-> s_full_t) and PV_t(j): O_t += P_t(j) V_j.  The tensor core
+        // runs one thread's MMAs in issue order, so S_t(j+1) overwrites the columns of P_t(j)
+        // only after PV_t(j) has read them, and each softmax warpgroup works on its tile while
+        // the tensor core runs the other tile's two products.  A commit signals the completion of
+        // every MMA issued before it: s_full_t after S_t(j+1) therefore also means PV_t(j) is done,
+        // so the softmax may correct O_t in place before it hands over P_t(j+1).
+        // With a single K/V stage (D=128 with RoPE) S(j+1) has to wait for the stage to be
+        // released after PV(j), so both tiles' S(j+1) follow the release.
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
-            const uint32_t dS = tmem + (i ? C::COL_S1 : C::COL_S0);
-            const uint32_t dO = tmem + (i ? C::COL_O1 : C::COL_O0);
-            const uint32_t aP = tmem + (i ? C::COL_P1 : C::COL_P0);
-            const uint32_t sQi = smem_u32(sQ + i * C::Q_TILES * C::TILE_BYTES);
-            uint64_t* s_full = bar_s_full + i;
-            uint64_t* s_free = bar_s_free + i;
-            uint64_t* p_ready = bar_p_ready + i;
-            uint64_t* pv_done = bar_pv_done + i;
-            const int ni = i ? tile[1].nkv : tile[0].nkv;
+            constexpr uint32_t hiK = desc_sw128_hi(1024);
+            constexpr bool EARLY_S = C::STAGES > 1;
+            const int nt0 = tile[0].nkv, nt1 = tile[1].nkv;
             bool ok = mbar_wait(ROPE ? bar_q_ready : bar_q_full, 0);
             tc_fence_after();
             // Descriptors: the high words are constants, the low words advance with the start
             // address (16-byte units), so an MMA costs one add and the instruction itself.
-            constexpr uint32_t hiK = desc_sw128_hi(1024);
-            const uint32_t qlo = desc_sw128_lo(sQi, 16);
             const uint32_t kvlo0 = desc_sw128_lo(smem_u32(sKV), 16);
             const uint32_t vlo0 = desc_sw128_lo(smem_u32(sKV) + C::K_TILES * C::TILE_BYTES, C::TILE_BYTES / C::NBOX);
-            auto issue_s = [&](int j) {
+            auto issue_s = [&](int t, int j) {
+                const uint32_t qlo = desc_sw128_lo(smem_u32(sQ + t * C::Q_TILES * C::TILE_BYTES), 16);
+                const uint32_t dS = tmem + (t ? C::COL_S1 : C::COL_S0);
                 const uint32_t klo = kvlo0 + ((j % C::STAGES) * C::STAGE_BYTES >> 4);
                 // chains: (Qh,Kh) [+ (Qh,Kl) + (Ql,Kh) with RoPE]
                 constexpr int NCHAIN = ROPE ? 3 : 1;
@@ -320,9 +305,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                                (ch > 0 || kk > 0) ? 1u : 0u);
                     }
                 }
-                mma_commit(s_full);
+                mma_commit(bar_s_full + t);
             };
-            auto issue_pv = [&](int j) {
+            auto issue_pv = [&](int t, int j) {
+                const uint32_t dO = tmem + (t ? C::COL_O1 : C::COL_O0);
+                const uint32_t aP = tmem + (t ? C::COL_S1 : C::COL_S0);
                 const uint32_t vlo = vlo0 + ((j % C::STAGES) * C::STAGE_BYTES >> 4);
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -330,48 +317,57 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     mma_ts(dO, aP + kk * 8, desc_join(vlo + kk * (2048 >> 4), hiK), idesc_pv,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(pv_done);
+                if (j == (t ? nt1 : nt0) - 1) mma_commit(bar_o_done + t);
             };
             auto wait_k = [&](int j) {
                 const bool r = mbar_wait(bar_k_full + j % C::STAGES, (j / C::STAGES) & 1);
                 tc_fence_after();
                 return r;
             };
-            if (ok && ni > 0) {
+            const int nkv_all = max(nt0, nt1);
+            if (ok && nkv_all > 0) {
                 ok = wait_k(0);
-                if (ok) issue_s(0);
+                if (ok && nt0 > 0) issue_s(0, 0);
+                if (ok && nt1 > 0) issue_s(1, 0);
             }
-            for (int j = 0; j < nkv; ++j) {
+            for (int j = 0; j < nkv_all; ++j) {
                 const int s = j % C::STAGES;
-                if (j < ni) {
-                    if (ok && !C::P_ALIASES_S && j + 1 < ni) {
-                        ok = wait_k(j + 1) && mbar_wait(s_free, j & 1);
+                if (ok) {
+                    ok = mbar_wait(bar_v_full + s, (j / C::STAGES) & 1);
+                    tc_fence_after();
+                }
+                bool k_next = false;   // K(j+1) waited for
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const int n = t ? nt1 : nt0;
+                    if (j >= n) continue;
+                    if (ok) {
+                        ok = mbar_wait(bar_p_ready + t, j & 1);
                         tc_fence_after();
-                        if (ok) issue_s(j + 1);
                     }
-                    if (ok) ok = mbar_wait(bar_v_full + s, (j / C::STAGES) & 1) && mbar_wait(p_ready, j & 1);
-                    tc_fence_after();
-                    if (ok) issue_pv(j);
-                } else {
-                    // No work for this tile, but the stage's release still needs this warp's
-                    // arrival.  Wait until the stage holds tile j first: an arrival made earlier
-                    // could complete a later phase of kv_empty on its own and free the stage
-                    // while the other warp's MMAs still read it.
-                    mbar_wait(bar_k_full + s, (j / C::STAGES) & 1);
-                    mbar_wait(bar_v_full + s, (j / C::STAGES) & 1);
+                    if (ok) issue_pv(t, j);
+                    if (EARLY_S && ok && j + 1 < n) {
+                        if (!k_next) ok = wait_k(j + 1);
+                        k_next = true;
+                        if (ok) issue_s(t, j + 1);
+                    }
                 }
-                // this warp is done with stage s once its MMAs so far complete (S_i(j), PV_i(j))
+                // stage s is free once every MMA issued so far has completed
                 mma_commit(bar_kv_empty + s);
-                if (ok && C::P_ALIASES_S && j + 1 < ni) {
-                    // S_i(j+1) overwrites P_i(j): PV_i(j) must have consumed it
-                    ok = wait_k(j + 1) && mbar_wait(pv_done, j & 1);
-                    tc_fence_after();
-                    if (ok) issue_s(j + 1);
+                if (!EARLY_S && ok && j + 1 < nkv_all) {
+                    ok = wait_k(j + 1);
+                    if (ok && j + 1 < nt0) issue_s(0, j + 1);
+                    if (ok && j + 1 < nt1) issue_s(1, j + 1);
                 }
+            }
+            // a tile whose pipeline stopped early still gets its completion signal
+            if (!ok) {
+                mma_commit(bar_o_done + 0);
+                mma_commit(bar_o_done + 1);
             }
             // every MMA issued above must be complete before tensor memory is released
-            mma_commit(bar_mma_final + i);
-            mbar_wait(bar_mma_final + i, 0);
+            mma_commit(bar_mma_final);
+            mbar_wait(bar_mma_final, 0);
         }
       }
     } else {
@@ -387,7 +383,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS = tmem + lane_base + (wg ? C::COL_S1 : C::COL_S0);
         const uint32_t tO = tmem + lane_base + (wg ? C::COL_O1 : C::COL_O0);
-        const uint32_t tP = tmem + lane_base + (wg ? C::COL_P1 : C::COL_P0);
         const int qrow = T.r0 + row;                // absolute query row
         const long off_c = static_cast<long>(p.Skv) - p.Sq;
         bool ok = true;
@@ -437,26 +432,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         float l_run = 0.f;         // row sum of the fp32 weights (logsumexp)
         float l_mma = 0.f;         // row sum of the bf16-rounded weights (normalises O)
         const float sl2 = p.scale_log2;
-        // Turn passing: round r of group 0 waits turn_0 (phase r), exponentiates, hands turn_1;
-        // group 1 the reverse.  Group 1 gives group 0 the first turn.  Both groups run all nkv
-        // rounds (idle rounds only pass the turn), so neither waits for a hand-over that never
-        // comes; after a failed wait a group stops waiting but keeps handing over.
-        if (C::PINGPONG && wg == 1 && nkv > 0) mbar_arrive(bar_turn + 0);
-        for (int j = 0; j < nkv; ++j) {
-          const bool work = j < T.nkv;
-          uint32_t sr[4][32];
-          float mu = 0.f;
-          if (ok && work) {
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) ok = false;
+        const uint32_t tP = tS;    // P_t(j) is written over the first 64 columns of S_t
+        for (int j = 0; j < T.nkv; ++j) {
+            uint32_t sr[4][32];
+            if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) ok = false;
             tc_fence_after();
+            if (!ok) {
+                mbar_arrive(bar_p_ready + wg);   // keep the MMA thread's count; it stops on its own
+                continue;
+            }
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tmem_ld32(tS + cb * 32, sr[cb]);
             tmem_wait_ld();
-            if (!C::P_ALIASES_S) {
-                // S_i is in registers: the next S_i MMA may overwrite it
-                tc_fence_before();
-                mbar_arrive(bar_s_free + wg);
-            }
             const int k0 = (kv0 + j) * 128;
             if (MASK && qrow < p.Sq) {
                 // additive mask: S holds q.k unscaled, so add mask / scale; the exponent
@@ -503,10 +490,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 corr = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - tmax);
                 m_run = tmax;
             }
-            // O correction: only warps with a rescaling row, only once O holds earlier blocks
-            if (ok && j > 0 && __any_sync(0xffffffffu, need)) {
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) ok = false;
-                tc_fence_after();
+            // O correction, only in warps with a rescaling row and once O holds earlier blocks.
+            // O_t is at rest here: PV_t(j-1) completed before s_full_t(j) was signalled, and
+            // PV_t(j) is issued only after this warpgroup's p_ready arrival below.
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
                 for (int cb = 0; cb < D / 32; ++cb) {
                     uint32_t orr[32];
@@ -516,20 +503,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * corr);
                     tmem_st32(tO + cb * 32, orr);
                 }
-                tmem_wait_st();
             }
             l_run *= corr;
             l_mma *= corr;
-            mu = (m_run == -INFINITY) ? 0.f : m_run;
-            if (!C::P_ALIASES_S && j > 0) {
-                // P_i(j-1) must have been consumed by PV_i(j-1) before it is overwritten
-                if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) { ok = false; }
-                tc_fence_after();
-            }
-          }
-          // wait for this group's exponentiation turn (every round, also idle ones)
-          if (C::PINGPONG && ok && !__all_sync(0xffffffffu, mbar_wait(bar_turn + wg, j & 1))) ok = false;
-          if (ok && work) {
+            const float mu = (m_run == -INFINITY) ? 0.f : m_run;
             // p = exp2(s*scale*log2e - mu) in fp32, rounded to bf16 for the PV MMA.  Two row sums:
             // the exact one (for the logsumexp) and the sum of the rounded values the MMA uses
             // (O is normalised by it, so the rounding of a dominant weight cancels).
@@ -563,10 +540,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(bar_p_ready + wg);
-          }
-          // hand the exponentiation turn to the other group (group 1 skips its last hand-over,
-          // which nobody would wait for)
-          if (C::PINGPONG && !(wg == 1 && j == nkv - 1)) mbar_arrive(bar_turn + (wg ^ 1));
         }
 
         // epilogue: O / l -> bf16 or fp32, lse.  The TMEM reads are warp-collective, so every
@@ -574,7 +547,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         if (T.active) {
             bool have = ok && T.nkv > 0;
             if (have) {
-                have = __all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (T.nkv - 1) & 1));
+                have = __all_sync(0xffffffffu, mbar_wait(bar_o_done + wg, 0));
                 tc_fence_after();
             }
             const bool store = qrow < p.Sq;
