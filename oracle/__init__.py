@@ -48,9 +48,11 @@ def _bind(path: str):
         lib.oracle_attn_bwd_f64.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
         lib.oracle_attn_fwd_mask_f64.argtypes = [P, P, P, P, I64, I64, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
         lib.oracle_attn_bwd_mask_f64.argtypes = [P, P, P, P, P, I64, I64, P, P, P, I, I, I, I, I, I, Dd, I, Dd, I]
+        lib.oracle_attn_bwd_sampled_f64.argtypes = [P, P, P, P, I, I, I, I, I, I, Dd, I, Dd, I, I, I, P, I, P, I,
+                                                    P, P, P]
         for f in (lib.oracle_rope_f64, lib.oracle_attn_fwd_f64, lib.oracle_attn_fwd_tiled_f64,
                   lib.oracle_decode_f64, lib.oracle_decode_split_f64, lib.oracle_attn_bwd_f64,
-                  lib.oracle_attn_fwd_mask_f64, lib.oracle_attn_bwd_mask_f64):
+                  lib.oracle_attn_fwd_mask_f64, lib.oracle_attn_bwd_mask_f64, lib.oracle_attn_bwd_sampled_f64):
             f.restype = I
     return lib
 
@@ -248,6 +250,27 @@ def attn_bwd(q, k, v, dout, scale: float, causal: bool, rope_base: float = 0.0, 
     _check(_load().oracle_attn_bwd_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                        B, Hq, Hkv, Sq, Skv, D, float(scale), int(bool(causal)),
                                        float(rope_base), int(q_pos0)))
+    return dq, dk, dv
+
+
+def attn_bwd_sampled(q, k, v, dout, scale: float, causal: bool, rope_base: float, q_pos0: int, b: int, kvh: int,
+                     rows, keys):
+    """The backward of one (batch b, kv head kvh) group at chosen places, fp64: dq of every q head
+    of the group at query rows `rows` ([g, len(rows), D]), dk and dv of the kv head at keys `keys`
+    ([len(keys), D] each).  Same definition as attn_bwd, for full-size problems."""
+    q, k, v, g_ = _f32(q), _f32(k), _f32(v), _f32(dout)
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    keys = np.ascontiguousarray(keys, dtype=np.int64)
+    g = Hq // Hkv
+    dq = np.empty((g, rows.shape[0], D), dtype=np.float64)
+    dk = np.empty((keys.shape[0], D), dtype=np.float64)
+    dv = np.empty((keys.shape[0], D), dtype=np.float64)
+    _check(_load().oracle_attn_bwd_sampled_f64(_ptr(q), _ptr(k), _ptr(v), _ptr(g_), B, Hq, Hkv, Sq, Skv, D,
+                                               float(scale), int(bool(causal)), float(rope_base), int(q_pos0),
+                                               int(b), int(kvh), _ptr(rows), rows.shape[0], _ptr(keys),
+                                               keys.shape[0], _ptr(dq), _ptr(dk), _ptr(dv)))
     return dq, dk, dv
 
 

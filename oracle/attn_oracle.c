@@ -40,6 +40,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORACLE_OK 0
 #define ORACLE_ERR_INVALID_ARG 1
@@ -670,5 +673,139 @@ int oracle_attn_fwd_mask_f64(const float* q, const float* k, const float* v, con
             free(qd);
         }
     }
+    return fail ? ORACLE_ERR_NOMEM : ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------------------------------ */
+/* Backward at sampled rows and keys of one (batch, kv head) group                             */
+/* ------------------------------------------------------------------------------------------ */
+
+/* The same definition as oracle_attn_bwd_f64 ([P1] flash_backward_head: P from the full score row,
+ * dP = dO . v_j, D = sum_j p_j dP_j, dS = p (dP - D); dQ = scale sum_j dS_j k_j, dK_j = scale
+ * sum_i dS_ij q_i, dV_j = sum_i p_ij dO_i; [P2] the kv head's gradients summed over its q heads
+ * and RoPE undone by the negated angle), evaluated only where a full-size problem is checked:
+ *   dq_s [g][nrows][D]  dq of every q head of kv head `kvh` of batch `b` at query rows rows[]
+ *   dk_s, dv_s [nkeys][D]  dk, dv of that kv head at keys keys[]
+ * Every query row of the group is still evaluated in full (its P and D need the whole row); only
+ * the sums that are not asked for are skipped.  Rows are split among threads, each with its own
+ * partial sums for the sampled keys, added up in thread order at the end.                     */
+int oracle_attn_bwd_sampled_f64(const float* q, const float* k, const float* v, const float* dout, int B, int Hq,
+                                int Hkv, int Sq, int Skv, int D, double scale, int causal, double rope_base,
+                                int q_pos0, int b, int kvh, const int64_t* rows, int nrows, const int64_t* keys,
+                                int nkeys, double* dq_s, double* dk_s, double* dv_s) {
+    int st = check_dims(B, Hq, Hkv, Sq, Skv, D);
+    if (st) return st;
+    if (rope_base > 0.0 && D % 2) return ORACLE_ERR_INVALID_ARG;
+    if (b < 0 || b >= B || kvh < 0 || kvh >= Hkv || nrows < 0 || nkeys < 0) return ORACLE_ERR_INVALID_ARG;
+    for (int r = 0; r < nrows; ++r)
+        if (rows[r] < 0 || rows[r] >= Sq) return ORACLE_ERR_INVALID_ARG;
+    for (int t = 0; t < nkeys; ++t)
+        if (keys[t] < 0 || keys[t] >= Skv) return ORACLE_ERR_INVALID_ARG;
+    const int g = Hq / Hkv;
+    double* Kd = (double*)malloc(sizeof(double) * (size_t)Skv * D);
+    double* Vd = (double*)malloc(sizeof(double) * (size_t)Skv * D);
+    int nthr = 1;
+#ifdef _OPENMP
+    nthr = omp_get_max_threads();
+#endif
+    double* part = (double*)calloc((size_t)nthr * 2 * (nkeys > 0 ? nkeys : 1) * D, sizeof(double));
+    int* slot = (int*)malloc(sizeof(int) * (size_t)(Sq > 0 ? Sq : 1));   /* row -> index in rows[], or -1 */
+    if (!Kd || !Vd || !part || !slot) {
+        free(Kd), free(Vd), free(part), free(slot);
+        return ORACLE_ERR_NOMEM;
+    }
+    gather_head(k, b, kvh, Skv, Hkv, D, rope_base, Kd);
+    gather_head(v, b, kvh, Skv, Hkv, D, 0.0, Vd);
+    for (int i = 0; i < Sq; ++i) slot[i] = -1;
+    for (int r = 0; r < nrows; ++r) slot[rows[r]] = r;
+    for (long e = 0; e < (long)g * nrows * D; ++e) dq_s[e] = 0.0;
+    int fail = 0;
+#pragma omp parallel
+    {
+        int tid = 0;
+#ifdef _OPENMP
+        tid = omp_get_thread_num();
+#endif
+        double* dKp = part + (size_t)tid * 2 * (nkeys > 0 ? nkeys : 1) * D;
+        double* dVp = dKp + (size_t)(nkeys > 0 ? nkeys : 1) * D;
+        double* s = (double*)malloc(sizeof(double) * (size_t)Skv);
+        double* dP = (double*)malloc(sizeof(double) * (size_t)Skv);
+        double* qd = (double*)malloc(sizeof(double) * (size_t)D);
+        double* go = (double*)malloc(sizeof(double) * (size_t)D);
+        double* dqr = (double*)malloc(sizeof(double) * (size_t)D);
+        if (!s || !dP || !qd || !go || !dqr) {
+#pragma omp atomic write
+            fail = 1;
+        } else {
+#pragma omp for schedule(dynamic, 4) collapse(2)
+            for (int hg = 0; hg < g; ++hg) {
+                for (int i = 0; i < Sq; ++i) {
+                    const int hq = kvh * g + hg;
+                    const long qoff = (((long)b * Sq + i) * Hq + hq) * D;
+                    const int nvis = visible_keys(i, Sq, Skv, causal);
+                    if (nvis <= 0) continue; /* no gradient through this row; dq stays 0 */
+                    for (int d = 0; d < D; ++d) qd[d] = (double)q[qoff + d];
+                    if (rope_base > 0.0) rope_vec(qd, (double)q_pos0 + (double)i, D, rope_base);
+                    for (int d = 0; d < D; ++d) go[d] = (double)dout[qoff + d];
+                    double m = -INFINITY;
+                    for (int j = 0; j < nvis; ++j) {
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d) dot += qd[d] * Kd[(long)j * D + d];
+                        s[j] = scale * dot;
+                        if (s[j] > m) m = s[j];
+                    }
+                    double l = 0.0;
+                    for (int j = 0; j < nvis; ++j) l += exp(s[j] - m);
+                    double Dsum = 0.0;
+                    for (int j = 0; j < nvis; ++j) {
+                        const double p = exp(s[j] - m) / l;
+                        double dot = 0.0;
+                        for (int d = 0; d < D; ++d) dot += go[d] * Vd[(long)j * D + d];
+                        dP[j] = dot;
+                        Dsum += p * dot;
+                    }
+                    if (slot[i] >= 0) {
+                        for (int d = 0; d < D; ++d) dqr[d] = 0.0;
+                        for (int j = 0; j < nvis; ++j) {
+                            const double p = exp(s[j] - m) / l;
+                            const double dS = p * (dP[j] - Dsum);
+                            for (int d = 0; d < D; ++d) dqr[d] += scale * dS * Kd[(long)j * D + d];
+                        }
+                        if (rope_base > 0.0) rope_vec(dqr, -((double)q_pos0 + (double)i), D, rope_base);
+                        double* dst = dq_s + ((long)hg * nrows + slot[i]) * D;
+                        for (int d = 0; d < D; ++d) dst[d] = dqr[d];
+                    }
+                    for (int t = 0; t < nkeys; ++t) {
+                        const long j = keys[t];
+                        if (j >= nvis) continue;
+                        const double p = exp(s[j] - m) / l;
+                        const double dS = p * (dP[j] - Dsum);
+                        for (int d = 0; d < D; ++d) {
+                            dKp[(long)t * D + d] += scale * dS * qd[d];
+                            dVp[(long)t * D + d] += p * go[d];
+                        }
+                    }
+                }
+            }
+        }
+        free(s), free(dP), free(qd), free(go), free(dqr);
+    }
+    if (!fail) {
+        for (int t = 0; t < nkeys; ++t) {
+            double* dkr = dk_s + (long)t * D;
+            double* dvr = dv_s + (long)t * D;
+            for (int d = 0; d < D; ++d) dkr[d] = dvr[d] = 0.0;
+            for (int th = 0; th < nthr; ++th) {
+                const double* dKp = part + (size_t)th * 2 * nkeys * D;
+                const double* dVp = dKp + (size_t)nkeys * D;
+                for (int d = 0; d < D; ++d) {
+                    dkr[d] += dKp[(long)t * D + d];
+                    dvr[d] += dVp[(long)t * D + d];
+                }
+            }
+            if (rope_base > 0.0) rope_vec(dkr, -(double)keys[t], D, rope_base);
+        }
+    }
+    free(Kd), free(Vd), free(part), free(slot);
     return fail ? ORACLE_ERR_NOMEM : ORACLE_OK;
 }

@@ -640,6 +640,28 @@ def pin_backward_invariants():
     _close(dv, mv.reshape(B, Skv, Hkv, G, D).sum(axis=3), 1e-12, "GQA dv = summed MHA dv")
 
 
+def pin_sampled_backward_matches_full_backward():
+    """The sampled backward of one (batch, kv head) group (used to check full-size problems)
+    equals the full backward at its rows and keys: GQA with RoPE at a query offset and causal
+    rows that see no key (Sq > Skv), and a non-causal MQA case."""
+    for seed, (B, Hq, Hkv, Sq, Skv, D, causal, rb, qp) in ((93, (2, 4, 2, 37, 29, 16, True, 10000.0, 16)),
+                                                            (94, (1, 3, 1, 40, 40, 8, False, 0.0, 0))):
+        q = normal_f32(seed, 0, (B, Sq, Hq, D))
+        k = normal_f32(seed, 1, (B, Skv, Hkv, D))
+        v = normal_f32(seed, 2, (B, Skv, Hkv, D))
+        g = normal_f32(seed, 3, (B, Sq, Hq, D))
+        dq, dk, dv = oracle.attn_bwd(q, k, v, g, 0.3, causal, rb, qp)
+        G = Hq // Hkv
+        rows, keys = np.array([0, 5, Sq - 1]), np.array([0, 7, Skv - 1])
+        for b in range(B):
+            for kvh in range(Hkv):
+                sq, sk, sv = oracle.attn_bwd_sampled(q, k, v, g, 0.3, causal, rb, qp, b, kvh, rows, keys)
+                for hg in range(G):
+                    _close(sq[hg], dq[b, rows, kvh * G + hg], 1e-12, "sampled dq")
+                _close(sk, dk[b, keys, kvh], 1e-12, "sampled dk")
+                _close(sv, dv[b, keys, kvh], 1e-12, "sampled dv")
+
+
 def pin_additive_mask():
     """An additive mask of zeros changes nothing; -inf above the diagonal is the causal mask; a
     constant mask c leaves o unchanged and adds c to lse; -inf on one key equals attention
