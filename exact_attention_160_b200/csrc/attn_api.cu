@@ -19,6 +19,7 @@
 #include "rope.cuh"
 #include "backward.cuh"
 #include "backward_mma.cuh"
+#include "backward_tc.cuh"
 
 using namespace attn;
 
@@ -78,6 +79,29 @@ bool make_tmap_bshd_rows(CUtensorMap* m, const void* ptr, int B, int S, int H, i
 
 bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D) {
     return make_tmap_bshd_rows(m, ptr, B, S, H, D, 128);
+}
+
+// fp32 array [rows][cols] viewed 2-D with a box of 128 columns x 1 row, no swizzle; columns past
+// `cols` read as 0.  The row stride (cols * 4 bytes) must be a multiple of 16.
+bool make_tmap_rows_f32(CUtensorMap* m, const void* ptr, long rows, int cols) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) {
+        cuda_failure("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", "entry point unavailable");
+        return false;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+    cuuint32_t box[2] = {128, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char buf[96];
+        snprintf(buf, sizeof(buf), "CUresult %d (rows %ld, cols %d)", static_cast<int>(r), rows, cols);
+        cuda_failure("cuTensorMapEncodeTiled", buf);
+    }
+    return r == CUDA_SUCCESS;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -528,7 +552,7 @@ attn_status launch_bwd(const T* q, const T* k, const T* v, const T* o, const flo
 // Layout of the bf16 (tensor-core) attn_bwd workspace: rope table, D_i, and with RoPE the
 // rotated q and k as hi/lo bf16 pairs.
 struct BmWorkspace {
-    size_t tab_off, d_off, qh_off, ql_off, kh_off, kl_off, total;
+    size_t tab_off, d_off, l2_off, qh_off, ql_off, kh_off, kl_off, total;
     int positions;
 };
 
@@ -541,12 +565,84 @@ BmWorkspace bm_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, bool ro
     const size_t kb = rope ? static_cast<size_t>(B) * Skv * Hkv * D * 2 : 0;
     w.tab_off = 0;
     w.d_off = round_up(tab, 256);
-    w.qh_off = round_up(w.d_off + static_cast<size_t>(B) * Hq * Sq * sizeof(float), 256);
+    w.l2_off = round_up(w.d_off + static_cast<size_t>(B) * Hq * Sq * sizeof(float), 256);
+    w.qh_off = round_up(w.l2_off + static_cast<size_t>(B) * Hq * Sq * sizeof(float), 256);
     w.ql_off = round_up(w.qh_off + qb, 256);
     w.kh_off = round_up(w.ql_off + qb, 256);
     w.kl_off = round_up(w.kh_off + kb, 256);
     w.total = round_up(w.kl_off + kb, 256);
     return w;
+}
+
+// The tensor-core (tcgen05) backward for unmasked bf16 problems whose query length is a multiple
+// of 4 (the per-row LSE and D arrays are read as 2-D TMA rows); the mma.sync kernels cover the rest.
+bool bwd_tc_eligible(int Sq, const MaskArg& mk) { return mk.ptr == nullptr && Sq % 4 == 0; }
+
+template <int D, bool ROPE>
+attn_status launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const __nv_bfloat16* v,
+                          const __nv_bfloat16* o, const float* lse, const __nv_bfloat16* dout, void* dq, void* dk,
+                          void* dv, bool g_f32, int B, int Hq, int Hkv, int Sq, int Skv, float scale, int causal,
+                          const float2* tab, int q_pos0, uint8_t* ws, const BmWorkspace& w, cudaStream_t st) {
+    float* Dvec = reinterpret_cast<float*>(ws + w.d_off);
+    float* lse2 = reinterpret_cast<float*>(ws + w.l2_off);
+    const long nq = static_cast<long>(B) * Sq * Hq;
+    bwd_rowdot_kernel<D><<<static_cast<unsigned>((nq * (D / 8) + 255) / 256), 256, 0, st>>>(o, dout, Dvec, nq, Sq, Hq);
+    attn_status s = launch_status("bwd_rowdot_kernel");
+    if (s != ATTN_OK) return s;
+    bwd_lse2_kernel<<<static_cast<unsigned>(min((nq + 255) / 256, 148L * 32)), 256, 0, st>>>(lse, lse2, nq);
+    if ((s = launch_status("bwd_lse2_kernel")) != ATTN_OK) return s;
+    const __nv_bfloat16 *qh = q, *ql = q, *kh = k, *kl = k;
+    if (ROPE) {
+        uint32_t* pqh = reinterpret_cast<uint32_t*>(ws + w.qh_off);
+        uint32_t* pql = reinterpret_cast<uint32_t*>(ws + w.ql_off);
+        uint32_t* pkh = reinterpret_cast<uint32_t*>(ws + w.kh_off);
+        uint32_t* pkl = reinterpret_cast<uint32_t*>(ws + w.kl_off);
+        const long nqp = nq * (D / 2), nkp = static_cast<long>(B) * Skv * Hkv * (D / 2);
+        bwd_rope_split_kernel<<<static_cast<unsigned>(min((nqp + 255) / 256, 148L * 64)), 256, 0, st>>>(
+            reinterpret_cast<const uint32_t*>(q), pqh, pql, tab, nqp, Sq, Hq, D, q_pos0);
+        if ((s = launch_status("bwd_rope_split_kernel(q)")) != ATTN_OK) return s;
+        bwd_rope_split_kernel<<<static_cast<unsigned>(min((nkp + 255) / 256, 148L * 64)), 256, 0, st>>>(
+            reinterpret_cast<const uint32_t*>(k), pkh, pkl, tab, nkp, Skv, Hkv, D, 0);
+        if ((s = launch_status("bwd_rope_split_kernel(k)")) != ATTN_OK) return s;
+        qh = reinterpret_cast<const __nv_bfloat16*>(pqh);
+        ql = reinterpret_cast<const __nv_bfloat16*>(pql);
+        kh = reinterpret_cast<const __nv_bfloat16*>(pkh);
+        kl = reinterpret_cast<const __nv_bfloat16*>(pkl);
+    }
+    CUtensorMap tq, tql, tk, tkl, tv, tdo, tl2, tdv;
+    if (!make_tmap_bshd(&tq, qh, B, Sq, Hq, D) || !make_tmap_bshd(&tql, ql, B, Sq, Hq, D) ||
+        !make_tmap_bshd(&tk, kh, B, Skv, Hkv, D) || !make_tmap_bshd(&tkl, kl, B, Skv, Hkv, D) ||
+        !make_tmap_bshd(&tv, v, B, Skv, Hkv, D) || !make_tmap_bshd(&tdo, dout, B, Sq, Hq, D) ||
+        !make_tmap_rows_f32(&tl2, lse2, static_cast<long>(B) * Hq, Sq) ||
+        !make_tmap_rows_f32(&tdv, Dvec, static_cast<long>(B) * Hq, Sq))
+        return ATTN_ERR_CUDA;
+    using C = BtCfg<D, ROPE>;
+    BtParams p{};
+    p.lse2 = lse2;
+    p.Dvec = Dvec;
+    p.tab = tab;
+    p.B = B, p.Hq = Hq, p.Hkv = Hkv, p.Sq = Sq, p.Skv = Skv, p.q_pos0 = q_pos0, p.causal = causal;
+    p.scale = scale;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    auto kdq = bwd_dq_tc_kernel<D, ROPE>;
+    auto kkv = bwd_dkdv_tc_kernel<D, ROPE>;
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(kdq), C::SMEM_Q, "bwd_dq_tc_kernel set-up")) != ATTN_OK)
+        return s;
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(kkv), C::SMEM_K, "bwd_dkdv_tc_kernel set-up")) != ATTN_OK)
+        return s;
+    const long grid_q = static_cast<long>((Sq + 127) / 128) * B * Hq;
+    const long grid_k = static_cast<long>((Skv + 127) / 128) * B * Hkv;
+    if (grid_q > 2147483647L || grid_k > 2147483647L) return ATTN_ERR_UNSUPPORTED;
+    p.g_f32 = g_f32 ? static_cast<float*>(dq) : nullptr;
+    p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dq);
+    kdq<<<static_cast<unsigned>(grid_q), kBtThreads, C::SMEM_Q, st>>>(tq, tql, tk, tkl, tv, tdo, p);
+    if ((s = launch_status("bwd_dq_tc_kernel")) != ATTN_OK) return s;
+    p.g_f32 = g_f32 ? static_cast<float*>(dk) : nullptr;
+    p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
+    p.g2_f32 = g_f32 ? static_cast<float*>(dv) : nullptr;
+    p.g2_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
+    kkv<<<static_cast<unsigned>(grid_k), kBtThreads, C::SMEM_K, st>>>(tq, tql, tk, tkl, tv, tdo, tl2, tdv, p);
+    return launch_status("bwd_dkdv_tc_kernel");
 }
 
 template <int D, bool ROPE>
@@ -773,6 +869,17 @@ attn_status bwd_impl(const void* q, const void* k, const void* v, const void* o,
     using bf = __nv_bfloat16;
     const bf *qb = static_cast<const bf*>(q), *kb = static_cast<const bf*>(k), *vb = static_cast<const bf*>(v),
              *ob = static_cast<const bf*>(o), *gb = static_cast<const bf*>(dout);
+    if (bwd_tc_eligible(Sq, mk)) {
+        if (D == 64)
+            return rope ? launch_bwd_tc<64, true>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
+                                                  causal, tab, q_pos0, ws, wm, st)
+                        : launch_bwd_tc<64, false>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv,
+                                                   scale, causal, tab, q_pos0, ws, wm, st);
+        return rope ? launch_bwd_tc<128, true>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
+                                               causal, tab, q_pos0, ws, wm, st)
+                    : launch_bwd_tc<128, false>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
+                                                causal, tab, q_pos0, ws, wm, st);
+    }
     if (D == 64)
         return rope ? launch_bwd_mma<64, true>(qb, kb, vb, ob, lse, gb, dq, dk, dv, g_f32, B, Hq, Hkv, Sq, Skv, scale,
                                                causal, tab, q_pos0, ws, wm, st, mk)

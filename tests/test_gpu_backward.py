@@ -53,6 +53,12 @@ CASES = [
       seed=209),
     P("bf16_noncausal_masked_mqa", "bf16", 2, 4, 1, 77, 200, 64, False, 0.125, seed=210),
     P("bf16_causal_sq_gt_skv", "bf16", 1, 2, 2, 150, 90, 64, True, 0.125, seed=211),
+    # shapes the tcgen05 backward takes (unmasked, Sq a multiple of 4): rows with no visible key,
+    # several key and query tiles with ragged ends, MQA, GQA at D=128 with RoPE
+    P("tc_bf16_sq_gt_skv", "bf16", 1, 2, 2, 300, 170, 64, True, 0.125, seed=212),
+    P("tc_bf16_noncausal_mqa", "bf16", 2, 4, 1, 260, 330, 64, False, 0.125, seed=213),
+    P("tc_bf16_d128_gqa_rope", "bf16", 1, 8, 2, 384, 384, 128, True, 0.0884, rope_base=10000.0, seed=214),
+    P("tc_bf16_d64_bottom_right", "bf16", 2, 6, 3, 196, 452, 64, True, 0.125, seed=215),
 ]
 
 
@@ -114,6 +120,39 @@ def test_backward_full_size_c2():
     for name, got, ref in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r)):
         err = _rel_err(got.cpu().numpy().astype(np.float64), ref)
         assert err <= 2e-2, (name, err)
+
+
+@pytest.mark.parametrize("w", [si.C3, si.C5], ids=["c3_gqa_rope", "c5_d128_peaked"])
+def test_backward_full_size_sampled(w):
+    """Full-size GQA 32/8 causal with RoPE (B2 S4096 D64) and long-context D=128 with peaked scores
+    (B1 H16 S16384): the library's bf16 forward and its backward with fp32 gradients, in the
+    configuration bench.py times, against the oracle's exact backward of two (batch, kv head)
+    groups at sampled query rows (first, tile edges, last, random) and keys -- every q head of
+    the group at those rows."""
+    x, g, gb = _inputs(w)
+    q, k, v = (_dev(x, n, w) for n in ("q", "k", "v"))
+    ws = None
+    if w.rope_base > 0:
+        ws = torch.empty(ea.fwd_workspace_bytes(q, k, w.rope_base, w.q_pos0), dtype=torch.uint8, device="cuda")
+    o, lse = ea.attn_fwd_ex(q, k, v, w.scale, w.causal, w.rope_base, w.q_pos0, workspace=ws)
+    dq, dk, dv = ea.attn_bwd(q, k, v, o, lse, bits_to_dev(gb), w.scale, w.causal, w.rope_base, w.q_pos0,
+                             grad_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert ea.read_device_status() == 0
+    dq, dk, dv = (t.cpu().numpy().astype(np.float64) for t in (dq, dk, dv))
+    rng = np.random.default_rng(w.seed)
+    G = w.Hq // w.Hkv
+    for b, kvh in ((0, 0), (w.B - 1, w.Hkv - 1)):
+        rows = np.unique(np.concatenate([[0, 1, 127, 128, w.Sq // 2, w.Sq - 1], rng.integers(0, w.Sq, 6)]))
+        keys = np.unique(np.concatenate([[0, 1, 127, 128, w.Skv // 2, w.Skv - 1], rng.integers(0, w.Skv, 6)]))
+        rq, rk, rv = oracle.attn_bwd_sampled(x["q"], x["k"], x["v"], g, w.scale, w.causal, w.rope_base, w.q_pos0,
+                                             b, kvh, rows, keys)
+        for hg in range(G):
+            err = _rel_err(dq[b, rows, kvh * G + hg], rq[hg])
+            assert err <= 1e-2, ("dq", b, kvh * G + hg, err)
+        assert _rel_err(dk[b, keys, kvh], rk) <= 1e-2, ("dk", b, kvh)
+        assert _rel_err(dv[b, keys, kvh], rv) <= 1e-2, ("dv", b, kvh)
+    assert np.isfinite(dq).all() and np.isfinite(dk).all() and np.isfinite(dv).all()
 
 
 def test_backward_rejects_bad_workspace():
