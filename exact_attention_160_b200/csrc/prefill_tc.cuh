@@ -69,13 +69,22 @@ struct TcCfg {
     static constexpr int Q_TILES = ROPE ? 2 : 1;      // Qh, Ql
     static constexpr int STAGE_BYTES = (K_TILES + 1) * TILE_BYTES;
     static constexpr int Q_BYTES = 2 * Q_TILES * TILE_BYTES;
-    static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES;
+    // D=64: the PV product runs with N = 80, its last 16 columns reading a block of bf16 ones in
+    // shared memory, so column 64 of O accumulates the row sum of the rounded P the MMA used (and
+    // every O correction rescales it with O).  One block serves every stage: the descriptor of
+    // stage s reaches it through its leading-byte offset (ones - V_s).
+    static constexpr bool ONES = (D == 64);
+    static constexpr int N_PV = ONES ? D + 16 : D;
+    static constexpr int ONES_BYTES = ONES ? 128 * 128 : 0;
+    static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES + ONES_BYTES;
     static constexpr int SMEM_BYTES = SMEM_DATA + 1024 /* alignment slack */ + 256 /* barriers */;
-    static_assert(8 * (10 + 3 * STAGES) + 4 <= 256, "barrier area");
-    // TMEM columns: S_t of query tile t at [128 t, 128 t + 128); P_t (bf16, 64 columns) is written
-    // over the first half of S_t once the softmax holds S_t in registers; O_t after both S tiles.
-    static constexpr uint32_t COL_S0 = 0, COL_S1 = 128;
-    static constexpr uint32_t COL_O0 = 256, COL_O1 = 256 + D;
+    static_assert(8 * (12 + 3 * STAGES) + 4 <= 256, "barrier area");
+    // TMEM columns: each query tile keeps S_t and O_t in one half of the 512 columns, S_t first;
+    // P_t (bf16, 64 columns) is written over the first half of S_t once the softmax holds S_t in
+    // registers.  (A P·V product whose A operand and accumulator lie in different halves ran
+    // markedly slower on B200.)
+    static constexpr uint32_t COL_S0 = 0, COL_O0 = 128;
+    static constexpr uint32_t COL_S1 = 256, COL_O1 = 384;
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -127,14 +136,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;                                   // [2][Q_TILES][TILE_BYTES]
     uint8_t* sKV = smem + C::Q_BYTES;                     // [STAGES][(K_TILES+1)][TILE_BYTES]
+    uint8_t* sOnes = sKV + C::STAGES * C::STAGE_BYTES;    // [128 keys][64] bf16 ones (ONES only)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_DATA);
     uint64_t* bar_q_full = bars + 0;
     uint64_t* bar_q_ready = bars + 1;
     uint64_t* bar_s_full = bars + 2;       // [2] S_t(j) computed (commit after its MMAs)
-    uint64_t* bar_p_ready = bars + 4;      // [2] softmax t wrote P_t(j) (and corrected O_t)
-    uint64_t* bar_o_done = bars + 6;       // [2] the last PV_t completed
-    uint64_t* bar_mma_final = bars + 8;    // every MMA of the CTA completed
-    uint64_t* bar_k_full = bars + 10;      // [STAGES]
+    uint64_t* bar_p_ready = bars + 4;      // [2 tiles][2 halves] softmax t wrote keys [64h, 64h+64) of P_t(j)
+    uint64_t* bar_o_done = bars + 8;       // [2] the last PV_t completed
+    uint64_t* bar_mma_final = bars + 10;   // every MMA of the CTA completed
+    uint64_t* bar_k_full = bars + 12;      // [STAGES]
     uint64_t* bar_v_full = bar_k_full + C::STAGES;
     uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_kv_empty + C::STAGES);
@@ -188,7 +198,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         mbar_init(bar_q_ready, 256);   // both softmax warpgroups
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_s_full + i, 1);
-            mbar_init(bar_p_ready + i, 128);
+            mbar_init(bar_p_ready + 2 * i, 128);
+            mbar_init(bar_p_ready + 2 * i + 1, 128);
             mbar_init(bar_o_done + i, 1);
         }
         mbar_init(bar_mma_final, 1);
@@ -208,6 +219,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
+    }
+    if (C::ONES) {
+        // bf16 1.0 everywhere (the swizzle only permutes it), visible to the tensor core
+        uint4* o4 = reinterpret_cast<uint4*>(sOnes);
+        for (int i = tid; i < C::ONES_BYTES / 16; i += kTcThreads) o4[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -276,7 +293,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         // released after PV(j), so both tiles' S(j+1) follow the release.
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
-            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(128, C::N_PV, true);
             constexpr uint32_t hiK = desc_sw128_hi(1024);
             constexpr bool EARLY_S = C::STAGES > 1;
             const int nt0 = tile[0].nkv, nt1 = tile[1].nkv;
@@ -285,7 +302,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             // Descriptors: the high words are constants, the low words advance with the start
             // address (16-byte units), so an MMA costs one add and the instruction itself.
             const uint32_t kvlo0 = desc_sw128_lo(smem_u32(sKV), 16);
-            const uint32_t vlo0 = desc_sw128_lo(smem_u32(sKV) + C::K_TILES * C::TILE_BYTES, C::TILE_BYTES / C::NBOX);
+            // V of stage s: the second 64-wide N block is D's upper half (D=128) or the ones
+            // block (D=64, leading-byte offset ones - V_s)
+            auto v_lo = [&](int s) {
+                const uint32_t va = smem_u32(sKV) + s * C::STAGE_BYTES + C::K_TILES * C::TILE_BYTES;
+                return desc_sw128_lo(va, C::ONES ? smem_u32(sOnes) - va : C::TILE_BYTES / C::NBOX);
+            };
             auto issue_s = [&](int t, int j) {
                 const uint32_t qlo = desc_sw128_lo(smem_u32(sQ + t * C::Q_TILES * C::TILE_BYTES), 16);
                 const uint32_t dS = tmem + (t ? C::COL_S1 : C::COL_S0);
@@ -307,17 +329,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 }
                 mma_commit(bar_s_full + t);
             };
-            auto issue_pv = [&](int t, int j) {
+            // PV_t(j) for keys [64 half, 64 half + 64): issued as soon as the softmax has written
+            // that half of P_t(j), so the product overlaps the exponentials of the other half
+            auto issue_pv_half = [&](int t, int j, int half) {
                 const uint32_t dO = tmem + (t ? C::COL_O1 : C::COL_O0);
                 const uint32_t aP = tmem + (t ? C::COL_S1 : C::COL_S0);
-                const uint32_t vlo = vlo0 + ((j % C::STAGES) * C::STAGE_BYTES >> 4);
+                const uint32_t vlo = v_lo(j % C::STAGES);
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int k4 = 0; k4 < 4; ++k4) {
                     // keys [16kk, 16kk+16): 16 rows of 128 B in every 64-wide D box
+                    const int kk = 4 * half + k4;
                     mma_ts(dO, aP + kk * 8, desc_join(vlo + kk * (2048 >> 4), hiK), idesc_pv,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (j == (t ? nt1 : nt0) - 1) mma_commit(bar_o_done + t);
+                if (half == 1 && j == (t ? nt1 : nt0) - 1) mma_commit(bar_o_done + t);
             };
             auto wait_k = [&](int j) {
                 const bool r = mbar_wait(bar_k_full + j % C::STAGES, (j / C::STAGES) & 1);
@@ -341,11 +366,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 for (int t = 0; t < 2; ++t) {
                     const int n = t ? nt1 : nt0;
                     if (j >= n) continue;
-                    if (ok) {
-                        ok = mbar_wait(bar_p_ready + t, j & 1);
-                        tc_fence_after();
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        if (ok) {
+                            ok = mbar_wait_spin(bar_p_ready + 2 * t + half, j & 1);
+                            tc_fence_after();
+                        }
+                        if (ok) issue_pv_half(t, j, half);
                     }
-                    if (ok) issue_pv(t, j);
                     if (EARLY_S && ok && j + 1 < n) {
                         if (!k_next) ok = wait_k(j + 1);
                         k_next = true;
@@ -435,10 +463,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         const uint32_t tP = tS;    // P_t(j) is written over the first 64 columns of S_t
         for (int j = 0; j < T.nkv; ++j) {
             uint32_t sr[4][32];
-            if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) ok = false;
+            if (ok && !__all_sync(0xffffffffu, mbar_wait_spin(bar_s_full + wg, j & 1))) ok = false;
             tc_fence_after();
             if (!ok) {
-                mbar_arrive(bar_p_ready + wg);   // keep the MMA thread's count; it stops on its own
+                // keep the MMA thread's counts; it stops on its own
+                mbar_arrive(bar_p_ready + 2 * wg);
+                mbar_arrive(bar_p_ready + 2 * wg + 1);
                 continue;
             }
 #pragma unroll
@@ -495,7 +525,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             // PV_t(j) is issued only after this warpgroup's p_ready arrival below.
             if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll
-                for (int cb = 0; cb < D / 32; ++cb) {
+                for (int cb = 0; cb < (C::N_PV + 31) / 32; ++cb) {
                     uint32_t orr[32];
                     tmem_ld32(tO + cb * 32, orr);
                     tmem_wait_ld();
@@ -526,20 +556,29 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     const float p1 = fast_exp2(t1);
                     lt2[e & 3] = f2_add(lt2[e & 3], f2_pack(p0, p1));
                     pk[e] = pack_bf16x2(p0, p1);
-                    lr2[e & 3] = f2_add(lr2[e & 3], f2_pack(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
+                    if (!C::ONES)
+                        lr2[e & 3] = f2_add(lr2[e & 3], f2_pack(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                 }
                 tmem_st16(tP + cb * 16, pk);
+                if (cb == 1) {
+                    // keys [0, 64) of P are in TMEM: the first half of PV may start
+                    tmem_wait_st();
+                    tc_fence_before();
+                    mbar_arrive(bar_p_ready + 2 * wg);
+                }
             }
             {
                 float a, c;
                 f2_unpack(f2_add(f2_add(lt2[0], lt2[1]), f2_add(lt2[2], lt2[3])), a, c);
                 l_run += a + c;
-                f2_unpack(f2_add(f2_add(lr2[0], lr2[1]), f2_add(lr2[2], lr2[3])), a, c);
-                l_mma += a + c;
+                if (!C::ONES) {
+                    f2_unpack(f2_add(f2_add(lr2[0], lr2[1]), f2_add(lr2[2], lr2[3])), a, c);
+                    l_mma += a + c;
+                }
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar_p_ready + wg);
+            mbar_arrive(bar_p_ready + 2 * wg + 1);
         }
 
         // epilogue: O / l -> bf16 or fp32, lse.  The TMEM reads are warp-collective, so every
@@ -551,6 +590,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 tc_fence_after();
             }
             const bool store = qrow < p.Sq;
+            if (C::ONES && have) {
+                // the row sum of the rounded weights, accumulated by the PV MMA in column D of O
+                uint32_t sr1[32];
+                tmem_ld32(tO + D, sr1);
+                tmem_wait_ld();
+                l_mma = __uint_as_float(sr1[0]);
+            }
             const float inv = (have && l_mma > 0.f) ? 1.f / l_mma : 0.f;
             // a key split writes its normalised partial O (fp32) and its logsumexp to its slabs
             float* out_f32 = p.o_f32;
