@@ -592,6 +592,22 @@ def run_gpu(args):
     barrier(dist, device)
 
     peaks, how = load_peaks()
+    if args.backward_only:
+        # the backward of the workload alone (a profiling aid): value = its TFLOP/s
+        w = si.WORKLOADS[args.workload]
+        br = bench_backward_gpu(w, args, torch, ea, dist, device, args.steps)
+        bms = max_over_ranks(br["ms"], dist, device)
+        out = {"metric": "attention backward TFLOP/s", "value": round(whole_job_rate(br["flop"], bms, world) / 1e12, 3),
+               "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+               "ms_per_step": round(bms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+               "dtype": "bf16", "data": "synthetic", "config": {"workload": w.name, "part": "backward"},
+               "roofline": roofline_backward(br["flop"], bms, peaks, how)}
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+        if dist is not None:
+            barrier(dist, device)
+            dist.destroy_process_group()
+        return
     cpu_on = rank == 0 and world == 1 and not args.no_cpu_baseline
     sec_steps = max(5, args.steps // 3)
     w = si.WORKLOADS[args.workload]
@@ -742,6 +758,8 @@ def main(argv=None):
     ap.add_argument("--headline-only", action="store_true",
                     help="time the headline workload only (no per-configuration objects)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only attn_bwd on the workload (a profiling aid; not the benchmark line)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

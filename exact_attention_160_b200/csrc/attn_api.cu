@@ -269,6 +269,7 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     p.mask_bs = mk.bs;
     p.mask_hs = mk.hs;
     p.inv_scale = 1.f / scale;
+    p.mask_vec4 = mk.ptr != nullptr && aligned16(mk.ptr) && Skv % 4 == 0 && mk.bs % 4 == 0 && mk.hs % 4 == 0;
     p.kv_splits = 1;
     if (splits > 1) {
         if (!p.single_tile || splits > kMaxKvSplits || !o_part || !lse_part) return ATTN_ERR_UNSUPPORTED;

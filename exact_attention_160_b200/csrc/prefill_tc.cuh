@@ -104,6 +104,7 @@ struct TcParams {
     const float* mask;        // additive mask on the scaled scores, or null
     long mask_bs, mask_hs;    // its batch and head strides (elements; 0 broadcasts); rows of Skv
     float inv_scale;          // 1 / scale: the mask enters the raw scores as mask / scale
+    int mask_vec4;            // 1: every mask row starts 16-byte aligned (base, strides, Skv multiples of 4)
     int kv_splits;            // >= 1; > 1 (single-tile mode only): each query tile's key tiles are
                               // divided among this many CTAs, which write partials
     float* o_part;            // [kv_splits][B][Sq][Hq][D] fp32 partial O, normalised per split
@@ -480,12 +481,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 // (s * scale + mask) * log2(e) - m then keeps its form
                 const float* mrow = p.mask + b * p.mask_bs + T.h * p.mask_hs + static_cast<long>(qrow) * p.Skv + k0;
                 const int ncol = p.Skv - k0;
+                if (p.mask_vec4 && ncol >= 128) {
+                    // 16-byte loads (mask rows 16-byte aligned): a quarter of the L1 wavefronts
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb)
+                    for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (cb * 32 + e < ncol)
-                            sr[cb][e] = __float_as_uint(__uint_as_float(sr[cb][e]) + __ldg(mrow + cb * 32 + e) * p.inv_scale);
+                        for (int e4 = 0; e4 < 8; ++e4) {
+                            const float4 m4 = __ldg(reinterpret_cast<const float4*>(mrow + cb * 32 + 4 * e4));
+                            const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                            for (int u = 0; u < 4; ++u)
+                                sr[cb][4 * e4 + u] = __float_as_uint(__uint_as_float(sr[cb][4 * e4 + u]) + mm[u] * p.inv_scale);
+                        }
+                } else {
+#pragma unroll
+                    for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (cb * 32 + e < ncol)
+                                sr[cb][e] = __float_as_uint(__uint_as_float(sr[cb][e]) + __ldg(mrow + cb * 32 + e) * p.inv_scale);
+                }
             }
             // mask: keys past Skv, and (causal) keys beyond this row's diagonal
             const long lim_causal = p.causal ? static_cast<long>(qrow) + off_c : static_cast<long>(p.Skv) - 1;
