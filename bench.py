@@ -331,7 +331,9 @@ def bench_prefill_gpu(w: si.Prefill, args, torch, ea, dist, device, steps: int, 
             ea.attn_fwd_masked(q, k, v, mt, w.scale, w.causal, w.rope_base, w.q_pos0, o=o, lse=lse, workspace=ws)
 
     # rope: table + rotated K + prefill; key splits add the combine
-    launches_per_step = (1 if w.rope_base <= 0 else 3) + (1 if splits > 1 else 0)
+    # RoPE: the cos/sin table and (unless K is rotated inside the prefill kernel) the K hi/lo pass
+    rope_launches = 0 if w.rope_base <= 0 else (1 if os.environ.get("ATTN_ROPE_K_FORM") == "fused" else 2)
+    launches_per_step = 1 + rope_launches + (1 if splits > 1 else 0)
     with ClockSampler(device.index) as clk:
         ms = time_steps(step, steps, args.warmup, flush, torch, dist, device)
     status = ea.read_device_status()
@@ -670,6 +672,23 @@ def run_gpu(args):
         e["what"] = "attn_fwd_masked on C2's shapes: shared fp32 [Sq, Skv] additive mask plus the causal mask"
         e["roofline"]["traffic"] = None
         configs["c2_masked_shared_mask"] = e
+        # C3 with K rotated inside the prefill kernel instead of by the K hi/lo pre-pass (the two
+        # RoPE forms side by side; the pre-pass is the library's default)
+        prev = os.environ.get("ATTN_ROPE_K_FORM")
+        os.environ["ATTN_ROPE_K_FORM"] = "fused"
+        try:
+            cr = bench_prefill_gpu(si.C3, args, torch, ea, dist, device, sec_steps)
+        finally:
+            if prev is None:
+                del os.environ["ATTN_ROPE_K_FORM"]
+            else:
+                os.environ["ATTN_ROPE_K_FORM"] = prev
+        cr["ms"] = max_over_ranks(cr["ms"], dist, device)
+        e = prefill_entry(si.C3, cr, peaks, how, world, None)
+        e["what"] = ("C3 with RoPE on K applied inside the prefill kernel (ATTN_ROPE_K_FORM=fused) instead of "
+                     "the K hi/lo pre-pass; same oracle as C3")
+        e["roofline"]["traffic"] = None
+        configs["c3_rope_k_fused_form"] = e
         if w.name != si.C4.name:
             dec = bench_decode_gpu(si.C4, args, torch, ea, dist, device, max(5, args.steps // 2))
             dms = max_over_ranks(dec["ms"], dist, device)

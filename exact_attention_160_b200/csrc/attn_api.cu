@@ -5,6 +5,7 @@
 #include <math.h>
 #include <stdint.h>
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -202,6 +203,18 @@ int fwd_kv_splits(int B, int Hq, int Sq, int Skv, attn_dtype dtype) {
     return n >= 2 ? static_cast<int>(n) : 1;
 }
 
+// RoPE form of the bf16 forward: K rotated once beforehand into hi + lo halves that every CTA
+// then reads (the default), or rotated inside the prefill kernel by two warps of each CTA as its
+// tiles land (ATTN_ROPE_K_FORM=fused in the environment, read at every call).  Every K tile is
+// read by about ceil(Sq / 128) * G / 2 CTAs; the in-kernel form repeats its rotation that many
+// times and, measured on B200, is slower on every shape tried (GQA 32/8 causal, B2 S4096 D64:
+// 648 vs 359 us; Sq 128 against Skv 8192: 105 vs 75 us), because two warps rotating 128 keys per
+// tile fall behind the tile pipeline.  It is kept for that comparison.
+bool rope_k_fused() {
+    const char* f = getenv("ATTN_ROPE_K_FORM");
+    return f != nullptr && strcmp(f, "fused") == 0;
+}
+
 // Workspace of attn_fwd_ex: with RoPE the cos/sin table and the rotated K as hi/lo bf16 halves;
 // with key splits the fp32 partial O and logsumexp of every split.
 struct ExWorkspace {
@@ -234,15 +247,14 @@ ExWorkspace ex_workspace(int B, int Hq, int Hkv, int Sq, int Skv, int D, attn_dt
     return w;
 }
 
-template <int D, bool ROPE>
+template <int D, int ROPE>
 attn_status launch_tc(const void* q, const void* k, const void* klo, const void* v, void* o, bool o_f32, float* lse,
                       int B, int Hq, int Hkv, int Sq, int Skv, float scale, int causal, const float2* tab, int q_pos0,
                       cudaStream_t st, MaskArg mk, int splits, float* o_part, float* lse_part) {
     CUtensorMap tq, tk, tkl, tv;
     if (!make_tmap_bshd(&tq, q, B, Sq, Hq, D) || !make_tmap_bshd(&tk, k, B, Skv, Hkv, D) ||
-        !make_tmap_bshd(&tv, v, B, Skv, Hkv, D) || !make_tmap_bshd(&tkl, ROPE ? klo : k, B, Skv, Hkv, D))
+        !make_tmap_bshd(&tv, v, B, Skv, Hkv, D) || !make_tmap_bshd(&tkl, ROPE == kRopeKSplit ? klo : k, B, Skv, Hkv, D))
         return ATTN_ERR_CUDA;   // g_last_error set by make_tmap_bshd
-    using C = TcCfg<D, ROPE>;
     TcParams p{};
     p.o = o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o);
     p.o_f32 = o_f32 ? static_cast<float*>(o) : nullptr;
@@ -281,12 +293,13 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     if (grid > 2147483647L) return ATTN_ERR_UNSUPPORTED;
     // the masked kernel is a separate instantiation, so the unmasked one carries no mask code
     auto kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true> : prefill_tc_kernel<D, ROPE, false>;
+    const int smem_bytes = TcCfg<D, ROPE>::SMEM_BYTES;
     // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds fewer
     // than the split asks for would stall in setmaxnreg.inc, so such a build is refused.
-    attn_status ps = prepare_kernel(reinterpret_cast<const void*>(kern), C::SMEM_BYTES, "prefill_tc_kernel set-up",
+    attn_status ps = prepare_kernel(reinterpret_cast<const void*>(kern), smem_bytes, "prefill_tc_kernel set-up",
                                     kTcLaunchRegsMin);
     if (ps != ATTN_OK) return ps;
-    kern<<<static_cast<unsigned>(grid), kTcThreads, C::SMEM_BYTES, st>>>(tq, tk, tkl, tv, p);
+    kern<<<static_cast<unsigned>(grid), kTcThreads, smem_bytes, st>>>(tq, tk, tkl, tv, p);
     attn_status s = launch_status("prefill_tc_kernel");
     if (s != ATTN_OK || p.kv_splits == 1) return s;
     // merge of the key splits, a programmatic dependent launch (it waits for the split grid)
@@ -364,21 +377,36 @@ attn_status fwd_impl(const void* q, const void* k, const void* v, void* o, float
                        : launch_f32<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab, q_pos0, st, mk);
     }
     if (!rope) {
-        return D == 64 ? launch_tc<64, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
+        return D == 64 ? launch_tc<64, kRopeNone>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
                                               nullptr, 0, st, mk, splits, o_part, lse_part)
-                       : launch_tc<128, false>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
+                       : launch_tc<128, kRopeNone>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
                                                nullptr, 0, st, mk, splits, o_part, lse_part);
+    }
+    if (rope_k_fused()) {
+        // K rotated inside the prefill kernel as its tiles land
+        return D == 64 ? launch_tc<64, kRopeKFused>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal,
+                                                    tab, q_pos0, st, mk, splits, o_part, lse_part)
+                       : launch_tc<128, kRopeKFused>(q, k, nullptr, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale,
+                                                     causal, tab, q_pos0, st, mk, splits, o_part, lse_part);
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     uint32_t* khi = reinterpret_cast<uint32_t*>(ws + w.khi_off);
     uint32_t* klo = reinterpret_cast<uint32_t*>(ws + w.klo_off);
     const long npairs = static_cast<long>(B) * Skv * Hkv * (D / 2);
-    rope_split_kv_kernel<<<static_cast<unsigned>((npairs + 255) / 256 < 148 * 64 ? (npairs + 255) / 256 : 148 * 64), 256,
-                           0, st>>>(static_cast<const uint32_t*>(k), khi, klo, tab, npairs, Skv, Hkv, D);
+    const long nchunks = npairs / 4;
+    if (D % 8 == 0 && aligned16(k) && nchunks < (1L << 30)) {
+        rope_split_kv_vec_kernel<<<static_cast<unsigned>((nchunks + 255) / 256 < 148 * 32 ? (nchunks + 255) / 256 : 148 * 32),
+                                   256, 0, st>>>(static_cast<const uint4*>(k), reinterpret_cast<uint4*>(khi),
+                                                 reinterpret_cast<uint4*>(klo), reinterpret_cast<const float4*>(tab),
+                                                 static_cast<int>(nchunks), Skv, Hkv, D);
+    } else {
+        rope_split_kv_kernel<<<static_cast<unsigned>((npairs + 255) / 256 < 148 * 64 ? (npairs + 255) / 256 : 148 * 64),
+                               256, 0, st>>>(static_cast<const uint32_t*>(k), khi, klo, tab, npairs, Skv, Hkv, D);
+    }
     if ((s = launch_status("rope_split_kv_kernel")) != ATTN_OK) return s;
-    return D == 64 ? launch_tc<64, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
+    return D == 64 ? launch_tc<64, kRopeKSplit>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
                                          q_pos0, st, mk, splits, o_part, lse_part)
-                   : launch_tc<128, true>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
+                   : launch_tc<128, kRopeKSplit>(q, khi, klo, v, o, o_f32, lse, B, Hq, Hkv, Sq, Skv, scale, causal, tab,
                                           q_pos0, st, mk, splits, o_part, lse_part);
 }
 

@@ -54,9 +54,13 @@ constexpr int kRegsControl = 72;
 constexpr int kRegsSoftmax = 208;
 constexpr int kTcLaunchRegsMin = (128 * kRegsControl + 256 * kRegsSoftmax + kTcThreads - 1) / kTcThreads;
 constexpr float kRescaleThreshold = 8.0f;
+// RoPE forms of the kernel: none; K rotated beforehand into hi + lo halves (rope_split_kv_kernel);
+// K loaded as it is and rotated into hi + lo halves in shared memory by the two idle warps of the
+// control warpgroup (warps 2 and 3) while the ring runs ahead.
+constexpr int kRopeNone = 0, kRopeKSplit = 1, kRopeKFused = 2;
 constexpr float kLn2 = 0.69314718055994531f;
 
-template <int D, bool ROPE>
+template <int D, int ROPE>
 struct TcCfg {
     static constexpr int BM = 128;                    // query rows per tile
     static constexpr int BN = 128;                    // keys per KV tile
@@ -78,7 +82,7 @@ struct TcCfg {
     static constexpr int ONES_BYTES = ONES ? 128 * 128 : 0;
     static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES + ONES_BYTES;
     static constexpr int SMEM_BYTES = SMEM_DATA + 1024 /* alignment slack */ + 256 /* barriers */;
-    static_assert(8 * (12 + 3 * STAGES) + 4 <= 256, "barrier area");
+    static_assert(8 * (12 + 4 * STAGES) + 4 <= 256, "barrier area");
     // TMEM columns: each query tile keeps S_t and O_t in one half of the 512 columns, S_t first;
     // P_t (bf16, 64 columns) is written over the first half of S_t once the softmax holds S_t in
     // registers.  (A P·V product whose A operand and accumulator lie in different halves ran
@@ -127,7 +131,7 @@ __device__ __forceinline__ int tc_kv_tiles(const TcParams& p, int r0) {
     return n < nkv_all ? static_cast<int>(n) : nkv_all;
 }
 
-template <int D, bool ROPE, bool MASK>
+template <int D, int ROPE, bool MASK>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
@@ -148,7 +152,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     uint64_t* bar_k_full = bars + 12;      // [STAGES]
     uint64_t* bar_v_full = bar_k_full + C::STAGES;
     uint64_t* bar_kv_empty = bar_v_full + C::STAGES;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_kv_empty + C::STAGES);
+    uint64_t* bar_k_rot = bar_kv_empty + C::STAGES;   // [STAGES] K(j) rotated in place (kRopeKFused)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_k_rot + C::STAGES);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -208,6 +213,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             mbar_init(bar_k_full + s, 1);
             mbar_init(bar_v_full + s, 1);
             mbar_init(bar_kv_empty + s, 1);   // one commit from the MMA thread
+            mbar_init(bar_k_rot + s, 64);     // the two rotating warps
         }
         mbar_fence_init();
     }
@@ -215,7 +221,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
-        if (ROPE) tma_prefetch_desc(&tm_klo);
+        if (ROPE == kRopeKSplit) tma_prefetch_desc(&tm_klo);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -259,11 +265,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 if (!mbar_wait(bar_kv_empty + s, ph ^ 1)) break;
                 issued = j + 1;
                 uint8_t* st = sKV + s * C::STAGE_BYTES;
-                mbar_arrive_expect_tx(bar_k_full + s, C::K_TILES * C::TILE_BYTES);
+                // kRopeKFused: the raw K tile lands in the Kh slot and is rotated there
+                mbar_arrive_expect_tx(bar_k_full + s, (ROPE == kRopeKSplit ? 2 : 1) * C::TILE_BYTES);
                 for (int bx = 0; bx < C::NBOX; ++bx) {
                     tma_load_4d(&tm_k, bar_k_full + s, st + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
                                 (kv0 + j) * 128, b, pol_kv);
-                    if (ROPE)
+                    if (ROPE == kRopeKSplit)
                         tma_load_4d(&tm_klo, bar_k_full + s, st + C::TILE_BYTES + bx * (C::TILE_BYTES / C::NBOX),
                                     bx * 64, kvh, (kv0 + j) * 128, b, pol_kv);
                 }
@@ -346,7 +353,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 if (half == 1 && j == (t ? nt1 : nt0) - 1) mma_commit(bar_o_done + t);
             };
             auto wait_k = [&](int j) {
-                const bool r = mbar_wait(bar_k_full + j % C::STAGES, (j / C::STAGES) & 1);
+                uint64_t* kb = ROPE == kRopeKFused ? bar_k_rot : bar_k_full;
+                const bool r = mbar_wait(kb + j % C::STAGES, (j / C::STAGES) & 1);
                 tc_fence_after();
                 return r;
             };
@@ -397,6 +405,61 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             // every MMA issued above must be complete before tensor memory is released
             mma_commit(bar_mma_final);
             mbar_wait(bar_mma_final, 0);
+        }
+      } else if (ROPE == kRopeKFused) {
+        // =============================== K rotation (warps 2, 3) ========================
+        // Each K tile is rotated in place as soon as it lands: key r of the tile (position
+        // (kv0 + j) * 128 + r, as for the pre-rotated form) is split into hi = bf16(k') in the Kh
+        // slot and lo = bf16(k' - hi) in the Kl slot; thread u handles keys u and u + 64.  The
+        // pairs (2i, 2i+1) share a 16-byte chunk, which the 128-byte swizzle moves whole.
+        const int u = (warp - 2) * 32 + lane;
+        for (int j = 0; j < nkv; ++j) {
+            const int s = j % C::STAGES;
+            if (!mbar_wait(bar_k_full + s, (j / C::STAGES) & 1)) break;
+            uint8_t* kh = sKV + s * C::STAGE_BYTES;
+            uint8_t* kl = kh + C::TILE_BYTES;
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int r = u + 64 * rr;
+                const long pos = static_cast<long>(kv0 + j) * 128 + r;
+                if (pos < p.Skv) {
+                    const float4* tab4 = reinterpret_cast<const float4*>(p.rope_tab + pos * (D / 2));
+#pragma unroll 1
+                    for (int bx = 0; bx < C::NBOX; ++bx) {
+#pragma unroll 2
+                        for (int ck = 0; ck < 8; ++ck) {
+                            const uint32_t o = bx * (C::TILE_BYTES / C::NBOX) + sw128_offset(r, ck);
+                            const uint4 w = *reinterpret_cast<const uint4*>(kh + o);
+                            const float4 c01 = __ldg(tab4 + bx * 16 + ck * 2);
+                            const float4 c23 = __ldg(tab4 + bx * 16 + ck * 2 + 1);
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                            const float2 cs[4] = {make_float2(c01.x, c01.y), make_float2(c01.z, c01.w),
+                                                  make_float2(c23.x, c23.y), make_float2(c23.z, c23.w)};
+                            uint32_t hh[4], ll[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float x0 = bf16lo_to_f32(ww[e]), x1 = bf16hi_to_f32(ww[e]);
+                                const float y0 = x0 * cs[e].x - x1 * cs[e].y;
+                                const float y1 = x0 * cs[e].y + x1 * cs[e].x;
+                                hh[e] = pack_bf16x2(y0, y1);
+                                ll[e] = pack_bf16x2(y0 - bf16lo_to_f32(hh[e]), y1 - bf16hi_to_f32(hh[e]));
+                            }
+                            *reinterpret_cast<uint4*>(kh + o) = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+                            *reinterpret_cast<uint4*>(kl + o) = make_uint4(ll[0], ll[1], ll[2], ll[3]);
+                        }
+                    }
+                } else {
+                    // keys past Skv: TMA zero-filled Kh; Kl gets zeros too
+#pragma unroll
+                    for (int bx = 0; bx < C::NBOX; ++bx)
+#pragma unroll
+                        for (int ck = 0; ck < 8; ++ck)
+                            *reinterpret_cast<uint4*>(kl + bx * (C::TILE_BYTES / C::NBOX) + sw128_offset(r, ck)) =
+                                make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();   // generic-proxy writes -> the tensor core's reads
+            mbar_arrive(bar_k_rot + s);
         }
       }
     } else {

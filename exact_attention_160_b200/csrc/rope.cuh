@@ -12,6 +12,8 @@
 
 namespace attn {
 
+constexpr int kRopeMaxHalf = 128;   // pairs whose denominators rope_table_kernel caches
+
 __device__ __forceinline__ double rope_theta(double pos, int pair, int D, double base) {
     return pos / pow(base, 2.0 * static_cast<double>(pair) / static_cast<double>(D));
 }
@@ -20,7 +22,13 @@ __device__ __forceinline__ double rope_theta(double pos, int pair, int D, double
 // dim whose frequencies are used (the true dim when the vectors are zero-padded to D); pairs at
 // or past Dfreq/2 are padding and get the identity (1, 0).
 __global__ void rope_table_kernel(float2* __restrict__ tab, int P, int D, double base, int Dfreq) {
+    // base^(2i/Dfreq) once per block (the same pow and division as rope_theta, so the table is
+    // bit-identical to evaluating rope_theta per entry)
+    __shared__ double denom[kRopeMaxHalf];
     const int half = D / 2;
+    for (int i = threadIdx.x; i < half && i < kRopeMaxHalf; i += blockDim.x)
+        denom[i] = pow(base, 2.0 * static_cast<double>(i) / static_cast<double>(Dfreq));
+    __syncthreads();
     const long n = static_cast<long>(P) * half;
     for (long idx = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; idx < n;
          idx += static_cast<long>(gridDim.x) * blockDim.x) {
@@ -31,7 +39,8 @@ __global__ void rope_table_kernel(float2* __restrict__ tab, int P, int D, double
             continue;
         }
         double s, c;
-        sincos(rope_theta(static_cast<double>(p), i, Dfreq, base), &s, &c);
+        const double th = i < kRopeMaxHalf ? static_cast<double>(p) / denom[i] : rope_theta(static_cast<double>(p), i, Dfreq, base);
+        sincos(th, &s, &c);
         tab[idx] = make_float2(static_cast<float>(c), static_cast<float>(s));
     }
 }
@@ -115,6 +124,35 @@ __global__ void rope_split_kv_kernel(const uint32_t* __restrict__ k, uint32_t* _
         const uint32_t hi = pack_bf16x2(y0, y1);
         khi[idx] = hi;
         klo[idx] = pack_bf16x2(y0 - bf16lo_to_f32(hi), y1 - bf16hi_to_f32(hi));
+    }
+}
+
+// The same split with 16-byte accesses: thread = 8 consecutive elements (4 pairs) of one key
+// row, with 32-bit index arithmetic.  Needs k, khi, klo and tab 16-byte aligned, D a multiple of
+// 8 and rows * D / 8 < 2^31.
+__global__ void rope_split_kv_vec_kernel(const uint4* __restrict__ k, uint4* __restrict__ khi, uint4* __restrict__ klo,
+                                         const float4* __restrict__ tab, int nchunks, int S, int Hkv, int D) {
+    const int cpr = D / 8;   // chunks per row
+    for (int idx = blockIdx.x * blockDim.x + threadIdx.x; idx < nchunks; idx += gridDim.x * blockDim.x) {
+        const int row = idx / cpr, c = idx - row * cpr;   // row = (b*S + j)*Hkv + kvh
+        const int j = (row / Hkv) % S;
+        const float4* t = tab + (static_cast<long>(j) * (D / 2) + 4 * c) / 2;
+        const float4 c01 = __ldg(t), c23 = __ldg(t + 1);
+        const uint4 w = k[idx];
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+        const float cs[8] = {c01.x, c01.y, c01.z, c01.w, c23.x, c23.y, c23.z, c23.w};
+        uint32_t hh[4], ll[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = bf16lo_to_f32(ww[e]), x1 = bf16hi_to_f32(ww[e]);
+            const float cr = cs[2 * e], sr = cs[2 * e + 1];
+            const float y0 = x0 * cr - x1 * sr;
+            const float y1 = x0 * sr + x1 * cr;
+            hh[e] = pack_bf16x2(y0, y1);
+            ll[e] = pack_bf16x2(y0 - bf16lo_to_f32(hh[e]), y1 - bf16hi_to_f32(hh[e]));
+        }
+        khi[idx] = make_uint4(hh[0], hh[1], hh[2], hh[3]);
+        klo[idx] = make_uint4(ll[0], ll[1], ll[2], ll[3]);
     }
 }
 
