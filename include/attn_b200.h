@@ -115,7 +115,10 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
  * live there); attn_fwd and a NULL workspace run unsplit.  The result is the same attention
  * up to rounding.
  * bf16 path: rotated Q and K are carried as a pair of bf16 values (hi + lo) each, so the
- * rotated operands keep about 16 mantissa bits; QK^T runs as three bf16 MMA chains.
+ * rotated operands keep about 16 mantissa bits; QK^T runs as three bf16 MMA chains.  K is
+ * rotated once per call by a pre-pass into the workspace; with ATTN_ROPE_K_FORM=fused in the
+ * environment (read at every call) the prefill kernel rotates each K tile in shared memory
+ * instead -- the same result up to rounding, kept as the measured alternative (it is slower).
  */
 attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                         int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal,
