@@ -51,6 +51,12 @@ struct BtCfg {
     // first accumulator (dQ or dV), [256,384) dP or dP^T (dS^T over its first 64 in dkdv),
     // [384, 384+D) dK.  Each ts product's A operand and accumulator share a half of TMEM.
     static constexpr uint32_t COL_S = 0, COL_ACC = 128, COL_DP = 256, COL_DK = 384;
+    // dq kernel: S and dP in the first half; dQ and two dS buffers (dS(j) in buffer j % 2) in the
+    // second, so S(j+1) and dP(j+1) can be computed while the compute warps still form dS(j).
+    // (The dQ product's A operand, dS, and its accumulator share the second half.)
+    static constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_ACC = 256, DQ_COL_DS = 384;
+    // the pipelined order issues S(j+1) before dQ(j) releases stage j, so it needs two stages
+    static constexpr bool DQ_PIPE = STAGES_Q >= 2;
 };
 
 struct BtParams {
@@ -166,7 +172,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
     uint64_t* bar_k_full = bars + 5;        // [ST]
     uint64_t* bar_v_full = bar_k_full + ST;
     uint64_t* bar_empty = bar_v_full + ST;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_empty + ST);
+    uint64_t* bar_s_free = bar_empty + ST;  // the compute warps hold S(j), dP(j) in registers
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_s_free + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nqt = (p.Sq + 127) / 128;
@@ -194,6 +201,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
             mbar_init(bar_v_full + s, 1);
             mbar_init(bar_empty + s, 1);
         }
+        mbar_init(bar_s_free, 256);
         mbar_fence_init();
     }
     if (warp == 1) {
@@ -204,6 +212,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    constexpr uint32_t cS = C::DQ_PIPE ? C::DQ_COL_S : C::COL_S;
+    constexpr uint32_t cDP = C::DQ_PIPE ? C::DQ_COL_DP : C::COL_DP;
+    constexpr uint32_t cACC = C::DQ_PIPE ? C::DQ_COL_ACC : C::COL_ACC;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -242,15 +253,20 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
     } else if (warp == 1) {
         if (lane == 0) {
             // per key tile j:  S(j) = Q K_j^T, dP(j) = dO V_j^T -> s_full; the compute warps
-            // write dS(j) over S -> p_ready; dQ += dS(j) K_j; stage free; S(j+1), dP(j+1)
+            // write dS(j) -> p_ready; dQ += dS(j) K_j; stage free.  Pipelined (two or more
+            // stages): S(j+1), dP(j+1) are issued as soon as the compute warps have S(j), dP(j) in
+            // registers (s_free), before dQ(j), so the tensor core computes them while dS(j) is
+            // formed; dS(j) goes to its own buffer (j % 2), which dQ(j-2) -- issued before S(j),
+            // hence complete by s_full(j) -- has finished reading.  Otherwise dS(j) is written
+            // over S and S(j+1) follows dQ(j).
             bool ok = mbar_wait(bar_fix, 0);
             tc_fence_after();
             const uint32_t uQ = smem_u32(sQ), uG = smem_u32(sG);
             auto stage = [&](int j) { return smem_u32(sKV + (j % ST) * C::STAGE_Q); };
             auto issue_scores = [&](int j) {
                 const uint32_t k = stage(j);
-                bt_issue_scores<D, ROPE>(tmem + C::COL_S, uQ, uQ + C::TILE, k, k + C::TILE);
-                bt_issue_scores<D, false>(tmem + C::COL_DP, uG, uG, k + (C::NT - 1) * C::TILE, 0);
+                bt_issue_scores<D, ROPE>(tmem + cS, uQ, uQ + C::TILE, k, k + C::TILE);
+                bt_issue_scores<D, false>(tmem + cDP, uG, uG, k + (C::NT - 1) * C::TILE, 0);
                 mma_commit(bar_s_full);
             };
             auto wait_kv = [&](int j) {
@@ -263,13 +279,22 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
                 if (ok) issue_scores(0);
             }
             for (int j = 0; j < nkv; ++j) {
+                if (C::DQ_PIPE && j + 1 < nkv) {
+                    if (ok) {
+                        ok = mbar_wait(bar_s_free, j & 1);
+                        tc_fence_after();
+                    }
+                    if (ok) ok = wait_kv(j + 1);
+                    if (ok) issue_scores(j + 1);
+                }
                 if (ok) {
                     ok = mbar_wait(bar_p_ready, j & 1);
                     tc_fence_after();
                 }
-                if (ok) bt_issue_acc<D, ROPE>(tmem + C::COL_ACC, tmem + C::COL_S, stage(j), j == 0);
+                const uint32_t aDS = C::DQ_PIPE ? tmem + C::DQ_COL_DS + 64 * (j & 1) : tmem + C::COL_S;
+                if (ok) bt_issue_acc<D, ROPE>(tmem + cACC, aDS, stage(j), j == 0);
                 mma_commit(bar_empty + j % ST);
-                if (ok && j + 1 < nkv) {
+                if (!C::DQ_PIPE && ok && j + 1 < nkv) {
                     ok = wait_kv(j + 1);
                     if (ok) issue_scores(j + 1);
                 }
@@ -283,9 +308,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
         const int row = (warp & 3) * 32 + lane;
         const int qrow = i * 128 + row;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + C::COL_S + 64 * wg;
-        const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * wg;
-        const uint32_t tDS = tmem + lane_base + C::COL_S + 32 * wg;
+        const uint32_t tS = tmem + lane_base + cS + 64 * wg;
+        const uint32_t tP = tmem + lane_base + cDP + 64 * wg;
         const long lrow = (static_cast<long>(b) * p.Hq + h) * p.Sq + qrow;
         const bool live = qrow < p.Sq;
         const float l2 = live ? p.lse2[lrow] : INFINITY;
@@ -307,7 +331,15 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
                 tmem_ld32(tP + 32, dr[1]);
                 tmem_wait_ld();
             }
-            compute_sync();
+            const uint32_t tDS = C::DQ_PIPE ? tmem + lane_base + C::DQ_COL_DS + 64 * (j & 1) + 32 * wg
+                                            : tmem + lane_base + C::COL_S + 32 * wg;
+            if (C::DQ_PIPE) {
+                // S(j), dP(j) are in registers: the MMA thread may overwrite them with S(j+1), dP(j+1)
+                tc_fence_before();
+                mbar_arrive(bar_s_free);
+            } else {
+                compute_sync();   // dS(j) is written over S(j), which the other warpgroup reads
+            }
             if (ok) {
                 const long k0 = static_cast<long>(j) * 128 + 64 * wg;   // first key of this half
                 const bool edge = k0 + 63 > lim;
@@ -350,7 +382,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
         }
         uint32_t acc[D / 2];
         if (have) {
-            tmem_ld_half<D>(tmem + lane_base + C::COL_ACC + wg * (D / 2), acc);
+            tmem_ld_half<D>(tmem + lane_base + cACC + wg * (D / 2), acc);
         } else {
 #pragma unroll
             for (int e = 0; e < D / 2; ++e) acc[e] = 0u;
