@@ -655,9 +655,9 @@ attn_status launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     p.scale_log2 = scale * 1.4426950408889634f;
     auto kdq = bwd_dq_tc_kernel<D, ROPE>;
     auto kkv = bwd_dkdv_tc_kernel<D, ROPE>;
-    if ((s = prepare_kernel(reinterpret_cast<const void*>(kdq), C::SMEM_Q, "bwd_dq_tc_kernel set-up")) != ATTN_OK)
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(kdq), C::SMEM_Q, "bwd_dq_tc_kernel set-up", kBtLaunchRegsMin)) != ATTN_OK)
         return s;
-    if ((s = prepare_kernel(reinterpret_cast<const void*>(kkv), C::SMEM_K, "bwd_dkdv_tc_kernel set-up")) != ATTN_OK)
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(kkv), C::SMEM_K, "bwd_dkdv_tc_kernel set-up", kBtLaunchRegsMin)) != ATTN_OK)
         return s;
     const long grid_q = static_cast<long>((Sq + 127) / 128) * B * Hq;
     const long grid_k = static_cast<long>((Skv + 127) / 128) * B * Hkv;

@@ -28,6 +28,13 @@
 namespace attn {
 
 constexpr int kBtThreads = 384;
+// Register split (setmaxnreg): the TMA/MMA warpgroup gives registers up, the two compute
+// warpgroups (which hold S and dP rows, 128 values a thread) take them.  The launch must hold
+// 128 * 72 + 256 * 216 registers (168 a thread); the host checks the compiled count.  Per
+// sub-partition: (72 + 2 * 216) * 32 = 16128 <= 16384.
+constexpr int kBtRegsControl = 72;
+constexpr int kBtRegsCompute = 216;
+constexpr int kBtLaunchRegsMin = (128 * kBtRegsControl + 256 * kBtRegsCompute + kBtThreads - 1) / kBtThreads;
 
 template <int D, bool ROPE>
 struct BtCfg {
@@ -216,7 +223,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
     constexpr uint32_t cDP = C::DQ_PIPE ? C::DQ_COL_DP : C::COL_DP;
     constexpr uint32_t cACC = C::DQ_PIPE ? C::DQ_COL_ACC : C::COL_ACC;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      setmaxnreg_dec<kBtRegsControl>();
+      if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_q = l2_policy_evict_first();
             const uint64_t pol_kv = l2_policy_evict_last();
@@ -303,7 +312,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
             mma_commit(bar_final);
             mbar_wait(bar_final, 0);
         }
-    } else if (warp >= 4) {
+      }
+    } else {
+        setmaxnreg_inc<kBtRegsCompute>();
         const int wg = (warp - 4) >> 2;
         const int row = (warp & 3) * 32 + lane;
         const int qrow = i * 128 + row;
@@ -467,7 +478,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 0) {
+    if (warp < 4) {
+      setmaxnreg_dec<kBtRegsControl>();
+      if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_kv = l2_policy_evict_first();
             const uint64_t pol_q = l2_policy_evict_last();
@@ -541,7 +554,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
             mma_commit(bar_final);
             mbar_wait(bar_final, 0);
         }
-    } else if (warp >= 4) {
+      }
+    } else {
+        setmaxnreg_inc<kBtRegsCompute>();
         const int wg = (warp - 4) >> 2;
         const int row = (warp & 3) * 32 + lane;
         const int key = j * 128 + row;
