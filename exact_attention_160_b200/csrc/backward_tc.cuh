@@ -353,7 +353,16 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
             }
             if (ok) {
                 const long k0 = static_cast<long>(j) * 128 + 64 * wg;   // first key of this half
-                const bool edge = k0 + 63 > lim;
+                // keys past this row's causal limit or past Skv: S = -inf, so P = 0 and dS = 0.  A
+                // separate pass, taken only by warps with such a key, keeps the loop below free of
+                // per-element checks.
+                if (__any_sync(0xffffffffu, k0 + 63 > lim)) {
+#pragma unroll
+                    for (int cb = 0; cb < 2; ++cb)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (k0 + cb * 32 + e > lim) sr[cb][e] = __float_as_uint(-INFINITY);
+                }
                 uint32_t pk[2][16];
 #pragma unroll
                 for (int cb = 0; cb < 2; ++cb) {
@@ -365,11 +374,6 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
                                   p0, p1);
                         p0 = fast_exp2(p0);
                         p1 = fast_exp2(p1);
-                        if (edge) {
-                            const long kk = k0 + cb * 32 + 2 * e;
-                            if (kk > lim) p0 = 0.f;
-                            if (kk + 1 > lim) p1 = 0.f;
-                        }
                         const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[cb][2 * e]), __uint_as_float(dr[cb][2 * e + 1])),
                                                   ndvx2);
                         float d0, d1;
@@ -589,7 +593,17 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
                 const long q0 = static_cast<long>(i) * 128 + 64 * wg;
                 // visible iff q < Sq and (not causal or q >= key - off)
                 const long qmin = p.causal ? static_cast<long>(key) - off_c : 0;
-                const bool edge = q0 < qmin || q0 + 63 >= p.Sq;
+                // hidden queries: S^T = -inf, so P^T = 0 and dS^T = 0 (a separate pass, taken only
+                // by warps that have one, keeps the loop below free of per-element checks)
+                if (__any_sync(0xffffffffu, q0 < qmin || q0 + 63 >= p.Sq)) {
+#pragma unroll
+                    for (int cb = 0; cb < 2; ++cb)
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const long qq = q0 + cb * 32 + e;
+                            if (qq < qmin || qq >= p.Sq) sr[cb][e] = __float_as_uint(-INFINITY);
+                        }
+                }
                 // 16 query columns at a time, stored as soon as they are formed (few live registers)
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
@@ -608,11 +622,6 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
                                   p0, p1);
                         p0 = fast_exp2(p0);
                         p1 = fast_exp2(p1);
-                        if (edge) {
-                            const long qq = q0 + 2 * idx;
-                            if (qq < qmin || qq >= p.Sq) p0 = 0.f;
-                            if (qq + 1 < qmin || qq + 1 >= p.Sq) p1 = 0.f;
-                        }
                         const uint64_t t = f2_add(f2_pack(__uint_as_float(dr[cb][el]), __uint_as_float(dr[cb][el + 1])),
                                                   f2_pack(-da, -db));
                         float d0, d1;
