@@ -64,6 +64,12 @@ struct BtCfg {
     static constexpr uint32_t DQ_COL_S = 0, DQ_COL_DP = 128, DQ_COL_ACC = 256, DQ_COL_DS = 384;
     // the pipelined order issues S(j+1) before dQ(j) releases stage j, so it needs two stages
     static constexpr bool DQ_PIPE = STAGES_Q >= 2;
+    // dkdv kernel at D = 64: P^T and dS^T get buffers of their own (first half: S^T, dV, P^T;
+    // second half: dP^T, dK, dS^T), so S^T(i+1) and dP^T(i+1) can be computed while the compute
+    // warps still form P^T(i) and dS^T(i).  At D = 128 the accumulators leave no room.
+    static constexpr bool KV_PIPE = D == 64 && STAGES_K >= 2;
+    static constexpr uint32_t KV_COL_S = 0, KV_COL_DV = 128, KV_COL_PT = 192;
+    static constexpr uint32_t KV_COL_DP = 256, KV_COL_DK = 384, KV_COL_DST = 448;
 };
 
 struct BtParams {
@@ -440,7 +446,9 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
     uint64_t* bar_final = bars + 4;
     uint64_t* bar_full = bars + 5;          // [ST]
     uint64_t* bar_empty = bar_full + ST;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_empty + ST);
+    uint64_t* bar_s_free = bar_empty + ST;  // KV_PIPE: the compute warps hold S^T(i), dP^T(i) in registers
+    uint64_t* bar_pd_free = bar_s_free + 1; // KV_PIPE: dV(i), dK(i) completed (the P^T/dS^T buffers are free)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_pd_free + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nkt = (p.Skv + 127) / 128, nqt = (p.Sq + 127) / 128;
@@ -471,6 +479,8 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
             mbar_init(bar_full + s, 1);
             mbar_init(bar_empty + s, 1);
         }
+        mbar_init(bar_s_free, 256);
+        mbar_init(bar_pd_free, 1);
         mbar_fence_init();
     }
     if (warp == 1) {
@@ -481,6 +491,12 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    constexpr uint32_t cS = C::KV_PIPE ? C::KV_COL_S : C::COL_S;
+    constexpr uint32_t cDP = C::KV_PIPE ? C::KV_COL_DP : C::COL_DP;
+    constexpr uint32_t cDV = C::KV_PIPE ? C::KV_COL_DV : C::COL_ACC;
+    constexpr uint32_t cDK = C::KV_PIPE ? C::KV_COL_DK : C::COL_DK;
+    constexpr uint32_t cPT = C::KV_PIPE ? C::KV_COL_PT : C::COL_S;     // P^T (A of dV)
+    constexpr uint32_t cDST = C::KV_PIPE ? C::KV_COL_DST : C::COL_DP;  // dS^T (A of dK)
 
     if (warp < 4) {
       setmaxnreg_dec<kBtRegsControl>();
@@ -518,15 +534,19 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
     } else if (warp == 1) {
         if (lane == 0) {
             // per (q head, query tile) iteration:  S^T = K Q^T, dP^T = V dO^T -> s_full; the compute
-            // warps write P^T and dS^T over them -> p_ready; dV += P^T dO, dK += dS^T Q; stage free
+            // warps write P^T and dS^T -> p_ready; dV += P^T dO, dK += dS^T Q; stage free.  KV_PIPE:
+            // S^T(i+1), dP^T(i+1) are issued once the compute warps hold S^T(i), dP^T(i) in
+            // registers (s_free), before dV(i), dK(i); P^T and dS^T have buffers of their own,
+            // released by pd_free.  Otherwise P^T, dS^T are written over S^T, dP^T and the next
+            // scores follow dV(i), dK(i).
             bool ok = mbar_wait(bar_fix, 0);
             tc_fence_after();
             const uint32_t uK = smem_u32(sK), uV = smem_u32(sV);
             auto stage = [&](int it) { return smem_u32(sQS + (it % ST) * C::STAGE_K); };
             auto issue_scores = [&](int it) {
                 const uint32_t q = stage(it);
-                bt_issue_scores<D, ROPE>(tmem + C::COL_S, uK, uK + C::TILE, q, q + C::TILE);
-                bt_issue_scores<D, false>(tmem + C::COL_DP, uV, uV, q + (C::NT - 1) * C::TILE, 0);
+                bt_issue_scores<D, ROPE>(tmem + cS, uK, uK + C::TILE, q, q + C::TILE);
+                bt_issue_scores<D, false>(tmem + cDP, uV, uV, q + (C::NT - 1) * C::TILE, 0);
                 mma_commit(bar_s_full);
             };
             auto wait_q = [&](int it) {
@@ -539,17 +559,26 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
                 if (ok) issue_scores(0);
             }
             for (int it = 0; it < n_it; ++it) {
+                if (C::KV_PIPE && it + 1 < n_it) {
+                    if (ok) {
+                        ok = mbar_wait(bar_s_free, it & 1);
+                        tc_fence_after();
+                    }
+                    if (ok) ok = wait_q(it + 1);
+                    if (ok) issue_scores(it + 1);
+                }
                 if (ok) {
                     ok = mbar_wait(bar_p_ready, it & 1);
                     tc_fence_after();
                 }
                 if (ok) {
                     const uint32_t q = stage(it);
-                    bt_issue_acc<D, ROPE>(tmem + C::COL_ACC, tmem + C::COL_S, q + (C::NT - 1) * C::TILE, it == 0);
-                    bt_issue_acc<D, ROPE>(tmem + C::COL_DK, tmem + C::COL_DP, q, it == 0);
+                    bt_issue_acc<D, ROPE>(tmem + cDV, tmem + cPT, q + (C::NT - 1) * C::TILE, it == 0);
+                    bt_issue_acc<D, ROPE>(tmem + cDK, tmem + cDST, q, it == 0);
                 }
+                if (C::KV_PIPE) mma_commit(bar_pd_free);
                 mma_commit(bar_empty + it % ST);
-                if (ok && it + 1 < n_it) {
+                if (!C::KV_PIPE && ok && it + 1 < n_it) {
                     ok = wait_q(it + 1);
                     if (ok) issue_scores(it + 1);
                 }
@@ -565,10 +594,10 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
         const int row = (warp & 3) * 32 + lane;
         const int key = j * 128 + row;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + C::COL_S + 64 * wg;
-        const uint32_t tP = tmem + lane_base + C::COL_DP + 64 * wg;
-        const uint32_t tPo = tmem + lane_base + C::COL_S + 32 * wg;
-        const uint32_t tDSo = tmem + lane_base + C::COL_DP + 32 * wg;
+        const uint32_t tS = tmem + lane_base + cS + 64 * wg;
+        const uint32_t tP = tmem + lane_base + cDP + 64 * wg;
+        const uint32_t tPo = tmem + lane_base + cPT + 32 * wg;
+        const uint32_t tDSo = tmem + lane_base + cDST + 32 * wg;
         const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
@@ -583,7 +612,13 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
                 tmem_ld32(tP + 32, dr[1]);
                 tmem_wait_ld();
             }
-            compute_sync();
+            if (C::KV_PIPE) {
+                // S^T(i), dP^T(i) are in registers: the MMA thread may overwrite them
+                tc_fence_before();
+                mbar_arrive(bar_s_free);
+            } else {
+                compute_sync();   // P^T, dS^T go over S^T, dP^T, which the other warpgroup reads
+            }
             if (ok) {
                 // this half's query columns q = 128 i + 64 wg + c; the key is hidden from query q
                 // past Sq, or (causal) when key > q + off
@@ -629,6 +664,11 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
                         pp[e] = pack_bf16x2(p0, p1);
                         pd[e] = pack_bf16x2(d0, d1);
                     }
+                    if (C::KV_PIPE && c == 0 && it > 0) {
+                        // the buffers still feed dV(i-1), dK(i-1) until those complete
+                        if (!__all_sync(0xffffffffu, mbar_wait(bar_pd_free, (it - 1) & 1))) ok = false;
+                        tc_fence_after();
+                    }
                     tmem_st8(tPo + 8 * c, pp);
                     tmem_st8(tDSo + 8 * c, pd);
                 }
@@ -648,14 +688,14 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
         const bool live = key < p.Skv;
         const long off = ((static_cast<long>(b) * p.Skv + key) * p.Hkv + kvh) * D + wg * (D / 2);
         if (have) {
-            tmem_ld_half<D>(tmem + lane_base + C::COL_ACC + wg * (D / 2), acc);
+            tmem_ld_half<D>(tmem + lane_base + cDV + wg * (D / 2), acc);
         } else {
 #pragma unroll
             for (int e = 0; e < D / 2; ++e) acc[e] = 0u;
         }
         if (live) bt_store<D / 2>(acc, 1.f, nullptr, p.g2_f32, p.g2_bf16, off);
         if (have) {
-            tmem_ld_half<D>(tmem + lane_base + C::COL_DK + wg * (D / 2), acc);
+            tmem_ld_half<D>(tmem + lane_base + cDK + wg * (D / 2), acc);
         }
         if (live) {
             const float2* cs = ROPE ? p.tab + static_cast<long>(key) * (D / 2) + wg * (D / 4) : nullptr;
