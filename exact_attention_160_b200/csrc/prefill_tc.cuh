@@ -80,8 +80,9 @@ struct TcCfg {
     // softmax warpgroups take turns for their exponentials (each group's loads, row max, stores
     // and hand-offs run while the other one exponentiates).  Measured on B200: 8% faster for
     // GQA 32/8 RoPE B2 S4096; without RoPE (one chain) 2-7% slower than the layout below, so
-    // only the RoPE kernels use it.
-    static constexpr bool EARLY = (D == 64 && ROPE != 0);
+    // only the RoPE kernels with pre-rotated K use it (the in-kernel K rotation needs warps 2
+    // and 3, and warp 2 issues MMAs here).
+    static constexpr bool EARLY = (D == 64 && ROPE == kRopeKSplit);
     // D=64 otherwise: the PV product runs with N = 80, its last 16 columns reading a block of
     // bf16 ones in shared memory, so column 64 of O accumulates the row sum of the rounded P the
     // MMA used (and every O correction rescales it with O).  One block serves every stage: the
