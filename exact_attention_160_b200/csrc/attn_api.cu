@@ -615,11 +615,10 @@ attn_status launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     float* Dvec = reinterpret_cast<float*>(ws + w.d_off);
     float* lse2 = reinterpret_cast<float*>(ws + w.l2_off);
     const long nq = static_cast<long>(B) * Sq * Hq;
-    bwd_rowdot_kernel<D><<<static_cast<unsigned>((nq * (D / 8) + 255) / 256), 256, 0, st>>>(o, dout, Dvec, nq, Sq, Hq);
+    bwd_rowdot_kernel<D><<<static_cast<unsigned>((nq * (D / 8) + 255) / 256), 256, 0, st>>>(o, dout, Dvec, nq, Sq, Hq,
+                                                                                       lse, lse2);
     attn_status s = launch_status("bwd_rowdot_kernel");
     if (s != ATTN_OK) return s;
-    bwd_lse2_kernel<<<static_cast<unsigned>(min((nq + 255) / 256, 148L * 32)), 256, 0, st>>>(lse, lse2, nq);
-    if ((s = launch_status("bwd_lse2_kernel")) != ATTN_OK) return s;
     const __nv_bfloat16 *qh = q, *ql = q, *kh = k, *kl = k;
     if (ROPE) {
         uint32_t* pqh = reinterpret_cast<uint32_t*>(ws + w.qh_off);

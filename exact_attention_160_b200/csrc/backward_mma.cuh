@@ -411,7 +411,8 @@ __global__ void bwd_rope_split_kernel(const uint32_t* __restrict__ x, uint32_t* 
 // lane, the row's lanes reduced with shuffles.
 template <int D>
 __global__ void bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-                                  float* __restrict__ Dvec, long nrows, int Sq, int Hq) {
+                                  float* __restrict__ Dvec, long nrows, int Sq, int Hq,
+                                  const float* __restrict__ lse = nullptr, float* __restrict__ lse2 = nullptr) {
     constexpr int LPR = D / 8;                   // lanes per row (8 or 16)
     const long t = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x;
     const long row = t / LPR;
@@ -433,7 +434,14 @@ __global__ void bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ o, const __n
         const int h = static_cast<int>(row % Hq);
         const int i = static_cast<int>((row / Hq) % Sq);
         const long b = row / (static_cast<long>(Hq) * Sq);
-        Dvec[(b * Hq + h) * Sq + i] = acc;
+        const long r = (b * Hq + h) * Sq + i;
+        Dvec[r] = acc;
+        // the tensor-core backward's log2-scaled LSE, same row order: rows with no visible key
+        // (LSE = -inf) get +inf, so that exp2(s - L2) is 0 for them
+        if (lse2 != nullptr) {
+            const float l = lse[r];
+            lse2[r] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+        }
     }
 }
 

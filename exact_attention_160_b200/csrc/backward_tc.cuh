@@ -710,14 +710,5 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
     }
 }
 
-// log2-scaled LSE for the tensor-core backward: rows with no visible key (LSE = -inf) get +inf,
-// so that exp2(s - L2) is 0 for them.
-__global__ void bwd_lse2_kernel(const float* __restrict__ lse, float* __restrict__ lse2, long n) {
-    for (long t = blockIdx.x * static_cast<long>(blockDim.x) + threadIdx.x; t < n;
-         t += static_cast<long>(gridDim.x) * blockDim.x) {
-        const float l = lse[t];
-        lse2[t] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
-    }
-}
 
 }  // namespace attn
