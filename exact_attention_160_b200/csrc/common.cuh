@@ -92,35 +92,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
-// The same wait by spinning on the non-blocking test (no suspension): for hand-offs on the
-// critical path, where a suspended waiter would resume late.  Bounded like mbar_wait.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, uint64_t timeout_ns = kWaitTimeoutNs) {
-    const uint32_t a = smem_u32(bar);
-    if (mbar_test(a, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-#pragma unroll 1
-        for (int i = 0; i < 256; ++i)
-            if (mbar_test(a, parity)) return true;
-        if (globaltimer_ns() - t0 > timeout_ns) {
-            record_error(ATTN_DEVICE_ERR_TIMEOUT);
-            return false;
-        }
-    }
-}
-
 // Programmatic dependent launch.  A grid launched with programmatic stream serialisation may be
 // scheduled before the grid ahead of it in the stream has finished: once every CTA of that grid
 // has called griddep_launch_dependents (or exited).  griddep_wait blocks until the grid ahead

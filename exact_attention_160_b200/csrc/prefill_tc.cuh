@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 if (j < nt) {
                     if (j + 1 < nt) {
                         if (ok) {
-                            ok = mbar_wait_spin(bar_s_free + t, j & 1);
+                            ok = mbar_wait(bar_s_free + t, j & 1);
                             tc_fence_after();
                         }
                         if (ok) ok = wait_k(j + 1);
@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         if (ok) {
-                            ok = mbar_wait_spin(bar_p_ready + 2 * t + half, j & 1);
+                            ok = mbar_wait(bar_p_ready + 2 * t + half, j & 1);
                             tc_fence_after();
                         }
                         if (ok) issue_pv_half(j, half);
@@ -491,7 +491,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         if (ok) {
-                            ok = mbar_wait_spin(bar_p_ready + 2 * t + half, j & 1);
+                            ok = mbar_wait(bar_p_ready + 2 * t + half, j & 1);
                             tc_fence_after();
                         }
                         if (ok) issue_pv_half(t, j, half);
@@ -651,7 +651,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             const bool mine = j < T.nkv;
             uint32_t sr[4][32];
             if (mine) {
-                if (ok && !__all_sync(0xffffffffu, mbar_wait_spin(bar_s_full + wg, j & 1))) ok = false;
+                if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) ok = false;
                 tc_fence_after();
             }
             const bool go = mine && ok;
@@ -731,7 +731,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 // P_t and O_t are free once PV_t(j-1) completed (issued when P_t(j-1) was handed
                 // over, long done by now); O is corrected before PV_t(j) may start
                 if (j > 0) {
-                    if (!__all_sync(0xffffffffu, mbar_wait_spin(bar_pv_done + wg, (j - 1) & 1))) ok = false;
+                    if (!__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) ok = false;
                     tc_fence_after();
                     if (__any_sync(0xffffffffu, need)) {
 #pragma unroll
@@ -811,7 +811,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         } else {
         for (int j = 0; j < T.nkv; ++j) {
             uint32_t sr[4][32];
-            if (ok && !__all_sync(0xffffffffu, mbar_wait_spin(bar_s_full + wg, j & 1))) ok = false;
+            if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_s_full + wg, j & 1))) ok = false;
             tc_fence_after();
             if (!ok) {
                 // keep the MMA thread's counts; it stops on its own
