@@ -26,9 +26,11 @@
 //     while one softmax warpgroup exponentiates its tile, the tensor core runs the other tile's
 //     two products, so the groups fall into alternating phases without any turn-taking barrier.
 //   * Lazy rescale: the running max used for the exponent only moves when the block max exceeds
-//     it by more than kRescaleThreshold (log2 units, i.e. a factor 256), which keeps P <= 256
-//     while skipping the O correction on almost every block.  The "running max is -inf" guard
-//     makes rows with no visible key yet contribute nothing.
+//     it by more than kRescaleThreshold (log2 units, 2^32), which keeps P <= 2^32 while skipping
+//     the O correction (a tcgen05.ld/st of the row of O on the softmax's critical path) on all
+//     but a few blocks even for peaked scores.  Nothing loses precision: P is rounded to bf16
+//     relative to its own size, and l and O (fp32) stay far from overflow (l <= Skv 2^32).  The
+//     "running max is -inf" guard makes rows with no visible key yet contribute nothing.
 //   * With RoPE, Q is rotated in shared memory right after its TMA load and K arrives
 //     pre-rotated; both carry hi + lo bf16 halves and S = Qh Kh^T + Qh Kl^T + Ql Kh^T.
 //   * MASK instantiations add an additive score mask (whisper-apr attention_generated.rs,
@@ -53,7 +55,7 @@ constexpr int kTcThreads = 384;
 constexpr int kRegsControl = 72;
 constexpr int kRegsSoftmax = 208;
 constexpr int kTcLaunchRegsMin = (128 * kRegsControl + 256 * kRegsSoftmax + kTcThreads - 1) / kTcThreads;
-constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThreshold = 32.0f;
 // RoPE forms of the kernel: none; K rotated beforehand into hi + lo halves (rope_split_kv_kernel);
 // K loaded as it is and rotated into hi + lo halves in shared memory by the two idle warps of the
 // control warpgroup (warps 2 and 3) while the ring runs ahead.
