@@ -59,6 +59,10 @@ CASES = [
     P("tc_bf16_noncausal_mqa", "bf16", 2, 4, 1, 260, 330, 64, False, 0.125, seed=213),
     P("tc_bf16_d128_gqa_rope", "bf16", 1, 8, 2, 384, 384, 128, True, 0.0884, rope_base=10000.0, seed=214),
     P("tc_bf16_d64_bottom_right", "bf16", 2, 6, 3, 196, 452, 64, True, 0.125, seed=215),
+    # D=64 with RoPE over several query and key tiles: the overlapped dq (dS double buffer) and
+    # dk/dv (P^T, dS^T buffers of their own) pipelines run many iterations per CTA
+    P("tc_bf16_d64_gqa_rope_multi_tile", "bf16", 1, 8, 2, 520, 520, 64, True, 0.125, rope_base=10000.0, seed=216),
+    P("tc_bf16_d64_noncausal_ragged", "bf16", 1, 4, 4, 388, 611, 64, False, 0.125, seed=217),
 ]
 
 

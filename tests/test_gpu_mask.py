@@ -18,6 +18,8 @@ CASES = [
     (P("per_head_gqa", "bf16", 1, 8, 2, 150, 260, 64, False, 0.125, seed=402), "per_head"),
     (P("key_padding", "bf16", 3, 4, 4, 130, 170, 64, False, 0.125, seed=403), "key_padding"),
     (P("rope_d128", "bf16", 1, 4, 2, 140, 140, 128, True, 0.0884, rope_base=10000.0, seed=404), "shared"),
+    # D=64 with RoPE: P in TMEM columns of its own, two MMA issuers, exponentiation turns
+    (P("rope_d64_gqa_per_head", "bf16", 1, 8, 2, 300, 420, 64, True, 0.125, rope_base=10000.0, seed=408), "per_head"),
     (P("rows_all_inf", "bf16", 1, 2, 2, 90, 90, 64, False, 0.125, seed=405), "dead_rows"),
     (P("fp32_shared", "fp32", 1, 2, 2, 100, 120, 64, True, 0.125, seed=406), "shared"),
     (P("padded_d40", "bf16", 1, 4, 4, 110, 110, 40, True, 0.158, seed=407), "per_batch"),
