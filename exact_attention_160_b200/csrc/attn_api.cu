@@ -656,7 +656,7 @@ attn_status launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     auto kkv = bwd_dkdv_tc_kernel<D, ROPE>;
     if ((s = prepare_kernel(reinterpret_cast<const void*>(kdq), C::SMEM_Q, "bwd_dq_tc_kernel set-up", kBtLaunchRegsMin)) != ATTN_OK)
         return s;
-    if ((s = prepare_kernel(reinterpret_cast<const void*>(kkv), C::SMEM_K, "bwd_dkdv_tc_kernel set-up", kBtLaunchRegsMin)) != ATTN_OK)
+    if ((s = prepare_kernel(reinterpret_cast<const void*>(kkv), C::SMEM_K, "bwd_dkdv_tc_kernel set-up", kBtKvLaunchRegsMin)) != ATTN_OK)
         return s;
     const long grid_q = static_cast<long>((Sq + 127) / 128) * B * Hq;
     const long grid_k = static_cast<long>((Skv + 127) / 128) * B * Hkv;
@@ -669,7 +669,7 @@ attn_status launch_bwd_tc(const __nv_bfloat16* q, const __nv_bfloat16* k, const 
     p.g_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dk);
     p.g2_f32 = g_f32 ? static_cast<float*>(dv) : nullptr;
     p.g2_bf16 = g_f32 ? nullptr : static_cast<__nv_bfloat16*>(dv);
-    kkv<<<static_cast<unsigned>(grid_k), kBtThreads, C::SMEM_K, st>>>(tq, tql, tk, tkl, tv, tdo, tl2, tdv, p);
+    kkv<<<static_cast<unsigned>(grid_k), kBtKvThreads, C::SMEM_K, st>>>(tq, tql, tk, tkl, tv, tdo, tl2, tdv, p);
     return launch_status("bwd_dkdv_tc_kernel");
 }
 

@@ -35,6 +35,17 @@ constexpr int kBtThreads = 384;
 constexpr int kBtRegsControl = 72;
 constexpr int kBtRegsCompute = 216;
 constexpr int kBtLaunchRegsMin = (128 * kBtRegsControl + 256 * kBtRegsCompute + kBtThreads - 1) / kBtThreads;
+// The dk/dv kernel forms P^T and dS^T elementwise (no reduction across a key's row), so its
+// compute work splits into four warpgroups of 32 query columns each with no exchange: four warps
+// per sub-partition hide each other's latencies.  640 threads launch with 96 registers each
+// (five warps per sub-partition); setmaxnreg moves them to the compute warps: 56 x 128 +
+// 104 x 512 = 60416 <= 96 x 640, and per sub-partition (56 + 4 * 104) * 32 = 15104 <= 16384.
+constexpr int kBtKvWarpgroups = 4;
+constexpr int kBtKvThreads = 128 + 128 * kBtKvWarpgroups;
+constexpr int kBtKvRegsControl = 56;
+constexpr int kBtKvRegsCompute = 104;
+constexpr int kBtKvLaunchRegsMin =
+    (128 * kBtKvRegsControl + 128 * kBtKvWarpgroups * kBtKvRegsCompute + kBtKvThreads - 1) / kBtKvThreads;
 
 template <int D, bool ROPE>
 struct BtCfg {
@@ -86,7 +97,8 @@ struct BtParams {
 
 // Named barrier of the two compute warpgroups (256 threads): every thread has read its S / dP
 // columns before any thread overwrites the first half of S / dP with bf16 operands.
-__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+template <int N = 256>
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory"); }
 
 // Store a row segment of n (= D/2) fp32 gradient values, optionally rotated back by -theta.
 template <int N>
@@ -110,6 +122,24 @@ __device__ __forceinline__ void bt_store(const uint32_t (&acc)[N], float mul, co
             dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]), pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
                                 pack_bf16x2(v[8 * e + 4], v[8 * e + 5]), pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
     }
+}
+
+// Read N (16, 32 or 64) accumulator columns of this thread's TMEM lane.
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[N]) {
+    if constexpr (N == 16) {
+        tmem_ld16(taddr, r);
+    } else if constexpr (N == 32) {
+        tmem_ld32(taddr, r);
+    } else {
+        uint32_t a[32], b[32];
+        tmem_ld32(taddr, a);
+        tmem_ld32(taddr + 32, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) r[e] = a[e], r[32 + e] = b[e];
+    }
+    tmem_wait_ld();
 }
 
 // Read D/2 accumulator columns [c0, c0 + D/2) of this thread's TMEM lane.
@@ -426,7 +456,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dq_tc_kernel(
 // dK, dV
 // ------------------------------------------------------------------------------------------
 template <int D, bool ROPE>
-__global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
+__global__ void __launch_bounds__(kBtKvThreads, 1) bwd_dkdv_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_ql,
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kl,
     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -472,14 +502,14 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
     if (tid == 0) {
         mbar_init(bar_fix, 1);
         mbar_init(bar_s_full, 1);
-        mbar_init(bar_p_ready, 256);
+        mbar_init(bar_p_ready, 128 * kBtKvWarpgroups);
         mbar_init(bar_acc_done, 1);
         mbar_init(bar_final, 1);
         for (int s = 0; s < ST; ++s) {
             mbar_init(bar_full + s, 1);
             mbar_init(bar_empty + s, 1);
         }
-        mbar_init(bar_s_free, 256);
+        mbar_init(bar_s_free, 128 * kBtKvWarpgroups);
         mbar_init(bar_pd_free, 1);
         mbar_fence_init();
     }
@@ -499,7 +529,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
     constexpr uint32_t cDST = C::KV_PIPE ? C::KV_COL_DST : C::COL_DP;  // dS^T (A of dK)
 
     if (warp < 4) {
-      setmaxnreg_dec<kBtRegsControl>();
+      setmaxnreg_dec<kBtKvRegsControl>();
       if (warp == 0) {
         if (lane == 0) {
             const uint64_t pol_kv = l2_policy_evict_first();
@@ -589,27 +619,30 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
         }
       }
     } else {
-        setmaxnreg_inc<kBtRegsCompute>();
+        setmaxnreg_inc<kBtKvRegsCompute>();
+        constexpr int CW = 128 / kBtKvWarpgroups;   // query columns of this warpgroup
+        constexpr int AC = D / kBtKvWarpgroups;     // accumulator columns this warpgroup stores
         const int wg = (warp - 4) >> 2;
         const int row = (warp & 3) * 32 + lane;
         const int key = j * 128 + row;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_base + cS + 64 * wg;
-        const uint32_t tP = tmem + lane_base + cDP + 64 * wg;
-        const uint32_t tPo = tmem + lane_base + cPT + 32 * wg;
-        const uint32_t tDSo = tmem + lane_base + cDST + 32 * wg;
+        const uint32_t tS = tmem + lane_base + cS + CW * wg;
+        const uint32_t tP = tmem + lane_base + cDP + CW * wg;
+        const uint32_t tPo = tmem + lane_base + cPT + (CW / 2) * wg;
+        const uint32_t tDSo = tmem + lane_base + cDST + (CW / 2) * wg;
         const uint64_t sl2x2 = f2_pack(p.scale_log2, p.scale_log2);
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int i = i0 + it % per_head;
-            uint32_t sr[2][32], dr[2][32];
+            uint32_t sr[CW / 32][32], dr[CW / 32][32];
             if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_s_full, it & 1))) ok = false;
             tc_fence_after();
             if (ok) {
-                tmem_ld32(tS, sr[0]);
-                tmem_ld32(tS + 32, sr[1]);
-                tmem_ld32(tP, dr[0]);
-                tmem_ld32(tP + 32, dr[1]);
+#pragma unroll
+                for (int cb = 0; cb < CW / 32; ++cb) {
+                    tmem_ld32(tS + 32 * cb, sr[cb]);
+                    tmem_ld32(tP + 32 * cb, dr[cb]);
+                }
                 tmem_wait_ld();
             }
             if (C::KV_PIPE) {
@@ -617,22 +650,22 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
                 tc_fence_before();
                 mbar_arrive(bar_s_free);
             } else {
-                compute_sync();   // P^T, dS^T go over S^T, dP^T, which the other warpgroup reads
+                compute_sync<128 * kBtKvWarpgroups>();   // P^T, dS^T go over S^T, dP^T, which other warpgroups read
             }
             if (ok) {
-                // this half's query columns q = 128 i + 64 wg + c; the key is hidden from query q
-                // past Sq, or (causal) when key > q + off
+                // this warpgroup's query columns q = 128 i + CW wg + c; the key is hidden from query
+                // q past Sq, or (causal) when key > q + off
                 const float* rows = reinterpret_cast<const float*>(sQS + (it % ST) * C::STAGE_K + C::NT * C::TILE);
-                const float4* l2v = reinterpret_cast<const float4*>(rows + 64 * wg);
-                const float4* dvv = reinterpret_cast<const float4*>(rows + 128 + 64 * wg);
-                const long q0 = static_cast<long>(i) * 128 + 64 * wg;
+                const float4* l2v = reinterpret_cast<const float4*>(rows + CW * wg);
+                const float4* dvv = reinterpret_cast<const float4*>(rows + 128 + CW * wg);
+                const long q0 = static_cast<long>(i) * 128 + CW * wg;
                 // visible iff q < Sq and (not causal or q >= key - off)
                 const long qmin = p.causal ? static_cast<long>(key) - off_c : 0;
                 // hidden queries: S^T = -inf, so P^T = 0 and dS^T = 0 (a separate pass, taken only
                 // by warps that have one, keeps the loop below free of per-element checks)
-                if (__any_sync(0xffffffffu, q0 < qmin || q0 + 63 >= p.Sq)) {
+                if (__any_sync(0xffffffffu, q0 < qmin || q0 + CW - 1 >= p.Sq)) {
 #pragma unroll
-                    for (int cb = 0; cb < 2; ++cb)
+                    for (int cb = 0; cb < CW / 32; ++cb)
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
                             const long qq = q0 + cb * 32 + e;
@@ -641,7 +674,7 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
                 }
                 // 16 query columns at a time, stored as soon as they are formed (few live registers)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < CW / 16; ++c) {
                     uint32_t pp[8], pd[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
@@ -684,22 +717,22 @@ __global__ void __launch_bounds__(kBtThreads, 1) bwd_dkdv_tc_kernel(
             have = __all_sync(0xffffffffu, mbar_wait(bar_acc_done, 0));
             tc_fence_after();
         }
-        uint32_t acc[D / 2];
+        uint32_t acc[AC];
         const bool live = key < p.Skv;
-        const long off = ((static_cast<long>(b) * p.Skv + key) * p.Hkv + kvh) * D + wg * (D / 2);
+        const long off = ((static_cast<long>(b) * p.Skv + key) * p.Hkv + kvh) * D + wg * AC;
         if (have) {
-            tmem_ld_half<D>(tmem + lane_base + cDV + wg * (D / 2), acc);
+            tmem_ld_cols<AC>(tmem + lane_base + cDV + wg * AC, acc);
         } else {
 #pragma unroll
-            for (int e = 0; e < D / 2; ++e) acc[e] = 0u;
+            for (int e = 0; e < AC; ++e) acc[e] = 0u;
         }
-        if (live) bt_store<D / 2>(acc, 1.f, nullptr, p.g2_f32, p.g2_bf16, off);
+        if (live) bt_store<AC>(acc, 1.f, nullptr, p.g2_f32, p.g2_bf16, off);
         if (have) {
-            tmem_ld_half<D>(tmem + lane_base + cDK + wg * (D / 2), acc);
+            tmem_ld_cols<AC>(tmem + lane_base + cDK + wg * AC, acc);
         }
         if (live) {
-            const float2* cs = ROPE ? p.tab + static_cast<long>(key) * (D / 2) + wg * (D / 4) : nullptr;
-            bt_store<D / 2>(acc, p.scale, cs, p.g_f32, p.g_bf16, off);
+            const float2* cs = ROPE ? p.tab + static_cast<long>(key) * (D / 2) + wg * (AC / 2) : nullptr;
+            bt_store<AC>(acc, p.scale, cs, p.g_f32, p.g_bf16, off);
         }
     }
     tc_fence_before();
