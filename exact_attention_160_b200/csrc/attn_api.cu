@@ -436,9 +436,15 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
     // The combine is a programmatic dependent launch: its CTAs may be scheduled while the last
     // split CTAs finish, which hides the launch gap; it waits (griddepcontrol.wait) for the
     // split grid to complete before reading the partials.
+    // Up to kDecodeWarpCombineSplits splits, one warp merges a (sequence, head) with all its
+    // loads in flight; more splits take the block-per-head kernel, which walks them in chunks.
+    const bool warp_combine = num_splits <= kDecodeWarpCombineSplits;
+    const long rows = static_cast<long>(B) * Hq;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(B) * static_cast<unsigned>(Hq));
-    cfg.blockDim = dim3(kCombineThreads);
+    cfg.gridDim = warp_combine ? dim3(static_cast<unsigned>((rows + kDecodeWarpCombineThreads / 32 - 1) /
+                                                            (kDecodeWarpCombineThreads / 32)))
+                               : dim3(static_cast<unsigned>(B) * static_cast<unsigned>(Hq));
+    cfg.blockDim = dim3(warp_combine ? kDecodeWarpCombineThreads : kCombineThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -446,12 +452,12 @@ attn_status launch_decode(const void* q, const void* kc, const void* vc, const i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, static_cast<const float*>(o_part),
-                                             static_cast<const float*>(lse_part), seqlens,
-                                             o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, warp_combine ? decode_combine_warp_kernel<D> : decode_combine_kernel<D>,
+                                             static_cast<const float*>(o_part), static_cast<const float*>(lse_part),
+                                             seqlens, o_f32 ? nullptr : static_cast<__nv_bfloat16*>(o),
                                              o_f32 ? static_cast<float*>(o) : nullptr, lse, B, Hq, Smax, num_splits);
-    if (e != cudaSuccess) return cuda_failure("decode_combine_kernel launch", cudaGetErrorString(e));
-    return launch_status("decode_combine_kernel");
+    if (e != cudaSuccess) return cuda_failure("decode combine launch", cudaGetErrorString(e));
+    return launch_status(warp_combine ? "decode_combine_warp_kernel" : "decode_combine_kernel");
 }
 
 // Workspace of a padded forward: q, k, v and o at Dp, then the inner call's own workspace.

@@ -379,4 +379,71 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(
     if (lse != nullptr && d == 0) lse[bh] = total > 0.f ? M + logf(total) : -INFINITY;
 }
 
+// The combine for at most kDecodeWarpCombineSplits splits: one warp per (sequence, q head), split
+// s in lane s for the logsumexp weights and D / 32 output dims per lane, every load of the row
+// issued before any result is used (one memory round trip, no shared memory or block barriers).
+constexpr int kDecodeWarpCombineSplits = 16;
+constexpr int kDecodeWarpCombineThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kDecodeWarpCombineThreads) decode_combine_warp_kernel(
+    const float* __restrict__ o_part, const float* __restrict__ lse_part,
+    const int32_t* __restrict__ seqlens, __nv_bfloat16* __restrict__ o, float* __restrict__ o_f32,
+    float* __restrict__ lse, int B, int Hq, int Smax, int max_splits) {
+    constexpr int E = D / 32;   // output dims per lane
+    const long bh = static_cast<long>(blockIdx.x) * (kDecodeWarpCombineThreads / 32) + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    griddep_wait();   // the split grid's partials are complete and visible after this
+    if (bh >= static_cast<long>(B) * Hq) return;   // whole warps leave together
+    const int b = static_cast<int>(bh / Hq);
+    int L = seqlens[b];   // clamped as the split kernel does (which reports the clamp)
+    L = L < 1 ? 1 : (L > Smax ? Smax : L);
+    const int nsplit = decode_num_splits(L, max_splits);
+    const long slot0 = bh * max_splits;
+    const float ls = lane < nsplit ? lse_part[slot0 + lane] : -INFINITY;
+    float x[kDecodeWarpCombineSplits][E];
+#pragma unroll
+    for (int sp = 0; sp < kDecodeWarpCombineSplits; ++sp) {
+        if (sp < nsplit) {
+            const float* src = o_part + (slot0 + sp) * D + lane * E;
+            if constexpr (E == 2) {
+                const float2 v = *reinterpret_cast<const float2*>(src);
+                x[sp][0] = v.x, x[sp][1] = v.y;
+            } else {
+                const float4 v = *reinterpret_cast<const float4*>(src);
+                x[sp][0] = v.x, x[sp][1] = v.y, x[sp][2] = v.z, x[sp][3] = v.w;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; ++e) x[sp][e] = 0.f;
+        }
+    }
+    float M = ls;
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, w));
+    const float wt = (M == -INFINITY || ls == -INFINITY) ? 0.f : __expf(ls - M);
+    float total = wt;
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) total += __shfl_xor_sync(0xffffffffu, total, w);
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < kDecodeWarpCombineSplits; ++sp) {
+        const float ws = __shfl_sync(0xffffffffu, wt, sp);   // 0 for sp >= nsplit
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = fmaf(ws, x[sp][e], acc[e]);
+    }
+    const float inv = total > 0.f ? 1.f / total : 0.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const float out = acc[e] * inv;
+        if (o_f32 != nullptr)
+            o_f32[bh * D + lane * E + e] = out;
+        else
+            o[bh * D + lane * E + e] = __float2bfloat16_rn(out);
+    }
+    if (lse != nullptr && lane == 0) lse[bh] = total > 0.f ? M + logf(total) : -INFINITY;
+}
+
 }  // namespace attn
