@@ -191,8 +191,8 @@ size_t attn_decode_workspace_size(int B, int Hq, int D, int num_splits);
  *   - Sizes: attn_decode_workspace_size(B, Hq, D, num_splits) must not exceed
  *     ATTN_NOALLOC_SCRATCH_BYTES, else ATTN_ERR_WORKSPACE (attn_last_error() says by how much).
  *   - Set-up: the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, which may load the library's GPU code onto that device); make that
- *     first call before any stream capture.  Failure returns ATTN_ERR_CUDA.
+ *     (cudaGetSymbolAddress, which may load the library's GPU code onto that device).  Failure
+ *     returns ATTN_ERR_CUDA.
  *   - Sharing: every call on a device uses the same array, and it keeps the last call's
  *     contents.  Calls that overlap on the GPU (different streams, no ordering between them)
  *     race on it and may return wrong results; order them on one stream or with events.
