@@ -291,8 +291,15 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     }
     const long grid = static_cast<long>(p.n_row_tiles) * B * p.heads_per_item * p.kv_splits;
     if (grid > 2147483647L) return ATTN_ERR_UNSUPPORTED;
-    // the masked kernel is a separate instantiation, so the unmasked one carries no mask code
-    auto kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true> : prefill_tc_kernel<D, ROPE, false>;
+    // The masked kernel is a separate instantiation, so the unmasked one carries no mask code.
+    // Single query tiles at D = 64 run with interleaved keys: the CTA's two softmax warpgroups
+    // take alternate key tiles of its one query tile, so that one works while the tensor core
+    // serves the other (at D = 128 the ring has too few stages for the pair).
+    auto kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true, false> : prefill_tc_kernel<D, ROPE, false, false>;
+    if constexpr (D == 64) {
+        if (p.single_tile)
+            kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true, true> : prefill_tc_kernel<D, ROPE, false, true>;
+    }
     const int smem_bytes = TcCfg<D, ROPE>::SMEM_BYTES;
     // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds fewer
     // than the split asks for would stall in setmaxnreg.inc, so such a build is refused.

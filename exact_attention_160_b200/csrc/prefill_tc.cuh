@@ -60,8 +60,9 @@ constexpr float kRescaleThreshold = 32.0f;
 // K loaded as it is and rotated into hi + lo halves in shared memory by the two idle warps of the
 // control warpgroup (warps 2 and 3) while the ring runs ahead.
 constexpr int kRopeNone = 0, kRopeKSplit = 1, kRopeKFused = 2;
-// named barriers of the exponentiation turns (0 is __syncthreads)
-constexpr uint32_t kTcBarTurn0 = 1, kTcBarTurn1 = 2;
+// named barriers of the exponentiation turns (0 is __syncthreads), of the in-CTA merge and of
+// one softmax warpgroup (4 + its index)
+constexpr uint32_t kTcBarTurn0 = 1, kTcBarTurn1 = 2, kTcBarMerge = 3, kTcBarGroup0 = 4;
 constexpr float kLn2 = 0.69314718055994531f;
 
 template <int D, int ROPE>
@@ -145,7 +146,10 @@ __device__ __forceinline__ int tc_kv_tiles(const TcParams& p, int r0) {
     return n < nkv_all ? static_cast<int>(n) : nkv_all;
 }
 
-template <int D, int ROPE, bool MASK>
+// ILV (interleaved keys, single-tile mode only): the two softmax warpgroups take alternate key
+// tiles of the CTA's one query tile and the epilogue merges their states.  A template parameter,
+// so that the other kernels carry none of its code.
+template <int D, int ROPE, bool MASK, bool ILV>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
@@ -183,11 +187,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const int rem = item % items_per_rowtile;
     const int b = rem / p.heads_per_item;
     const int hi = rem % p.heads_per_item;
+    // interleaved keys (below) need ring slots to spare: each step of the pair takes two
+    static_assert(!ILV || C::STAGES >= 3, "interleaved keys need three K/V stages or more");
+    constexpr bool ilv = ILV;
     TcTile tile[2];
     if (p.single_tile) {
         tile[0].h = tile[1].h = hi;
         tile[0].r0 = rt * 128;
-        tile[1].r0 = p.Sq;    // inactive
+        tile[1].r0 = ilv ? rt * 128 : p.Sq;    // the same rows, or inactive
     } else if (p.pair_heads) {
         tile[0].h = 2 * hi;
         tile[1].h = 2 * hi + 1;
@@ -211,8 +218,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         kv0 = split * base + min(split, extra);
         tile[0].nkv = base + (split < extra ? 1 : 0);
     }
+    // Interleaved keys: the CTA's key tiles u = 0, 1, 2, ... go alternately to the two softmax
+    // warpgroups (tile t takes u = 2j + t at its step j), each running its own online softmax
+    // over the same query rows.  Both then stream through the K/V ring in the order u, so every
+    // ring slot serves one tile; without interleaving slot j serves both tiles' step j.
+    const int n_keys = tile[0].nkv;   // this CTA's key tiles (interleaved mode)
+    if (ilv) {
+        tile[0].nkv = (n_keys + 1) / 2;
+        tile[1].nkv = n_keys / 2;
+    }
     const int kvh = tile[0].h / (p.Hq / p.Hkv);
     const int nkv = max(tile[0].nkv, tile[1].nkv);
+    const int n_loads = ilv ? n_keys : nkv;   // K/V tiles through the ring
+    // ring index (and key tile, from kv0) of tile t's step j
+    auto ring_of = [ilv](int t, int j) { return ilv ? 2 * j + t : j; };
 
     // ---- set-up --------------------------------------------------------------------------
     if (tid == 0) {
@@ -280,13 +299,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                                 tile[i].r0, b, pol_q);
             }
             int issued = 0;
-            for (int j = 0; j < nkv; ++j) {
+            for (int j = 0; j < n_loads; ++j) {
                 const int s = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
-                // EARLY: each MMA thread releases the stages its own tile used (j - STAGES < n_t)
+                // EARLY: each MMA thread releases the stages its own tile used (j - STAGES < n_t);
+                // interleaved keys: a slot serves one tile at a time, released on bar_kv_empty[s]
                 bool freed = true;
-                if (!C::EARLY || j < C::STAGES || j - C::STAGES < tile[0].nkv) freed = mbar_wait(bar_kv_empty + s, ph ^ 1);
-                if (C::EARLY && freed && (j < C::STAGES || j - C::STAGES < tile[1].nkv))
+                if (!C::EARLY || ilv || j < C::STAGES || j - C::STAGES < tile[0].nkv)
+                    freed = mbar_wait(bar_kv_empty + s, ph ^ 1);
+                if (C::EARLY && !ilv && freed && (j < C::STAGES || j - C::STAGES < tile[1].nkv))
                     freed = mbar_wait(bar_kv_empty + C::STAGES + s, ph ^ 1);
                 if (!freed) break;
                 issued = j + 1;
@@ -334,7 +355,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             const uint32_t dO = tmem + (t ? C::COL_O1 : C::COL_O0);
             const uint32_t aP = tmem + (t ? C::COL_P1 : C::COL_P0);
             auto issue_s = [&](int j) {
-                const uint32_t klo = kvlo0 + ((j % C::STAGES) * C::STAGE_BYTES >> 4);
+                const uint32_t klo = kvlo0 + ((ring_of(t, j) % C::STAGES) * C::STAGE_BYTES >> 4);
                 constexpr int NCHAIN = ROPE ? 3 : 1;
 #pragma unroll
                 for (int ch = 0; ch < NCHAIN; ++ch) {
@@ -351,7 +372,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 mma_commit(bar_s_full + t);
             };
             auto issue_pv_half = [&](int j, int half) {
-                const uint32_t va = smem_u32(sKV) + (j % C::STAGES) * C::STAGE_BYTES + C::K_TILES * C::TILE_BYTES;
+                const uint32_t va = smem_u32(sKV) + (ring_of(t, j) % C::STAGES) * C::STAGE_BYTES + C::K_TILES * C::TILE_BYTES;
                 const uint32_t vlo = desc_sw128_lo(va, C::TILE_BYTES / C::NBOX);
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
@@ -362,7 +383,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             };
             auto wait_k = [&](int j) {
                 uint64_t* kb = ROPE == kRopeKFused ? bar_k_rot : bar_k_full;
-                const bool r = mbar_wait(kb + j % C::STAGES, (j / C::STAGES) & 1);
+                const int u = ring_of(t, j);
+                const bool r = mbar_wait(kb + u % C::STAGES, (u / C::STAGES) & 1);
                 tc_fence_after();
                 return r;
             };
@@ -371,7 +393,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 if (ok) issue_s(0);
             }
             for (int j = 0; j < nkv; ++j) {
-                const int s = j % C::STAGES;
+                const int u = ring_of(t, j), s = u % C::STAGES;
                 if (j < nt) {
                     if (j + 1 < nt) {
                         if (ok) {
@@ -382,7 +404,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                         if (ok) issue_s(j + 1);
                     }
                     if (ok) {
-                        ok = mbar_wait(bar_v_full + s, (j / C::STAGES) & 1);
+                        ok = mbar_wait(bar_v_full + s, (u / C::STAGES) & 1);
                         tc_fence_after();
                     }
 #pragma unroll
@@ -395,7 +417,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     }
                     mma_commit(bar_pv_done + t);
                     if (j == nt - 1) mma_commit(bar_o_done + t);
-                    mma_commit(bar_kv_empty + t * C::STAGES + s);   // this tile is done with stage s
+                    mma_commit(bar_kv_empty + (ilv ? 0 : t * C::STAGES) + s);   // this tile is done with stage s
                 }
             }
             if (!ok) mma_commit(bar_o_done + t);
@@ -434,7 +456,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             auto issue_s = [&](int t, int j) {
                 const uint32_t qlo = desc_sw128_lo(smem_u32(sQ + t * C::Q_TILES * C::TILE_BYTES), 16);
                 const uint32_t dS = tmem + (t ? C::COL_S1 : C::COL_S0);
-                const uint32_t klo = kvlo0 + ((j % C::STAGES) * C::STAGE_BYTES >> 4);
+                const uint32_t klo = kvlo0 + ((ring_of(t, j) % C::STAGES) * C::STAGE_BYTES >> 4);
                 // chains: (Qh,Kh) [+ (Qh,Kl) + (Ql,Kh) with RoPE]
                 constexpr int NCHAIN = ROPE ? 3 : 1;
 #pragma unroll
@@ -457,7 +479,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             auto issue_pv_half = [&](int t, int j, int half) {
                 const uint32_t dO = tmem + (t ? C::COL_O1 : C::COL_O0);
                 const uint32_t aP = tmem + (t ? C::COL_S1 : C::COL_S0);
-                const uint32_t vlo = v_lo(j % C::STAGES);
+                const uint32_t vlo = v_lo(ring_of(t, j) % C::STAGES);
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
                     // keys [16kk, 16kk+16): 16 rows of 128 B in every 64-wide D box
@@ -467,9 +489,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 }
                 if (half == 1 && j == (t ? nt1 : nt0) - 1) mma_commit(bar_o_done + t);
             };
-            auto wait_k = [&](int j) {
+            auto wait_k = [&](int u) {   // K of ring index u in place
                 uint64_t* kb = ROPE == kRopeKFused ? bar_k_rot : bar_k_full;
-                const bool r = mbar_wait(kb + j % C::STAGES, (j / C::STAGES) & 1);
+                const bool r = mbar_wait(kb + u % C::STAGES, (u / C::STAGES) & 1);
                 tc_fence_after();
                 return r;
             };
@@ -477,9 +499,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             if (ok && nkv_all > 0) {
                 ok = wait_k(0);
                 if (ok && nt0 > 0) issue_s(0, 0);
+                if (ilv && ok && nt1 > 0) ok = wait_k(1);
                 if (ok && nt1 > 0) issue_s(1, 0);
             }
-            for (int j = 0; j < nkv_all; ++j) {
+            // Interleaved keys, per step j and tile t (ring index u = 2j + t):
+            //   PV_t(j) from slot u, release of slot u, S_t(j+1) from slot u + 2
+            for (int j = 0; ilv && j < nkv_all; ++j) {
+#pragma unroll
+                for (int t = 0; t < 2; ++t) {
+                    const int n = t ? nt1 : nt0;
+                    if (j >= n) continue;
+                    const int u = 2 * j + t, s = u % C::STAGES;
+                    if (ok) {
+                        ok = mbar_wait(bar_v_full + s, (u / C::STAGES) & 1);
+                        tc_fence_after();
+                    }
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        if (ok) {
+                            ok = mbar_wait(bar_p_ready + 2 * t + half, j & 1);
+                            tc_fence_after();
+                        }
+                        if (ok) issue_pv_half(t, j, half);
+                    }
+                    mma_commit(bar_kv_empty + s);
+                    if (ok && j + 1 < n) {
+                        ok = wait_k(u + 2);
+                        if (ok) issue_s(t, j + 1);
+                    }
+                }
+            }
+            for (int j = 0; !ilv && j < nkv_all; ++j) {
                 const int s = j % C::STAGES;
                 if (ok) {
                     ok = mbar_wait(bar_v_full + s, (j / C::STAGES) & 1);
@@ -529,7 +579,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         // pairs (2i, 2i+1) share a 16-byte chunk, which the 128-byte swizzle moves whole.
         constexpr int NROT = C::EARLY ? 32 : 64;   // warp 3 alone when warp 2 issues MMAs
         const int u = C::EARLY ? lane : (warp - 2) * 32 + lane;
-        for (int j = 0; j < nkv; ++j) {
+        for (int j = 0; j < n_loads; ++j) {   // j: ring index = key tile kv0 + j
             const int s = j % C::STAGES;
             if (!mbar_wait(bar_k_full + s, (j / C::STAGES) & 1)) break;
             uint8_t* kh = sKV + s * C::STAGE_BYTES;
@@ -670,7 +720,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             bool need = false;
             float corr = 1.f;
             if (go) {
-            const int k0 = (kv0 + j) * 128;
+            const int k0 = (kv0 + ring_of(wg, j)) * 128;
                 if (MASK && qrow < p.Sq) {
                     // additive mask: S holds q.k unscaled, so add mask / scale; the exponent
                     // (s * scale + mask) * log2(e) - m then keeps its form
@@ -824,7 +874,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tmem_ld32(tS + cb * 32, sr[cb]);
             tmem_wait_ld();
-            const int k0 = (kv0 + j) * 128;
+            const int k0 = (kv0 + ring_of(wg, j)) * 128;
             if (MASK && qrow < p.Sq) {
                 // additive mask: S holds q.k unscaled, so add mask / scale; the exponent
                 // (s * scale + mask) * log2(e) - m then keeps its form
@@ -946,13 +996,31 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         }
 
         }
-        // epilogue: O / l -> bf16 or fp32, lse.  The TMEM reads are warp-collective, so every
-        // lane of the warp takes part; only rows inside [0, Sq) are stored.
+        // Epilogue: O / l -> bf16 or fp32, and the logsumexp.  With interleaved keys the two
+        // warpgroups hold partial states (m_t, l_t, O_t) of the same rows: they exchange m and
+        // the row sums through shared memory (each in its own Q slot, free once its products are
+        // done) and each writes half of the columns of the merged
+        //   O = (a_0 O_0 + a_1 O_1) / (a_0 l_0 + a_1 l_1),  a_t = 2^(m_t - max(m_0, m_1)).
+        // The TMEM reads are warp-collective, so every lane of the warp takes part; only rows
+        // inside [0, Sq) are stored.
         if (T.active) {
-            bool have = ok && T.nkv > 0;
+            bool have = ok && T.nkv > 0;   // warp-uniform: this tile's O holds products
             if (have) {
                 have = __all_sync(0xffffffffu, mbar_wait(bar_o_done + wg, 0));
                 tc_fence_after();
+            } else if (ilv) {
+                // the merge below writes to the Q slot: its copy must have landed (no product
+                // waited for it) ...
+                mbar_wait(bar_q_full, 0);
+            }
+            // ... and with RoPE every row of it must be rotated: without a product of this tile
+            // nothing has ordered the other rows' rotation before this point (T.nkv is uniform
+            // over the warpgroup, so all of its threads meet here)
+            if (ilv && ROPE && T.nkv == 0) {
+                if (wg == 0)
+                    named_bar_sync(kTcBarGroup0, 128);
+                else
+                    named_bar_sync(kTcBarGroup0 + 1, 128);
             }
             const bool store = qrow < p.Sq;
             if (C::ONES && have) {
@@ -962,7 +1030,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 tmem_wait_ld();
                 l_mma = __uint_as_float(sr1[0]);
             }
-            const float inv = (have && l_mma > 0.f) ? 1.f / l_mma : 0.f;
+            float m_fin = m_run;                      // exponent base of the result
+            float l_fin = have ? l_run : 0.f;         // exact row sum (logsumexp)
+            float lm_fin = have ? l_mma : 0.f;        // row sum of the rounded weights (normalises O)
+            float a_own = 1.f, a_oth = 0.f;           // weights of this tile's O and the other's
+            bool oth = false;                         // warp-uniform: the other tile's O is read too
+            uint32_t tO_oth = 0;
+            if (ilv) {
+                const bool valid = have && l_run > 0.f;
+                const float m_own = valid ? m_run : -INFINITY;
+                float* xs = reinterpret_cast<float*>(sQ + wg * C::Q_TILES * C::TILE_BYTES);
+                const float* xo = reinterpret_cast<const float*>(sQ + (1 - wg) * C::Q_TILES * C::TILE_BYTES);
+                xs[row] = m_own;
+                xs[128 + row] = l_run;
+                xs[256 + row] = l_mma;
+                named_bar_sync(kTcBarMerge, 256);
+                tc_fence_after();   // the other group's o_done wait orders the reads of its O
+                const float m_o = xo[row], lr_o = xo[128 + row], lm_o = xo[256 + row];
+                m_fin = fmaxf(m_own, m_o);
+                a_own = valid ? fast_exp2(m_own - m_fin) : 0.f;
+                a_oth = m_o != -INFINITY ? fast_exp2(m_o - m_fin) : 0.f;
+                l_fin = (valid ? a_own * l_run : 0.f) + (m_o != -INFINITY ? a_oth * lr_o : 0.f);
+                lm_fin = (valid ? a_own * l_mma : 0.f) + (m_o != -INFINITY ? a_oth * lm_o : 0.f);
+                oth = __any_sync(0xffffffffu, m_o != -INFINITY);
+                tO_oth = tmem + lane_base + (wg ? C::COL_O0 : C::COL_O1);
+            }
+            const float inv = lm_fin > 0.f ? 1.f / lm_fin : 0.f;
             // a key split writes its normalised partial O (fp32) and its logsumexp to its slabs
             float* out_f32 = p.o_f32;
             __nv_bfloat16* out_bf16 = p.o;
@@ -973,38 +1066,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 out_bf16 = nullptr;
                 out_lse = p.lse_part + split * rows;
             }
+            // Each thread stores its own row, 16 bytes per instruction.  (Staging the rows in
+            // shared memory for whole-segment stores measured slower on B200 except for the fp32
+            // partials of key splits.)  With interleaved keys warpgroup t writes columns
+            // [t D/2, (t+1) D/2) of the merged O.
             const long orow_off = ((static_cast<long>(b) * p.Sq + qrow) * p.Hq + T.h) * D;
+            const int cb_lo = ilv ? wg * (D / 64) : 0;
+            constexpr int CB_ILV = D / 64;
 #pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
-                uint32_t orr[32];
-                if (have) {
-                    tmem_ld32(tO + cb * 32, orr);
-                    tmem_wait_ld();
-                } else {
+            for (int ci = 0; ci < D / 32; ++ci) {
+                if (ilv && ci >= CB_ILV) break;
+                const int cb = cb_lo + ci;
+                uint32_t orr[32], oro[32];
+                if (have) tmem_ld32(tO + cb * 32, orr);
+                if (oth) tmem_ld32(tO_oth + cb * 32, oro);
+                if (have || oth) tmem_wait_ld();
+                float v[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) orr[e] = 0u;
+                for (int e = 0; e < 32; ++e) {
+                    const float x = have ? a_own * __uint_as_float(orr[e]) : 0.f;
+                    v[e] = (oth ? fmaf(a_oth, __uint_as_float(oro[e]), x) : x) * inv;
                 }
                 if (!store) continue;
                 if (out_f32) {
                     float4* dst = reinterpret_cast<float4*>(out_f32 + orow_off + cb * 32);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dst[e] = make_float4(__uint_as_float(orr[4 * e]) * inv, __uint_as_float(orr[4 * e + 1]) * inv,
-                                             __uint_as_float(orr[4 * e + 2]) * inv, __uint_as_float(orr[4 * e + 3]) * inv);
+                    for (int e = 0; e < 8; ++e) dst[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
                 } else {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
                     uint4* dst = reinterpret_cast<uint4*>(out_bf16 + orow_off + cb * 32);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        dst[e] = make_uint4(pack_bf16x2(v[8 * e], v[8 * e + 1]), pack_bf16x2(v[8 * e + 2], v[8 * e + 3]),
+                                            pack_bf16x2(v[8 * e + 4], v[8 * e + 5]), pack_bf16x2(v[8 * e + 6], v[8 * e + 7]));
                 }
             }
-            if (store && out_lse != nullptr)
+            if (store && out_lse != nullptr && (!ilv || wg == 0))
                 out_lse[(static_cast<long>(b) * p.Hq + T.h) * p.Sq + qrow] =
-                    (have && l_run > 0.f) ? (m_run + fast_log2(l_run)) * kLn2 : -INFINITY;
+                    l_fin > 0.f ? (m_fin + fast_log2(l_fin)) * kLn2 : -INFINITY;
         }
     }
 
