@@ -82,6 +82,31 @@ bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D)
     return make_tmap_bshd_rows(m, ptr, B, S, H, D, 128);
 }
 
+// Output [B][S][H][D] (fp32 or bf16) for TMA stores of 32-column x 128-row boxes: 128-byte rows
+// with the 128-byte swizzle (fp32) or 64-byte rows with the 64-byte swizzle (bf16).
+bool make_tmap_out(CUtensorMap* m, void* ptr, int B, int S, int H, int D, bool f32) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) {
+        cuda_failure("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", "entry point unavailable");
+        return false;
+    }
+    const cuuint64_t es = f32 ? 4 : 2;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * es, (cuuint64_t)H * D * es, (cuuint64_t)S * H * D * es};
+    cuuint32_t box[4] = {32, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = enc(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, ptr, dims,
+                     strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char buf[96];
+        snprintf(buf, sizeof(buf), "CUresult %d (out dims %d,%d,%d,%d)", static_cast<int>(r), D, H, S, B);
+        cuda_failure("cuTensorMapEncodeTiled", buf);
+    }
+    return r == CUDA_SUCCESS;
+}
+
 // fp32 array [rows][cols] viewed 2-D with a box of 128 columns x 1 row, no swizzle; columns past
 // `cols` read as 0.  The row stride (cols * 4 bytes) must be a multiple of 16.
 bool make_tmap_rows_f32(CUtensorMap* m, const void* ptr, long rows, int cols) {
@@ -191,7 +216,11 @@ constexpr int kNumSms = 148;   // B200
 // Key splits of the tensor-core forward.  A bf16 problem whose query tiles fill at most half of
 // the SMs divides each tile's key tiles among up to kMaxKvSplits CTAs (at least two key tiles
 // each), so that the whole GPU works on it; the partials are merged by prefill_combine_kernel.
-// Depends on the sizes only, so the workspace query and the launch agree.
+// A split is taken only when it shortens each CTA's key loop by at least kMinSplitSaving key
+// tiles: the merge costs about as much as that (measured on B200: the Whisper-encoder shape, 12
+// key tiles, runs 1.7 us faster unsplit than in 2 splits + merge).  Depends on the sizes only, so
+// the workspace query and the launch agree.
+constexpr int kMinSplitSaving = 8;
 int fwd_kv_splits(int B, int Hq, int Sq, int Skv, attn_dtype dtype) {
     if (dtype == ATTN_FP32) return 1;
     const long tiles = static_cast<long>((Sq + 127) / 128) * B * Hq;
@@ -200,7 +229,9 @@ int fwd_kv_splits(int B, int Hq, int Sq, int Skv, attn_dtype dtype) {
     const long nkv = (static_cast<long>(Skv) + 127) / 128;
     if (n > nkv / 2) n = nkv / 2;
     if (n > kMaxKvSplits) n = kMaxKvSplits;
-    return n >= 2 ? static_cast<int>(n) : 1;
+    if (n < 2) return 1;
+    const long saved = nkv - (nkv + n - 1) / n;   // key tiles the longest chunk is spared
+    return saved >= kMinSplitSaving ? static_cast<int>(n) : 1;
 }
 
 // RoPE form of the bf16 forward: K rotated once beforehand into hi + lo halves that every CTA
@@ -296,9 +327,16 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     // take alternate key tiles of its one query tile, so that one works while the tensor core
     // serves the other (at D = 128 the ring has too few stages for the pair).
     auto kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true, false> : prefill_tc_kernel<D, ROPE, false, false>;
+    // Their output (or a key split's fp32 partial) leaves through TMA stores; the other kernels
+    // store from the threads and take the query map in that argument's place.
+    CUtensorMap to = tq;
     if constexpr (D == 64) {
-        if (p.single_tile)
+        if (p.single_tile) {
             kern = mk.ptr != nullptr ? prefill_tc_kernel<D, ROPE, true, true> : prefill_tc_kernel<D, ROPE, false, true>;
+            const bool ok = p.kv_splits > 1 ? make_tmap_out(&to, o_part, p.kv_splits * B, Sq, Hq, D, true)
+                                            : make_tmap_out(&to, o, B, Sq, Hq, D, o_f32);
+            if (!ok) return ATTN_ERR_CUDA;
+        }
     }
     const int smem_bytes = TcCfg<D, ROPE>::SMEM_BYTES;
     // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds fewer
@@ -306,7 +344,7 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
     attn_status ps = prepare_kernel(reinterpret_cast<const void*>(kern), smem_bytes, "prefill_tc_kernel set-up",
                                     kTcLaunchRegsMin);
     if (ps != ATTN_OK) return ps;
-    kern<<<static_cast<unsigned>(grid), kTcThreads, smem_bytes, st>>>(tq, tk, tkl, tv, p);
+    kern<<<static_cast<unsigned>(grid), kTcThreads, smem_bytes, st>>>(tq, tk, tkl, tv, to, p);
     attn_status s = launch_status("prefill_tc_kernel");
     if (s != ATTN_OK || p.kv_splits == 1) return s;
     // merge of the key splits, a programmatic dependent launch (it waits for the split grid)

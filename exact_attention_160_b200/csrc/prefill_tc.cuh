@@ -153,7 +153,7 @@ template <int D, int ROPE, bool MASK, bool ILV>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
-    const TcParams p) {
+    const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
     using C = TcCfg<D, ROPE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -233,6 +233,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     // ring index (and key tile, from kv0) of tile t's step j
     auto ring_of = [ilv](int t, int j) { return ilv ? 2 * j + t : j; };
 
+    // TMA copies, issued by thread 0: the query tiles, and K/V of ring index j into slot j % STAGES
+    auto load_q = [&](uint64_t pol) {
+        uint32_t qbytes = 0;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+            if (tile[i].active) qbytes += C::TILE_BYTES;
+        mbar_arrive_expect_tx(bar_q_full, qbytes);
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            if (!tile[i].active) continue;
+            uint8_t* dst = sQ + i * C::Q_TILES * C::TILE_BYTES;
+            for (int bx = 0; bx < C::NBOX; ++bx)
+                tma_load_4d(&tm_q, bar_q_full, dst + bx * (C::TILE_BYTES / C::NBOX), bx * 64, tile[i].h, tile[i].r0, b,
+                            pol);
+        }
+    };
+    auto load_kv = [&](int j, uint64_t pol) {
+        const int s = j % C::STAGES;
+        uint8_t* st = sKV + s * C::STAGE_BYTES;
+        // kRopeKFused: the raw K tile lands in the Kh slot and is rotated there
+        mbar_arrive_expect_tx(bar_k_full + s, (ROPE == kRopeKSplit ? 2 : 1) * C::TILE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx) {
+            tma_load_4d(&tm_k, bar_k_full + s, st + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh, (kv0 + j) * 128, b,
+                        pol);
+            if (ROPE == kRopeKSplit)
+                tma_load_4d(&tm_klo, bar_k_full + s, st + C::TILE_BYTES + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
+                            (kv0 + j) * 128, b, pol);
+        }
+        uint8_t* sv = st + C::K_TILES * C::TILE_BYTES;
+        mbar_arrive_expect_tx(bar_v_full + s, C::TILE_BYTES);
+        for (int bx = 0; bx < C::NBOX; ++bx)
+            tma_load_4d(&tm_v, bar_v_full + s, sv + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh, (kv0 + j) * 128, b,
+                        pol);
+    };
+    // the first ring loads find their slots free: issued during the set-up below
+    const int n_pre = n_loads < C::STAGES ? n_loads : C::STAGES;
+
     // ---- set-up --------------------------------------------------------------------------
     if (tid == 0) {
         mbar_init(bar_q_full, 1);
@@ -256,12 +293,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             mbar_init(bar_pv_done + i, 1);
         }
         mbar_fence_init();
-    }
-    if (warp == 0 && lane == 0) {
+        // The copies go out now, while the tensor memory is allocated and the block synchronises
+        // (the barriers they signal are initialised; nothing else touches their destinations).
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         if (ROPE == kRopeKSplit) tma_prefetch_desc(&tm_klo);
+        load_q(l2_policy_evict_first());
+        const uint64_t pol_kv = l2_policy_evict_last();
+        for (int j = 0; j < n_pre; ++j) load_kv(j, pol_kv);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, 512);
@@ -283,23 +323,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
       if (warp == 0) {
         // =============================== TMA producer ===================================
         if (lane == 0) {
-            const uint64_t pol_q = l2_policy_evict_first();
             const uint64_t pol_kv = l2_policy_evict_last();
-            uint32_t qbytes = 0;
-#pragma unroll
-            for (int i = 0; i < 2; ++i)
-                if (tile[i].active) qbytes += C::TILE_BYTES;
-            mbar_arrive_expect_tx(bar_q_full, qbytes);
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                if (!tile[i].active) continue;
-                uint8_t* dst = sQ + i * C::Q_TILES * C::TILE_BYTES;
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    tma_load_4d(&tm_q, bar_q_full, dst + bx * (C::TILE_BYTES / C::NBOX), bx * 64, tile[i].h,
-                                tile[i].r0, b, pol_q);
-            }
-            int issued = 0;
-            for (int j = 0; j < n_loads; ++j) {
+            int issued = n_pre;   // the query tiles and ring loads [0, n_pre) went out in the set-up
+            for (int j = n_pre; j < n_loads; ++j) {
                 const int s = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
                 // EARLY: each MMA thread releases the stages its own tile used (j - STAGES < n_t);
@@ -311,21 +337,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     freed = mbar_wait(bar_kv_empty + C::STAGES + s, ph ^ 1);
                 if (!freed) break;
                 issued = j + 1;
-                uint8_t* st = sKV + s * C::STAGE_BYTES;
-                // kRopeKFused: the raw K tile lands in the Kh slot and is rotated there
-                mbar_arrive_expect_tx(bar_k_full + s, (ROPE == kRopeKSplit ? 2 : 1) * C::TILE_BYTES);
-                for (int bx = 0; bx < C::NBOX; ++bx) {
-                    tma_load_4d(&tm_k, bar_k_full + s, st + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
-                                (kv0 + j) * 128, b, pol_kv);
-                    if (ROPE == kRopeKSplit)
-                        tma_load_4d(&tm_klo, bar_k_full + s, st + C::TILE_BYTES + bx * (C::TILE_BYTES / C::NBOX),
-                                    bx * 64, kvh, (kv0 + j) * 128, b, pol_kv);
-                }
-                uint8_t* sv = st + C::K_TILES * C::TILE_BYTES;
-                mbar_arrive_expect_tx(bar_v_full + s, C::TILE_BYTES);
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    tma_load_4d(&tm_v, bar_v_full + s, sv + bx * (C::TILE_BYTES / C::NBOX), bx * 64, kvh,
-                                (kv0 + j) * 128, b, pol_kv);
+                load_kv(j, pol_kv);
             }
             // no copy may still be landing in shared memory when the CTA exits
             mbar_wait(bar_q_full, 0);
@@ -1070,13 +1082,55 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             // shared memory for whole-segment stores measured slower on B200 except for the fp32
             // partials of key splits.)  With interleaved keys warpgroup t writes columns
             // [t D/2, (t+1) D/2) of the merged O.
+            if constexpr (ilv) {
+                // Interleaved keys (D = 64): warpgroup t's half of the output, 32 columns of the
+                // tile's 128 rows, leaves through one TMA store.  Each thread writes its row into
+                // a box in the K/V ring (free: both tiles' products are done) in the store's
+                // swizzled layout -- 16-byte chunk c of row r at chunk c ^ (r & 7) of a 128-byte
+                // row (fp32), or c ^ ((r >> 1) & 3) of a 64-byte row (bf16) -- which keeps the
+                // row-per-thread writes free of bank conflicts; rows past Sq are clipped by the
+                // store.  (Direct stores from the threads touch a different line per lane.)
+                static_assert(D == 64, "interleaved keys: one 32-column block per warpgroup");
+                uint32_t orr[32], oro[32];
+                if (have) tmem_ld32(tO + wg * 32, orr);
+                if (oth) tmem_ld32(tO_oth + wg * 32, oro);
+                if (have || oth) tmem_wait_ld();
+                float v[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const float x = have ? a_own * __uint_as_float(orr[e]) : 0.f;
+                    v[e] = (oth ? fmaf(a_oth, __uint_as_float(oro[e]), x) : x) * inv;
+                }
+                uint8_t* box = sKV + wg * 16384;   // 1024-byte aligned
+                if (out_f32) {
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        *reinterpret_cast<float4*>(box + row * 128 + ((c ^ (row & 7)) << 4)) =
+                            make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c)
+                        *reinterpret_cast<uint4*>(box + row * 64 + ((c ^ ((row >> 1) & 3)) << 4)) =
+                            make_uint4(pack_bf16x2(v[8 * c], v[8 * c + 1]), pack_bf16x2(v[8 * c + 2], v[8 * c + 3]),
+                                       pack_bf16x2(v[8 * c + 4], v[8 * c + 5]), pack_bf16x2(v[8 * c + 6], v[8 * c + 7]));
+                }
+                fence_proxy_async_smem();
+                if (wg == 0)
+                    named_bar_sync(kTcBarGroup0, 128);
+                else
+                    named_bar_sync(kTcBarGroup0 + 1, 128);
+                if (row == 0) {
+                    // the map covers [B'][Sq][Hq][D] with B' = kv_splits * B: split s, batch b at s B + b
+                    tma_store_4d(&tm_o, box, wg * 32, T.h, T.r0, (p.kv_splits > 1 ? split * p.B : 0) + b);
+                    tma_store_commit();
+                    tma_store_wait_all();
+                }
+            }
             const long orow_off = ((static_cast<long>(b) * p.Sq + qrow) * p.Hq + T.h) * D;
-            const int cb_lo = ilv ? wg * (D / 64) : 0;
-            constexpr int CB_ILV = D / 64;
 #pragma unroll
             for (int ci = 0; ci < D / 32; ++ci) {
-                if (ilv && ci >= CB_ILV) break;
-                const int cb = cb_lo + ci;
+                if (ilv) break;
+                const int cb = ci;
                 uint32_t orr[32], oro[32];
                 if (have) tmem_ld32(tO + cb * 32, orr);
                 if (oth) tmem_ld32(tO_oth + cb * 32, oro);

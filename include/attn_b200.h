@@ -150,8 +150,9 @@ size_t attn_fwd_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int Skv, int D
                                   float rope_base, int q_pos0);
 
 /* Key splits attn_fwd_ex uses for these sizes when given its workspace (1: unsplit):
- * min(148 / tiles, ceil(Skv/128) / 2, 16) for bf16 problems with tiles = ceil(Sq/128) * B * Hq
- * <= 74, when that is >= 2; 1 otherwise (and for ATTN_FP32).  Sizes <= 0 give 1.              */
+ * n = min(148 / tiles, nkv / 2, 16) for bf16 problems with tiles = ceil(Sq/128) * B * Hq <= 74
+ * and nkv = ceil(Skv/128), when n >= 2 and the split spares the longest chunk at least 8 key
+ * tiles (nkv - ceil(nkv / n) >= 8); 1 otherwise (and for ATTN_FP32).  Sizes <= 0 give 1.      */
 int attn_fwd_kv_splits(int B, int Hq, int Sq, int Skv, attn_dtype dtype);
 
 /*

@@ -71,24 +71,28 @@ def test_fwd_ex_validation(lib):
 
 
 def test_fwd_key_split_sizing(lib):
-    """Key splits: min(148 // tiles, ceil(Skv/128) // 2, 16) for bf16 problems of <= 74 query tiles;
-    their partials (splits x rows x (D + 1) floats) follow the RoPE part of the workspace."""
-    assert lib.attn_fwd_kv_splits(1, 6, 1500, 1500, 0) == 2      # 72 tiles, 12 key tiles
+    """Key splits: n = min(148 // tiles, ceil(Skv/128) // 2, 16) for bf16 problems of <= 74 query
+    tiles, taken when they spare the longest chunk >= 8 key tiles; their partials (splits x rows x
+    (D + 1) floats) follow the RoPE part of the workspace."""
+    assert lib.attn_fwd_kv_splits(1, 6, 1500, 1500, 0) == 1      # 72 tiles, 12 key tiles: spares 6
+    assert lib.attn_fwd_kv_splits(1, 2, 1500, 2100, 0) == 6      # 24 tiles, 17 key tiles: spares 14
     assert lib.attn_fwd_kv_splits(1, 8, 128, 4096, 0) == 16      # 8 tiles, 32 key tiles
-    assert lib.attn_fwd_kv_splits(1, 2, 300, 1000, 2) == 4       # bf16 in, fp32 out
+    assert lib.attn_fwd_kv_splits(1, 2, 300, 2100, 2) == 8       # bf16 in, fp32 out
+    assert lib.attn_fwd_kv_splits(1, 2, 300, 1000, 2) == 1       # 8 key tiles in 4 chunks: spares 6
     assert lib.attn_fwd_kv_splits(4, 8, 2048, 2048, 0) == 1      # 512 tiles
     assert lib.attn_fwd_kv_splits(1, 2, 300, 300, 0) == 1        # 3 key tiles
-    assert lib.attn_fwd_kv_splits(1, 6, 1500, 1500, 1) == 1      # fp32 path
-    assert lib.attn_fwd_kv_splits(0, 6, 1500, 1500, 0) == 1
-    rows = 1500 * 6
-    part = -(-2 * rows * 64 * 4 // 256) * 256 + -(-2 * rows * 4 // 256) * 256
-    assert lib.attn_fwd_ex_workspace_size(1, 6, 6, 1500, 1500, 64, 0, 0.0, 0) == part
-    # RoPE part: cos/sin table (1500 positions x 32 pairs x 8 B), then K hi and lo (bf16)
-    rope = 1500 * 32 * 8 + 2 * (1500 * 6 * 64 * 2)
-    assert lib.attn_fwd_ex_workspace_size(1, 6, 6, 1500, 1500, 64, 0, 10000.0, 0) == rope + part
+    assert lib.attn_fwd_kv_splits(1, 8, 128, 4096, 1) == 1       # fp32 path
+    assert lib.attn_fwd_kv_splits(0, 8, 128, 4096, 0) == 1
+    rows = 128 * 8
+    part = -(-16 * rows * 64 * 4 // 256) * 256 + -(-16 * rows * 4 // 256) * 256
+    assert lib.attn_fwd_ex_workspace_size(1, 8, 2, 128, 4096, 64, 0, 0.0, 0) == part
+    assert lib.attn_fwd_ex_workspace_size(1, 6, 6, 1500, 1500, 64, 0, 0.0, 0) == 0   # unsplit, no RoPE
+    # RoPE part: cos/sin table (4096 positions x 32 pairs x 8 B), then K hi and lo (bf16)
+    rope = 4096 * 32 * 8 + 2 * (4096 * 2 * 64 * 2)
+    assert lib.attn_fwd_ex_workspace_size(1, 8, 2, 128, 4096, 64, 0, 10000.0, 0) == rope + part
     # a non-NULL workspace below the size is refused before any launch
     P = FAKE
-    assert lib.attn_fwd_ex(P, P, P, P, None, 1, 6, 6, 1500, 1500, 64, 0.125, 0, 0, 0.0, 0, P, part - 1,
+    assert lib.attn_fwd_ex(P, P, P, P, None, 1, 8, 2, 128, 4096, 64, 0.125, 0, 0, 0.0, 0, P, part - 1,
                            None) == 5
 
 
@@ -98,8 +102,11 @@ def test_key_split_count_follows_its_documented_rule(lib):
         tiles = -(-Sq // 128) * B * Hq
         if dtype == 1 or tiles > 74:
             return 1
-        n = min(148 // tiles, -(-Skv // 128) // 2, 16)
-        return n if n >= 2 else 1
+        nkv = -(-Skv // 128)
+        n = min(148 // tiles, nkv // 2, 16)
+        if n < 2:
+            return 1
+        return n if nkv - (-(-nkv // n)) >= 8 else 1
     for B in (1, 2, 3):
         for Hq in (1, 2, 6, 8, 32):
             for Sq in (1, 127, 128, 129, 700, 1500, 4096):

@@ -20,20 +20,22 @@ def P(name, B, Hq, Hkv, Sq, Skv, D, causal, **kw):
     return si.Prefill(name, "bf16", B, Hq, Hkv, Sq, Skv, D, causal, scale, seed=kw.pop("seed", 501), **kw)
 
 
-# (workload, splits): splits = min(148 // tiles, ceil(Skv/128) // 2, 16) with
-# tiles = ceil(Sq/128) * B * Hq <= 74
+# (workload, splits): n = min(148 // tiles, nkv // 2, 16) with tiles = ceil(Sq/128) * B * Hq <= 74
+# and nkv = ceil(Skv/128), taken when nkv - ceil(nkv / n) >= 8
 CASES = [
-    (P("noncausal_ragged", 1, 4, 4, 700, 900, 64, False), 4),              # 24 tiles, 8 key tiles
-    (P("causal_empty_chunks", 1, 2, 2, 1024, 1024, 64, True), 4),          # row tile 0: 3 empty chunks
+    (P("noncausal_ragged", 1, 4, 4, 700, 2100, 64, False), 6),             # 24 tiles, 17 key tiles
+    (P("causal_empty_chunks", 1, 1, 1, 2048, 2048, 64, True), 8),          # row tile 0: 7 empty chunks
     (P("decode_like_gqa", 1, 8, 2, 128, 4096, 64, True, seed=502), 16),    # 8 tiles, 32 key tiles
     # offset 64: rows 0..63 of tile 0 see no key of its second chunk (partial lse = -inf)
-    (P("offset64_masked_partials", 1, 2, 2, 960, 1024, 64, True, seed=503), 4),
+    (P("offset64_masked_partials", 1, 1, 1, 1984, 2048, 64, True, seed=503), 8),
     (P("rope_gqa_offset", 1, 8, 2, 256, 2048, 64, True, rope_base=10000.0, q_pos0=1792, seed=504), 8),
-    (P("d128_peaked", 1, 2, 2, 640, 640, 128, True, qk_std=3.0, seed=505), 2),
+    (P("d128_peaked", 1, 2, 2, 2048, 2048, 128, True, qk_std=3.0, seed=505), 4),
     (P("d128_noncausal_gqa", 2, 4, 2, 130, 1200, 128, False, seed=506), 5),
     # Sq > Skv, causal: rows 0..179 see no key at all (O = 0, LSE = -inf in every partial)
-    (P("sq_gt_skv_dead_rows", 1, 2, 2, 700, 520, 64, True, seed=507), 2),
-    (P("padded_d80", 1, 2, 2, 300, 1000, 80, False, seed=508), 4),
+    (P("sq_gt_skv_dead_rows", 1, 1, 1, 2200, 2020, 64, True, seed=507), 8),
+    (P("padded_d80", 1, 2, 2, 300, 2100, 80, False, seed=508), 8),
+    # the Whisper-encoder shape (12 key tiles) runs unsplit: two chunks would spare only 6
+    (P("whisper_shape_unsplit", 1, 6, 6, 1500, 1500, 64, False, seed=510), 1),
 ]
 
 
@@ -81,12 +83,12 @@ def test_split_is_deterministic_and_stays_in_bounds():
 
 
 def test_split_with_additive_mask():
-    w = P("masked_split", 1, 4, 4, 300, 1100, 64, False, seed=509)
+    w = P("masked_split", 1, 4, 4, 300, 2200, 64, False, seed=509)
     x, dev = make_prefill(w)
-    assert ea.fwd_kv_splits(dev["q"], dev["k"], torch.float32) == 4     # 12 tiles, 9 key tiles
+    assert ea.fwd_kv_splits(dev["q"], dev["k"], torch.float32) == 9     # 12 tiles, 18 key tiles
     rng = np.random.default_rng(w.seed)
     m = rng.standard_normal((w.Sq, w.Skv)).astype(np.float32)
-    m[:, 700:] = -np.inf       # the last key tiles masked out: whole chunks without a visible key
+    m[:, 1500:] = -np.inf      # the last key tiles masked out: whole chunks without a visible key
     m[[3, 200], :] = -np.inf   # rows masked everywhere
     o, lse = ea.attn_fwd_masked(dev["q"], dev["k"], dev["v"], torch.from_numpy(m).cuda(), w.scale, False,
                                 out_dtype=torch.float32)
