@@ -102,8 +102,14 @@ struct TcCfg {
     // markedly slower on B200.)
     // EARLY: S_t, O_t (64) and P_t (64) fill the half: S0 [0,128) O0 [128,192) P0 [192,256),
     // S1 [256,384) O1 [384,448) P1 [448,512).
+    // D=64 with the ones block (P_SPLIT): keys [0, 64) of P_t go over the first 32 columns of S_t,
+    // keys [64, 128) into the 32 columns after O_t (O_t takes N_PV = 80 of the 128 after S_t), so
+    // that S_t(j+1) may overwrite S_t as soon as the first half of PV_t(j) has read its P.
+    static constexpr bool P_SPLIT = ONES;
     static constexpr uint32_t COL_S0 = 0, COL_O0 = 128, COL_P0 = EARLY ? 192 : 0;
     static constexpr uint32_t COL_S1 = 256, COL_O1 = 384, COL_P1 = EARLY ? 448 : 256;
+    static constexpr uint32_t COL_PH0 = COL_O0 + N_PV, COL_PH1 = COL_O1 + N_PV;   // P_SPLIT: keys [64, 128)
+    static_assert(!P_SPLIT || COL_PH1 + 32 <= 512, "TMEM columns");
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -190,6 +196,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     // interleaved keys (below) need ring slots to spare: each step of the pair takes two
     static_assert(!ILV || C::STAGES >= 3, "interleaved keys need three K/V stages or more");
     constexpr bool ilv = ILV;
+    // D=64 with the ones block (no RoPE): each query tile gets an MMA thread of its own (warps 1
+    // and 2), as in the EARLY layout, so that neither tile's products wait behind the other
+    // tile's hand-offs; a tcgen05.mma issue blocks while the tensor core is busy, which made one
+    // thread issuing both tiles' products in a fixed order the pacing resource.
+    constexpr bool kOnesTwoIssuers = C::ONES && ROPE != kRopeKFused;
+    constexpr bool kPerTileMma = C::EARLY || kOnesTwoIssuers;   // one MMA thread per query tile
     TcTile tile[2];
     if (p.single_tile) {
         tile[0].h = tile[1].h = hi;
@@ -280,7 +292,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             mbar_init(bar_p_ready + 2 * i + 1, 128);
             mbar_init(bar_o_done + i, 1);
         }
-        mbar_init(bar_mma_final, C::EARLY ? 2 : 1);   // one commit per MMA thread
+        mbar_init(bar_mma_final, kPerTileMma ? 2 : 1);   // one commit per MMA thread
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(bar_k_full + s, 1);
             mbar_init(bar_v_full + s, 1);
@@ -331,9 +343,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 // EARLY: each MMA thread releases the stages its own tile used (j - STAGES < n_t);
                 // interleaved keys: a slot serves one tile at a time, released on bar_kv_empty[s]
                 bool freed = true;
-                if (!C::EARLY || ilv || j < C::STAGES || j - C::STAGES < tile[0].nkv)
+                if (!kPerTileMma || ilv || j < C::STAGES || j - C::STAGES < tile[0].nkv)
                     freed = mbar_wait(bar_kv_empty + s, ph ^ 1);
-                if (C::EARLY && !ilv && freed && (j < C::STAGES || j - C::STAGES < tile[1].nkv))
+                if (kPerTileMma && !ilv && freed && (j < C::STAGES || j - C::STAGES < tile[1].nkv))
                     freed = mbar_wait(bar_kv_empty + C::STAGES + s, ph ^ 1);
                 if (!freed) break;
                 issued = j + 1;
@@ -436,9 +448,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             mma_commit(bar_mma_final);
             mbar_wait(bar_mma_final, 0);
         }
-      } else if (warp == 1) {
-        // =============================== MMA issuer ======================================
-        // One thread issues every MMA of both query tiles, interleaved per KV tile j as
+      } else if (warp == 1 || (kOnesTwoIssuers && warp == 2)) {
+        // =============================== MMA issuer(s) ===================================
+        // kOnesTwoIssuers: warp 1 issues the MMAs of query tile 0, warp 2 those of tile 1, each
+        // per KV tile j as  PV_t(j) first half, S_t(j+1), PV_t(j) second half  (P_SPLIT: the
+        // second half of P_t(j) does not sit in S_t's columns), releasing its stages on a barrier
+        // of its own (interleaved keys: the one of the slot, which serves one tile).
+        // Otherwise one thread issues every MMA of both query tiles, interleaved per KV tile j as
         //   PV_0(j)  S_0(j+1)  PV_1(j)  S_1(j+1)
         // where S_t(j) = Q_t K_j^T (-> s_full_t) and PV_t(j): O_t += P_t(j) V_j.  The tensor core
         // runs one thread's MMAs in issue order, so S_t(j+1) overwrites the columns of P_t(j)
@@ -490,7 +506,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             // that half of P_t(j), so the product overlaps the exponentials of the other half
             auto issue_pv_half = [&](int t, int j, int half) {
                 const uint32_t dO = tmem + (t ? C::COL_O1 : C::COL_O0);
-                const uint32_t aP = tmem + (t ? C::COL_S1 : C::COL_S0);
+                // P_SPLIT: the second half of P sits after O_t
+                const uint32_t aP = (C::P_SPLIT && half) ? tmem + (t ? C::COL_PH1 : C::COL_PH0) - 32
+                                                         : tmem + (t ? C::COL_S1 : C::COL_S0);
                 const uint32_t vlo = v_lo(ring_of(t, j) % C::STAGES);
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
@@ -499,6 +517,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     mma_ts(dO, aP + kk * 8, desc_join(vlo + kk * (2048 >> 4), hiK), idesc_pv,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 }
+                if (C::P_SPLIT && half == 1) mma_commit(bar_pv_done + t);   // P_t's second half is free again
                 if (half == 1 && j == (t ? nt1 : nt0) - 1) mma_commit(bar_o_done + t);
             };
             auto wait_k = [&](int u) {   // K of ring index u in place
@@ -508,6 +527,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 return r;
             };
             const int nkv_all = max(nt0, nt1);
+            if constexpr (kOnesTwoIssuers) {
+                const int t = warp - 1;
+                const int n = t ? nt1 : nt0;
+                if (ok && n > 0) {
+                    ok = wait_k(ring_of(t, 0));
+                    if (ok) issue_s(t, 0);
+                }
+                for (int j = 0; j < n; ++j) {
+                    const int u = ring_of(t, j), s = u % C::STAGES;
+                    if (ok) {
+                        ok = mbar_wait(bar_v_full + s, (u / C::STAGES) & 1);
+                        tc_fence_after();
+                    }
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        if (ok) {
+                            ok = mbar_wait(bar_p_ready + 2 * t + half, j & 1);
+                            tc_fence_after();
+                        }
+                        if (ok) issue_pv_half(t, j, half);
+                        if (half == 0 && ok && j + 1 < n) {
+                            ok = wait_k(ring_of(t, j + 1));
+                            if (ok) issue_s(t, j + 1);
+                        }
+                    }
+                    mma_commit(bar_kv_empty + (ilv ? 0 : t * C::STAGES) + s);   // this tile is done with stage s
+                }
+                if (!ok) mma_commit(bar_o_done + t);
+            } else {
             if (ok && nkv_all > 0) {
                 ok = wait_k(0);
                 if (ok && nt0 > 0) issue_s(0, 0);
@@ -533,12 +581,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                             tc_fence_after();
                         }
                         if (ok) issue_pv_half(t, j, half);
+                        // P_SPLIT: S_t(j+1) may follow the first half of PV_t(j)
+                        if (half == (C::P_SPLIT ? 0 : 1) && ok && j + 1 < n) {
+                            ok = wait_k(u + 2);
+                            if (ok) issue_s(t, j + 1);
+                        }
                     }
                     mma_commit(bar_kv_empty + s);
-                    if (ok && j + 1 < n) {
-                        ok = wait_k(u + 2);
-                        if (ok) issue_s(t, j + 1);
-                    }
                 }
             }
             for (int j = 0; !ilv && j < nkv_all; ++j) {
@@ -559,11 +608,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                             tc_fence_after();
                         }
                         if (ok) issue_pv_half(t, j, half);
-                    }
-                    if (EARLY_S && ok && j + 1 < n) {
-                        if (!k_next) ok = wait_k(j + 1);
-                        k_next = true;
-                        if (ok) issue_s(t, j + 1);
+                        // P_SPLIT: S_t(j+1) may follow the first half of PV_t(j)
+                        if (half == (C::P_SPLIT ? 0 : 1) && EARLY_S && ok && j + 1 < n) {
+                            if (!k_next) ok = wait_k(j + 1);
+                            k_next = true;
+                            if (ok) issue_s(t, j + 1);
+                        }
                     }
                 }
                 // stage s is free once every MMA issued so far has completed
@@ -578,6 +628,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             if (!ok) {
                 mma_commit(bar_o_done + 0);
                 mma_commit(bar_o_done + 1);
+            }
             }
             // every MMA issued above must be complete before tensor memory is released
             mma_commit(bar_mma_final);
@@ -702,7 +753,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         float l_run = 0.f;         // row sum of the fp32 weights (logsumexp)
         float l_mma = 0.f;         // row sum of the bf16-rounded weights (normalises O)
         const float sl2 = p.scale_log2;
-        const uint32_t tP = tS;    // P_t(j) is written over the first 64 columns of S_t
+        const uint32_t tP = tS;    // P_t(j) is written over the first 64 columns of S_t ...
+        // ... or, P_SPLIT, its keys [64, 128) after O_t
+        const uint32_t tPh = tmem + lane_base + (wg ? C::COL_PH1 : C::COL_PH0);
         if constexpr (C::EARLY) {
         // Exponentiation turns: warpgroup 0 exponentiates, then warpgroup 1, alternately; each
         // group's loads, row max, stores and hand-offs overlap the other group's exponentials.
@@ -947,9 +1000,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                 m_run = tmax;
             }
             // O correction, only in warps with a rescaling row and once O holds earlier blocks.
-            // O_t is at rest here: PV_t(j-1) completed before s_full_t(j) was signalled, and
-            // PV_t(j) is issued only after this warpgroup's p_ready arrival below.
+            // PV_t(j) is issued only after this warpgroup's p_ready arrivals below; PV_t(j-1) had
+            // completed before s_full_t(j) was signalled, except (P_SPLIT) its second half, which
+            // follows S_t(j) and is waited for here (and before the second half of P_t(j) takes
+            // its columns).
+            bool pv_prev = !(C::P_SPLIT && j > 0);   // PV_t(j-1) known complete
+            auto wait_pv_prev = [&]() {
+                if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) ok = false;
+                tc_fence_after();
+                pv_prev = true;
+            };
             if (j > 0 && __any_sync(0xffffffffu, need)) {
+                if (!pv_prev) wait_pv_prev();
 #pragma unroll
                 for (int cb = 0; cb < (C::N_PV + 31) / 32; ++cb) {
                     uint32_t orr[32];
@@ -985,7 +1047,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     if (!C::ONES)
                         lr2[e & 3] = f2_add(lr2[e & 3], f2_pack(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                 }
-                tmem_st16(tP + cb * 16, pk);
+                if (C::P_SPLIT && cb == 2 && !pv_prev) wait_pv_prev();
+                tmem_st16((C::P_SPLIT && cb >= 2) ? tPh + (cb - 2) * 16 : tP + cb * 16, pk);
                 if (cb == 1) {
                     // keys [0, 64) of P are in TMEM: the first half of PV may start
                     tmem_wait_st();
