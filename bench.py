@@ -551,7 +551,7 @@ def roofline_backward(flop: float, ms: float, peaks, how: str):
 
 def profile_name(w) -> str:
     return {si.C2.name: "prefill_tc_c2", si.C3.name: "prefill_tc_c3", si.C5.name: "prefill_tc_c5",
-            si.C4.name: "decode_split_c4", si.F2_WHISPER.name: "prefill_tc_whisper_split"}.get(w.name, "")
+            si.C4.name: "decode_split_c4", si.F2_WHISPER.name: "prefill_tc_whisper"}.get(w.name, "")
 
 
 # ------------------------------------------------------------------------------------------

@@ -200,7 +200,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     // and 2), as in the EARLY layout, so that neither tile's products wait behind the other
     // tile's hand-offs; a tcgen05.mma issue blocks while the tensor core is busy, which made one
     // thread issuing both tiles' products in a fixed order the pacing resource.
-    constexpr bool kOnesTwoIssuers = C::ONES && ROPE != kRopeKFused;
+    // The masked kernel keeps one MMA thread and P over S: its softmax is bound by the per-row
+    // mask loads, and the two groups' loads in step (which the per-tile MMA threads bring about)
+    // measured 11% slower on B200.
+    constexpr bool kOnesTwoIssuers = C::ONES && ROPE != kRopeKFused && !MASK;
+    constexpr bool kPSplit = C::P_SPLIT && !MASK;   // P's second half after O (TMEM layout above)
     constexpr bool kPerTileMma = C::EARLY || kOnesTwoIssuers;   // one MMA thread per query tile
     TcTile tile[2];
     if (p.single_tile) {
@@ -507,7 +511,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             auto issue_pv_half = [&](int t, int j, int half) {
                 const uint32_t dO = tmem + (t ? C::COL_O1 : C::COL_O0);
                 // P_SPLIT: the second half of P sits after O_t
-                const uint32_t aP = (C::P_SPLIT && half) ? tmem + (t ? C::COL_PH1 : C::COL_PH0) - 32
+                const uint32_t aP = (kPSplit && half) ? tmem + (t ? C::COL_PH1 : C::COL_PH0) - 32
                                                          : tmem + (t ? C::COL_S1 : C::COL_S0);
                 const uint32_t vlo = v_lo(ring_of(t, j) % C::STAGES);
 #pragma unroll
@@ -517,7 +521,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     mma_ts(dO, aP + kk * 8, desc_join(vlo + kk * (2048 >> 4), hiK), idesc_pv,
                            (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (C::P_SPLIT && half == 1) mma_commit(bar_pv_done + t);   // P_t's second half is free again
+                if (kPSplit && half == 1) mma_commit(bar_pv_done + t);   // P_t's second half is free again
                 if (half == 1 && j == (t ? nt1 : nt0) - 1) mma_commit(bar_o_done + t);
             };
             auto wait_k = [&](int u) {   // K of ring index u in place
@@ -582,7 +586,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                         }
                         if (ok) issue_pv_half(t, j, half);
                         // P_SPLIT: S_t(j+1) may follow the first half of PV_t(j)
-                        if (half == (C::P_SPLIT ? 0 : 1) && ok && j + 1 < n) {
+                        if (half == (kPSplit ? 0 : 1) && ok && j + 1 < n) {
                             ok = wait_k(u + 2);
                             if (ok) issue_s(t, j + 1);
                         }
@@ -609,7 +613,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                         }
                         if (ok) issue_pv_half(t, j, half);
                         // P_SPLIT: S_t(j+1) may follow the first half of PV_t(j)
-                        if (half == (C::P_SPLIT ? 0 : 1) && EARLY_S && ok && j + 1 < n) {
+                        if (half == (kPSplit ? 0 : 1) && EARLY_S && ok && j + 1 < n) {
                             if (!k_next) ok = wait_k(j + 1);
                             k_next = true;
                             if (ok) issue_s(t, j + 1);
@@ -1004,7 +1008,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             // completed before s_full_t(j) was signalled, except (P_SPLIT) its second half, which
             // follows S_t(j) and is waited for here (and before the second half of P_t(j) takes
             // its columns).
-            bool pv_prev = !(C::P_SPLIT && j > 0);   // PV_t(j-1) known complete
+            bool pv_prev = !(kPSplit && j > 0);   // PV_t(j-1) known complete
             auto wait_pv_prev = [&]() {
                 if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_pv_done + wg, (j - 1) & 1))) ok = false;
                 tc_fence_after();
@@ -1047,8 +1051,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                     if (!C::ONES)
                         lr2[e & 3] = f2_add(lr2[e & 3], f2_pack(bf16lo_to_f32(pk[e]), bf16hi_to_f32(pk[e])));
                 }
-                if (C::P_SPLIT && cb == 2 && !pv_prev) wait_pv_prev();
-                tmem_st16((C::P_SPLIT && cb >= 2) ? tPh + (cb - 2) * 16 : tP + cb * 16, pk);
+                if (kPSplit && cb == 2 && !pv_prev) wait_pv_prev();
+                tmem_st16((kPSplit && cb >= 2) ? tPh + (cb - 2) * 16 : tP + cb * 16, pk);
                 if (cb == 1) {
                     // keys [0, 64) of P are in TMEM: the first half of PV may start
                     tmem_wait_st();
