@@ -203,6 +203,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     // The masked kernel keeps one MMA thread and P over S: its softmax is bound by the per-row
     // mask loads, and the two groups' loads in step (which the per-tile MMA threads bring about)
     // measured 11% slower on B200.
+    // (At D=128 an MMA thread per tile measured 1.27 ms on C5 against 0.97: there the tensor work
+    // per step is twice as large and one thread's interleaved order keeps the pipe busier.)
     constexpr bool kOnesTwoIssuers = C::ONES && ROPE != kRopeKFused && !MASK;
     constexpr bool kPSplit = C::P_SPLIT && !MASK;   // P's second half after O (TMEM layout above)
     constexpr bool kPerTileMma = C::EARLY || kOnesTwoIssuers;   // one MMA thread per query tile
@@ -551,7 +553,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
                             tc_fence_after();
                         }
                         if (ok) issue_pv_half(t, j, half);
-                        if (half == 0 && ok && j + 1 < n) {
+                        // S_t(j+1) overwrites S_t: after the PV half that reads P from there
+                        if (half == (kPSplit ? 0 : 1) && ok && j + 1 < n) {
                             ok = wait_k(ring_of(t, j + 1));
                             if (ok) issue_s(t, j + 1);
                         }
