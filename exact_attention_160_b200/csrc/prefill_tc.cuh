@@ -12,19 +12,27 @@
 //   * One CTA holds two 128-row query tiles that read the same K/V: two q heads of one GQA group
 //     at the same rows when the group size is even, else two consecutive row tiles of one head.
 //     Each K/V tile is therefore loaded once for 256 query rows.  A problem small enough that its
-//     single tiles fit in one wave of the SMs runs one tile per CTA (the second tile inactive).
+//     single tiles fit in one wave of the SMs runs one tile per CTA; at D=64 the CTA's two softmax
+//     warpgroups then take alternate key tiles of that tile (interleaved keys, ILV), each with its
+//     own online-softmax state, and the epilogue merges the two states (at D=128 the second
+//     warpgroup idles).
 //   * Warp roles (3 warpgroups): warp 0 issues TMA loads (Q once, then a ring of K/V stages);
-//     warp 1 owns tensor memory and one of its threads issues every tcgen05.mma of the CTA from
-//     precomputed shared-memory descriptors; warps 4-7 and 8-11 are the softmax warpgroups of
-//     query tile 0 and 1, one thread per query row (a warp may only touch TMEM lanes
+//     warp 1 owns tensor memory; the tcgen05.mma of the CTA are issued from precomputed
+//     shared-memory descriptors by one thread of warp 1 (D=128), or by one thread of warp 1 for
+//     query tile 0 and one of warp 2 for tile 1 (D=64); warps 4-7 and 8-11 are the softmax
+//     warpgroups of query tile 0 and 1, one thread per query row (a warp may only touch TMEM lanes
 //     32*(warp%4) .. +31, so the row of a softmax thread is 32*(warp%4) + lane).
 //   * S = Q K^T is a bf16 MMA (A and B from shared memory, M=128, N=128) into TMEM; the softmax
 //     threads read their row of S with tcgen05.ld, compute P = exp2(S*scale*log2e - m) in fp32,
 //     round P to bf16 and write it back to TMEM over S; O += P V is an MMA with A = P from TMEM
 //     and B = V from shared memory (N = D), accumulating in TMEM.
-//   * The MMA thread interleaves the tiles per KV tile j as PV_0(j), S_0(j+1), PV_1(j), S_1(j+1):
-//     while one softmax warpgroup exponentiates its tile, the tensor core runs the other tile's
-//     two products, so the groups fall into alternating phases without any turn-taking barrier.
+//   * D=128: the MMA thread interleaves the tiles per KV tile j as PV_0(j), S_0(j+1), PV_1(j),
+//     S_1(j+1): while one softmax warpgroup exponentiates its tile, the tensor core runs the other
+//     tile's two products.  D=64 without RoPE: each tile's MMA thread issues PV_t(j) first half,
+//     S_t(j+1), PV_t(j) second half (P's second half lives outside S's columns), so S_t(j+1) runs
+//     while the second half of S_t(j) is exponentiated.  D=64 with RoPE (EARLY): P has columns of
+//     its own, S_t(j+1) is issued as soon as the softmax holds S_t(j) in registers, and the two
+//     softmax warpgroups take turns for their exponentials.
 //   * Lazy rescale: the running max used for the exponent only moves when the block max exceeds
 //     it by more than kRescaleThreshold (log2 units, 2^32), which keeps P <= 2^32 while skipping
 //     the O correction (a tcgen05.ld/st of the row of O on the softmax's critical path) on all
@@ -37,9 +45,11 @@
 //     compute_block_scores: score = dot * scale + mask) to the row of S in registers, as
 //     mask / scale on the unscaled dot products, before the row max.
 //
-// TMEM columns (512 allocated): S0 [0,128) S1 [128,256) O0, O1 (D each) after them; P_t overwrites
-// the first 64 columns of S_t (S_t is fully in registers by then, and the next S_t MMA is issued
-// after PV_t, which reads P_t first).
+// TMEM columns (512 allocated): tile t keeps S_t at [256t, 256t+128) and O_t after it (D columns,
+// or 80 at D=64 with the ones block).  P_t (bf16 pairs, 64 columns) overwrites the first 64
+// columns of S_t (D=128: S_t is fully in registers by then, and the next S_t MMA follows PV_t);
+// at D=64 without RoPE its keys [64, 128) go to the 32 columns after O_t instead; with RoPE
+// (EARLY) P_t has [256t+192, 256t+256) of its own.  TcCfg below has the exact offsets.
 #pragma once
 
 #include "common.cuh"
