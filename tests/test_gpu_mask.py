@@ -23,6 +23,10 @@ CASES = [
     (P("rows_all_inf", "bf16", 1, 2, 2, 90, 90, 64, False, 0.125, seed=405), "dead_rows"),
     (P("fp32_shared", "fp32", 1, 2, 2, 100, 120, 64, True, 0.125, seed=406), "shared"),
     (P("padded_d40", "bf16", 1, 4, 4, 110, 110, 40, True, 0.158, seed=407), "per_batch"),
+    # more query tiles than SMs: two query tiles per CTA (row tiles of one head, or two heads of a
+    # GQA pair), the mask boxes loaded by TMA (Skv a multiple of 4)
+    (P("two_tile_shared_causal", "bf16", 2, 8, 8, 1300, 1300, 64, True, 0.125, seed=409), "shared"),
+    (P("two_tile_per_head_gqa", "bf16", 1, 16, 8, 1200, 1240, 64, False, 0.125, seed=410), "per_head"),
 ]
 
 
