@@ -82,6 +82,26 @@ bool make_tmap_bshd(CUtensorMap* m, const void* ptr, int B, int S, int H, int D)
     return make_tmap_bshd_rows(m, ptr, B, S, H, D, 128);
 }
 
+// Additive fp32 mask viewed as [Bm][Hm][Sq][Skv] (Bm = 1 or Hm = 1 where the strides broadcast)
+// for TMA loads of 32-key x 128-row boxes with the 128-byte swizzle.  Returns false, with no
+// error recorded, when the encoder refuses the view (the caller then reads the mask per row).
+bool make_tmap_mask(CUtensorMap* m, const float* ptr, int B, int Hq, int Sq, int Skv, long bs, long hs) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t row = static_cast<cuuint64_t>(Skv) * 4;
+    const cuuint64_t plane = row * static_cast<cuuint64_t>(Sq);
+    const cuuint64_t hstride = hs ? static_cast<cuuint64_t>(hs) * 4 : plane;
+    const cuuint64_t Hm = hs ? Hq : 1, Bm = bs ? B : 1;
+    const cuuint64_t bstride = bs ? static_cast<cuuint64_t>(bs) * 4 : hstride * Hm;
+    cuuint64_t dims[4] = {(cuuint64_t)Skv, (cuuint64_t)Sq, Hm, Bm};
+    cuuint64_t strides[3] = {row, hstride, bstride};
+    cuuint32_t box[4] = {32, 128, 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(ptr), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Output [B][S][H][D] (fp32 or bf16) for TMA stores of 32-column x 128-row boxes: 128-byte rows
 // with the 128-byte swizzle (fp32) or 64-byte rows with the 64-byte swizzle (bf16).
 bool make_tmap_out(CUtensorMap* m, void* ptr, int B, int S, int H, int D, bool f32) {
@@ -338,13 +358,19 @@ attn_status launch_tc(const void* q, const void* k, const void* klo, const void*
             if (!ok) return ATTN_ERR_CUDA;
         }
     }
-    const int smem_bytes = TcCfg<D, ROPE>::SMEM_BYTES;
+    // Masked D=64 without RoPE: the mask arrives by TMA when its rows are 16-byte aligned (the
+    // kernel's smem holds the boxes either way; otherwise its threads read the mask per row).
+    CUtensorMap tmk = tq;
+    if constexpr (TcCfg<D, ROPE, true>::MASK_TMA)
+        p.mask_tma = mk.ptr != nullptr && p.mask_vec4 &&
+                     make_tmap_mask(&tmk, mk.ptr, B, Hq, Sq, Skv, mk.bs, mk.hs) ? 1 : 0;
+    const int smem_bytes = mk.ptr != nullptr ? TcCfg<D, ROPE, true>::SMEM_BYTES : TcCfg<D, ROPE, false>::SMEM_BYTES;
     // The warpgroups re-split the launch's registers with setmaxnreg; a launch that holds fewer
     // than the split asks for would stall in setmaxnreg.inc, so such a build is refused.
     attn_status ps = prepare_kernel(reinterpret_cast<const void*>(kern), smem_bytes, "prefill_tc_kernel set-up",
                                     kTcLaunchRegsMin);
     if (ps != ATTN_OK) return ps;
-    kern<<<static_cast<unsigned>(grid), kTcThreads, smem_bytes, st>>>(tq, tk, tkl, tv, to, p);
+    kern<<<static_cast<unsigned>(grid), kTcThreads, smem_bytes, st>>>(tq, tk, tkl, tv, to, tmk, p);
     attn_status s = launch_status("prefill_tc_kernel");
     if (s != ATTN_OK || p.kv_splits == 1) return s;
     // merge of the key splits, a programmatic dependent launch (it waits for the split grid)

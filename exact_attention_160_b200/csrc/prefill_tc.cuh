@@ -75,15 +75,22 @@ constexpr int kRopeNone = 0, kRopeKSplit = 1, kRopeKFused = 2;
 constexpr uint32_t kTcBarTurn0 = 1, kTcBarTurn1 = 2, kTcBarMerge = 3, kTcBarGroup0 = 4;
 constexpr float kLn2 = 0.69314718055994531f;
 
-template <int D, int ROPE>
+template <int D, int ROPE, bool MASK = false>
 struct TcCfg {
     static constexpr int BM = 128;                    // query rows per tile
     static constexpr int BN = 128;                    // keys per KV tile
     static constexpr int NBOX = D / 64;               // 128-byte-wide TMA boxes per row
     static constexpr int TILE_BYTES = BN * D * 2;     // one 128 x D bf16 tile
     static constexpr int KSTEPS = D / 16;             // MMA K steps of S = Q K^T
+    // Masked D=64 without RoPE (MASK_TMA): the additive mask reaches shared memory by TMA in
+    // 32-key x 128-row fp32 boxes (16 KB, 128-byte swizzle), MASK_SLOTS per query tile; the K/V
+    // ring gives up a stage for them.
+    static constexpr bool MASK_TMA = MASK && D == 64 && ROPE == 0;
+    static constexpr int MASK_SLOTS = MASK_TMA ? 2 : 0;
+    static constexpr int MASK_BOX_BYTES = 128 * 32 * 4;
+    static constexpr int MASK_BYTES = 2 * MASK_SLOTS * MASK_BOX_BYTES;
     // D=128 with RoPE holds four Q tiles (hi, lo for both query tiles): one K/V stage fits.
-    static constexpr int STAGES = (D == 64) ? (ROPE ? 3 : 4) : (ROPE ? 1 : 2);
+    static constexpr int STAGES = (D == 64) ? (ROPE ? 3 : (MASK_TMA ? 3 : 4)) : (ROPE ? 1 : 2);
     static constexpr int K_TILES = ROPE ? 2 : 1;      // Kh, Kl
     static constexpr int Q_TILES = ROPE ? 2 : 1;      // Qh, Ql
     static constexpr int STAGE_BYTES = (K_TILES + 1) * TILE_BYTES;
@@ -103,9 +110,9 @@ struct TcCfg {
     static constexpr bool ONES = (D == 64 && !EARLY);
     static constexpr int N_PV = ONES ? D + 16 : D;
     static constexpr int ONES_BYTES = ONES ? 128 * 128 : 0;
-    static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES + ONES_BYTES;
+    static constexpr int SMEM_DATA = Q_BYTES + STAGES * STAGE_BYTES + ONES_BYTES + MASK_BYTES;
     static constexpr int SMEM_BYTES = SMEM_DATA + 1024 /* alignment slack */ + 512 /* barriers */;
-    static_assert(8 * (16 + 5 * STAGES) + 4 <= 512, "barrier area");
+    static_assert(8 * (16 + 5 * STAGES + 4 * MASK_SLOTS) + 4 <= 512, "barrier area");
     // TMEM columns: each query tile keeps S_t and O_t in one half of the 512 columns, S_t first;
     // P_t (bf16, 64 columns) is written over the first half of S_t once the softmax holds S_t in
     // registers.  (A P·V product whose A operand and accumulator lie in different halves ran
@@ -140,6 +147,7 @@ struct TcParams {
     long mask_bs, mask_hs;    // its batch and head strides (elements; 0 broadcasts); rows of Skv
     float inv_scale;          // 1 / scale: the mask enters the raw scores as mask / scale
     int mask_vec4;            // 1: every mask row starts 16-byte aligned (base, strides, Skv multiples of 4)
+    int mask_tma;             // 1 (MASK_TMA kernels): the mask arrives by TMA through tm_m
     int kv_splits;            // >= 1; > 1 (single-tile mode only): each query tile's key tiles are
                               // divided among this many CTAs, which write partials
     float* o_part;            // [kv_splits][B][Sq][Hq][D] fp32 partial O, normalised per split
@@ -169,13 +177,14 @@ template <int D, int ROPE, bool MASK, bool ILV>
 __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
-    const __grid_constant__ CUtensorMap tm_o, const TcParams p) {
-    using C = TcCfg<D, ROPE>;
+    const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ CUtensorMap tm_m, const TcParams p) {
+    using C = TcCfg<D, ROPE, MASK>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = smem;                                   // [2][Q_TILES][TILE_BYTES]
     uint8_t* sKV = smem + C::Q_BYTES;                     // [STAGES][(K_TILES+1)][TILE_BYTES]
     uint8_t* sOnes = sKV + C::STAGES * C::STAGE_BYTES;    // [128 keys][64] bf16 ones (ONES only)
+    uint8_t* sMask = sOnes + C::ONES_BYTES;                // MASK_TMA: [2 tiles][MASK_SLOTS] 16 KB boxes
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::SMEM_DATA);
     uint64_t* bar_q_full = bars + 0;
     uint64_t* bar_q_ready = bars + 1;
@@ -189,7 +198,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
     uint64_t* bar_k_rot = bar_kv_empty + 2 * C::STAGES;   // [STAGES] K(j) rotated in place (kRopeKFused)
     uint64_t* bar_s_free = bar_k_rot + C::STAGES;     // [2] EARLY: softmax t holds S_t(j) in registers
     uint64_t* bar_pv_done = bar_s_free + 2;           // [2] EARLY: PV_t(j) completed (P_t free, O_t at rest)
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_pv_done + 2);
+    uint64_t* bar_m_full = bar_pv_done + 2;           // MASK_TMA: [2 tiles][MASK_SLOTS] mask box landed
+    uint64_t* bar_m_empty = bar_m_full + 2 * C::MASK_SLOTS;   // [2 tiles][MASK_SLOTS] its softmax read it
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_m_empty + 2 * C::MASK_SLOTS);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
@@ -319,6 +330,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
         for (int i = 0; i < 2; ++i) {
             mbar_init(bar_s_free + i, 128);
             mbar_init(bar_pv_done + i, 1);
+        }
+        for (int i = 0; i < 2 * C::MASK_SLOTS; ++i) {
+            mbar_init(bar_m_full + i, 1);
+            mbar_init(bar_m_empty + i, 128);   // every thread of the tile's softmax warpgroup
         }
         mbar_fence_init();
         // The copies go out now, while the tensor memory is allocated and the block synchronises
@@ -651,6 +666,40 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             mma_commit(bar_mma_final);
             mbar_wait(bar_mma_final, 0);
         }
+      } else if (C::MASK_SLOTS > 0 && (warp == 2 || warp == 3)) {
+        // =============================== mask producers (MASK_TMA) ========================
+        // Warp 2 loads the mask of query tile 0, warp 3 that of tile 1: per key tile of the
+        // query tile, four 32-key x 128-row fp32 boxes in key order through the tile's
+        // MASK_SLOTS slots (rows past Sq and keys past Skv arrive as zeros).  The mask is viewed
+        // as [Bm][Hm][Sq][Skv] with Bm or Hm = 1 where it broadcasts.
+        if constexpr (C::MASK_SLOTS > 0) if (lane == 0 && p.mask_tma) {
+            const int t = warp - 2;
+            const bool act = t ? tile[1].active : tile[0].active;
+            const int nt = t ? tile[1].nkv : tile[0].nkv;
+            const int r0 = t ? tile[1].r0 : tile[0].r0;
+            const int hm = p.mask_hs ? (t ? tile[1].h : tile[0].h) : 0;
+            const int bm = p.mask_bs ? b : 0;
+            uint64_t* mfull = bar_m_full + t * C::MASK_SLOTS;
+            uint64_t* mempty = bar_m_empty + t * C::MASK_SLOTS;
+            uint8_t* mbase = sMask + t * C::MASK_SLOTS * C::MASK_BOX_BYTES;
+            const uint64_t pol = l2_policy_evict_last();   // the mask is shared by every head it broadcasts to
+            int issued = 0;
+            bool okm = act;
+            for (int j = 0; okm && j < nt; ++j) {
+                const int k0 = (kv0 + ring_of(t, j)) * 128;
+                for (int c = 0; c < 4; ++c) {
+                    const int u = 4 * j + c, sl = u % C::MASK_SLOTS;
+                    okm = mbar_wait(mempty + sl, ((u / C::MASK_SLOTS) & 1) ^ 1);
+                    if (!okm) break;
+                    mbar_arrive_expect_tx(mfull + sl, C::MASK_BOX_BYTES);
+                    tma_load_4d(&tm_m, mfull + sl, mbase + sl * C::MASK_BOX_BYTES, k0 + 32 * c, r0, hm, bm, pol);
+                    issued = u + 1;
+                }
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int u = issued - C::MASK_SLOTS > 0 ? issued - C::MASK_SLOTS : 0; u < issued; ++u)
+                mbar_wait(mfull + u % C::MASK_SLOTS, (u / C::MASK_SLOTS) & 1);
+        }
       } else if (ROPE == kRopeKFused) {
         // =============================== K rotation (warps 2, 3) ========================
         // Each K tile is rotated in place as soon as it lands: key r of the tile (position
@@ -957,7 +1006,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) prefill_tc_kernel(
             for (int cb = 0; cb < 4; ++cb) tmem_ld32(tS + cb * 32, sr[cb]);
             tmem_wait_ld();
             const int k0 = (kv0 + ring_of(wg, j)) * 128;
-            if (MASK && qrow < p.Sq) {
+            if (C::MASK_SLOTS > 0 && p.mask_tma) {
+                // additive mask from the tile's slots: box c holds keys [32c, 32c+32) of all 128
+                // rows, 16-byte chunk e of row r at chunk e ^ (r & 7) (the load's 128-byte
+                // swizzle), so the row-per-thread reads are free of bank conflicts; S holds q.k
+                // unscaled, so the mask enters as mask / scale
+                const uint8_t* mrow = sMask + wg * C::MASK_SLOTS * C::MASK_BOX_BYTES + row * 128;
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    constexpr int MS = C::MASK_SLOTS > 0 ? C::MASK_SLOTS : 1;   // (kernels without the ring never get here)
+                    const int u = 4 * j + cb, sl = u % MS;
+                    if (ok && !__all_sync(0xffffffffu, mbar_wait(bar_m_full + wg * C::MASK_SLOTS + sl, (u / MS) & 1)))
+                        ok = false;
+                    const uint8_t* mb = mrow + sl * C::MASK_BOX_BYTES;
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const float4 m4 = *reinterpret_cast<const float4*>(mb + ((e4 ^ (row & 7)) << 4));
+                        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4)
+                            sr[cb][4 * e4 + q4] = __float_as_uint(__uint_as_float(sr[cb][4 * e4 + q4]) + mm[q4] * p.inv_scale);
+                    }
+                    // the slot may be refilled: this thread's generic-proxy reads of it are ordered
+                    // before the next TMA (async-proxy) write into it
+                    fence_proxy_async_smem();
+                    mbar_arrive(bar_m_empty + wg * C::MASK_SLOTS + sl);
+                }
+            } else if (MASK && qrow < p.Sq) {
                 // additive mask: S holds q.k unscaled, so add mask / scale; the exponent
                 // (s * scale + mask) * log2(e) - m then keeps its form
                 const float* mrow = p.mask + b * p.mask_bs + T.h * p.mask_hs + static_cast<long>(qrow) * p.Skv + k0;
