@@ -135,7 +135,9 @@ attn_status attn_fwd_ex(const void* q, const void* k, const void* v, void* o, fl
  *   for one [Sq, Skv] mask shared by every batch and head), 4-byte aligned, read on the device.
  *   -inf entries remove keys; a row whose scores are all -inf gets o = 0, lse = -inf.  Other
  *   arguments, workspace and errors as attn_fwd_ex (attn_fwd_ex_workspace_size gives the bytes).
- *   The mask is read with plain loads per row (it is a generality path: no TMA staging).
+ *   At D = 64 without RoPE, with every mask row 16-byte aligned (base, strides and Skv multiples
+ *   of 4 elements), the mask is staged into shared memory by TMA; otherwise each thread reads
+ *   its mask row with plain loads.
  */
 attn_status attn_fwd_masked(const void* q, const void* k, const void* v, const float* mask, int64_t mask_batch_stride,
                             int64_t mask_head_stride, void* o, float* lse, int B, int Hq, int Hkv, int Sq, int Skv,
