@@ -43,7 +43,9 @@
 //     pre-rotated; both carry hi + lo bf16 halves and S = Qh Kh^T + Qh Kl^T + Ql Kh^T.
 //   * MASK instantiations add an additive score mask (whisper-apr attention_generated.rs,
 //     compute_block_scores: score = dot * scale + mask) to the row of S in registers, as
-//     mask / scale on the unscaled dot products, before the row max.
+//     mask / scale on the unscaled dot products, before the row max.  At D=64 without RoPE the
+//     mask reaches shared memory by TMA (warps 2 and 3, swizzled boxes read conflict-free);
+//     otherwise each thread loads its row from global memory.
 //
 // TMEM columns (512 allocated): tile t keeps S_t at [256t, 256t+128) and O_t after it (D columns,
 // or 80 at D=64 with the ones block).  P_t (bf16 pairs, 64 columns) overwrites the first 64
