@@ -70,6 +70,22 @@ def test_fwd_ex_validation(lib):
     assert lib.attn_fwd_ex(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0.1, 1, 0, 10000.0, -1, P, need, None) == 1
 
 
+def test_fwd_masked_validation(lib):
+    """attn_fwd_masked rejects a missing or misaligned mask and negative strides, and applies the
+    forward's own checks, before any launch."""
+    P = FAKE
+
+    def call(mask=P, bs=0, hs=0, B=1, Hq=2, Hkv=2):
+        return lib.attn_fwd_masked(P, P, P, mask, bs, hs, P, None, B, Hq, Hkv, 8, 8, 64, 0.125, 0, 0, 0.0, 0,
+                                   None, 0, None)
+    assert call(mask=None) == 1
+    assert call(mask=ctypes.c_void_p((1 << 20) + 2)) == 1     # not 4-byte aligned
+    assert call(bs=-1) == 1
+    assert call(hs=-64) == 1
+    assert call(B=0) == 1
+    assert call(Hq=3, Hkv=2) == 2
+
+
 def test_fwd_key_split_sizing(lib):
     """Key splits: n = min(148 // tiles, ceil(Skv/128) // 2, 16) for bf16 problems of <= 74 query
     tiles, taken when they spare the longest chunk >= 8 key tiles; their partials (splits x rows x
